@@ -1,0 +1,320 @@
+"""Plain fp64 CPU oracle of VMoBA per-layer sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  This module defines what the CUDA library must
+compute, step by step and in float64, so that the kernels can be checked
+against it.  Only the test suite, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import it; the library itself never does
+and shares no code with it.
+
+Sources (VMoBA: Mixture-of-Block Attention for Video Diffusion Models):
+
+* [notes] papernotes.org ICLR 2026 notes, section "Method / overall
+  framework" and "Key designs" 1-3 (the only page with the formulas);
+* [digest] paperlayer.ai section digest of arXiv 2506.23858, sections
+  3.1-3.4.
+
+Every function below names the passage it follows.  Where the pages leave a
+step open, the reading taken is stated in the function's docstring:
+
+1. "Normalised similarity" (notes, key design 3; digest 3.4) is read as a
+   softmax over the head's whole s x N_b pool of scores S = scale * q . b,
+   scale = 1/sqrt(head_dim).  Every term is >= 0, the total is 1 so tau is
+   the fraction of similarity mass kept, and the order equals the order of S.
+2. The stopping rule uses ">=" (the printed formula), not "exceeds".
+3. Ties in the ranking are broken by (query index asc, block index asc).
+4. tau at or above the pool's total mass selects every pair.
+5. A query row with no selected block gets O = 0, LSE = -inf, dQ = 0.
+6. K and V are permuted together; Q and the output keep the original order.
+7. Blocks are numbered row-major over the (T/bt, H/bh, W/bw) grid and
+   tokens inside a block are in (t, y, x) order.
+8. The selection mask is a constant for the backward pass (no gradient
+   flows through the pooled blocks or the threshold).
+
+Pins (what ties each function to something other than itself) are in
+``tests/test_oracle_pins.py``; each function's docstring lists them.
+
+Array conventions: Q, K, V, O, dO, dQ, dK, dV are ``[s][n_heads][d]``
+float64 in original token order ``t*H*W + y*W + x``.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+MODES = {0: "1D", 1: "2D", 2: "3D"}
+
+
+# --------------------------------------------------------------------------
+# Partition (notes, key design 1: layer-wise recurrent 1D-2D-3D partition)
+# --------------------------------------------------------------------------
+
+def mode_for_layer(layer: int) -> int:
+    """Partition mode of layer l: l mod 3 = 0 -> 1D, 1 -> 2D, 2 -> 3D.
+
+    [notes] key design 1; [digest] 3.2.  Pinned: tests check the cycle.
+    """
+    if layer < 0:
+        raise ValueError("layer index must be >= 0")
+    return layer % 3
+
+
+def mode_box(mode: int, T: int, H: int, W: int, bt: int, bh: int, bw: int) -> tuple:
+    """Block box of a mode.
+
+    [notes] key design 1: 1D groups tokens of adjacent frames (box bt x H x W);
+    2D groups tokens of one spatial region across all frames (T x bh x bw);
+    3D cuts local spatio-temporal patches (bt x bh x bw).
+    """
+    if mode == 0:
+        return (bt, H, W)
+    if mode == 1:
+        return (T, bh, bw)
+    if mode == 2:
+        return (bt, bh, bw)
+    raise ValueError(f"mode must be 0, 1 or 2, got {mode}")
+
+
+def check_box(T: int, H: int, W: int, box: tuple) -> None:
+    bt, bh, bw = box
+    if min(bt, bh, bw) < 1 or T % bt or H % bh or W % bw:
+        raise ValueError(f"box {box} does not divide the latent {(T, H, W)}")
+
+
+def partition_order(T: int, H: int, W: int, box: tuple) -> np.ndarray:
+    """Key permutation of the partition: K'[p] = K[perm[p]].
+
+    [notes] key design 1 writes the partition as a rearrange of K in (T H W)
+    order; read here as (pt bt)(ph bh)(pw bw) -> (pt ph pw)(bt bh bw), i.e.
+    blocks row-major over the box grid, (t, y, x) order inside a block.
+    Pinned: brute-force coordinate enumeration; 3D boxes that equal a 1D or
+    2D box give the same partition; every block holds one box of tokens.
+    """
+    check_box(T, H, W, box)
+    bt, bh, bw = box
+    idx = np.arange(T * H * W).reshape(T // bt, bt, H // bh, bh, W // bw, bw)
+    return idx.transpose(0, 2, 4, 1, 3, 5).reshape(-1).copy()
+
+
+def block_of_token(T: int, H: int, W: int, box: tuple) -> np.ndarray:
+    """Block index of every original token (inverse view of partition_order)."""
+    perm = partition_order(T, H, W, box)
+    L = box[0] * box[1] * box[2]
+    blk = np.empty(T * H * W, dtype=np.int64)
+    blk[perm] = np.arange(perm.size) // L
+    return blk
+
+
+def permute_keys(K: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """K' = rearranged K, returned as [n_heads][s][d] (block-contiguous)."""
+    return np.ascontiguousarray(K[perm].transpose(1, 0, 2))
+
+
+def pool_blocks(K: np.ndarray, T: int, H: int, W: int, box: tuple) -> np.ndarray:
+    """Block tensor B = mean(K') per block, [n_heads][N_b][d].
+
+    [notes] key design 1: B = mean(K') over each block of the rearranged keys.
+    Pinned: brute-force coordinate sums; constant keys give B = K; the mean
+    of the block means equals the mean of all keys.
+    """
+    perm = partition_order(T, H, W, box)
+    L = box[0] * box[1] * box[2]
+    Kp = permute_keys(K, perm)
+    n_h, s, d = Kp.shape
+    return Kp.reshape(n_h, s // L, L, d).mean(axis=2)
+
+
+# --------------------------------------------------------------------------
+# Scores (notes, key design 2: global block selection, S = q_i b_i^T)
+# --------------------------------------------------------------------------
+
+def block_scores(Q: np.ndarray, B: np.ndarray, scale: float) -> np.ndarray:
+    """Pool of head i: S_i = scale * q_i b_i^T, returned as [n_heads][s][N_b].
+
+    [notes] key design 2 (M_i = TopkMask(q_i b_i^T, k)) and key design 3
+    (S^ = q_i b_i^T); the 1/sqrt(d) temperature is reading 1.
+    Pinned: equals the block-average of the token-level logits (linearity of
+    the mean), computed from the full logit matrix.
+    """
+    Qh = Q.transpose(1, 0, 2)                      # [n_h][s][d]
+    return scale * np.matmul(Qh, B.transpose(0, 2, 1))
+
+
+# --------------------------------------------------------------------------
+# Threshold selection (notes, key design 3; digest 3.3 and 3.4)
+# --------------------------------------------------------------------------
+
+def normalised_pool(S_h: np.ndarray) -> np.ndarray:
+    """p = exp(S - max S) / sum exp(S - max S) over the head's whole pool (reading 1)."""
+    e = np.exp(S_h - S_h.max())
+    return e / e.sum()
+
+
+def threshold_select(S_h: np.ndarray, tau: float):
+    """Global threshold selection for one head.
+
+    [notes] key design 3: sort the global pool descending and take
+    k = min{k' : sum_{j<=k'} Sorted(S^)_j >= tau} over normalised similarity;
+    [digest] 3.4 says the same in words.  Ties: (query asc, block asc).
+
+    Returns (mask [s][N_b] bool, stats) with stats = dict(k, cut_score, mass)
+    where mass is the cumulative normalised mass of the k selected pairs.
+    Pinned: minimality (c_k >= tau > c_{k-1}), density bound
+    k/(s N_b) < tau + 1/(s N_b), monotonicity in tau, brute-force subset
+    enumeration on tiny pools, and the selected set scoring at least as high
+    as every unselected pair.
+    """
+    if not (tau > 0.0) or math.isnan(tau):
+        raise ValueError("tau must be > 0")
+    flat = S_h.reshape(-1)
+    p = normalised_pool(S_h).reshape(-1)
+    order = np.argsort(-flat, kind="stable")       # descending, ties by flat index
+    c = np.cumsum(p[order])
+    reached = np.flatnonzero(c >= tau)
+    k = int(reached[0]) + 1 if reached.size else flat.size
+    mask = np.zeros(flat.size, dtype=bool)
+    mask[order[:k]] = True
+    stats = dict(k=k, cut_score=float(flat[order[k - 1]]), mass=float(c[k - 1]))
+    return mask.reshape(S_h.shape), stats
+
+
+def select_all_heads(S: np.ndarray, tau: float):
+    """threshold_select for every head: mask [n_heads][s][N_b], list of stats."""
+    masks, stats = [], []
+    for h in range(S.shape[0]):
+        m, st = threshold_select(S[h], tau)
+        masks.append(m)
+        stats.append(st)
+    return np.stack(masks), stats
+
+
+# --------------------------------------------------------------------------
+# Sparse attention over the selected pairs (notes, overall framework:
+# "attention only on the selected blocks, same shape as full attention")
+# --------------------------------------------------------------------------
+
+def allowed_keys(sel_h: np.ndarray, blk: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """Token-level mask [len(rows)][s]: key n allowed for row i iff block(n) is selected."""
+    return sel_h[rows][:, blk]
+
+
+def attention_fwd_rows(Qh, Kh, Vh, sel_h, blk, scale, rows):
+    """Forward of the masked softmax attention for the given query rows of one head.
+
+    Definition (reading 5 for empty rows): a_in = scale q_i.k_n over keys whose
+    block is selected for row i; LSE_i = log sum exp a_in; O_i = softmax(a_i) V.
+    Pinned: tau = 1 equals torch's scaled_dot_product_attention in fp64; any
+    mask equals SDPA with the same boolean mask on non-empty rows.
+    Returns O [len(rows)][d], LSE [len(rows)].
+    """
+    A = scale * (Qh[rows] @ Kh.T)
+    allow = allowed_keys(sel_h, blk, rows)
+    A = np.where(allow, A, -np.inf)
+    has = allow.any(axis=1)
+    m = np.where(has, A.max(axis=1), 0.0)
+    P = np.exp(A - m[:, None])                      # exp(-inf) = 0 on masked keys
+    l = P.sum(axis=1)
+    O = np.zeros((len(rows), Vh.shape[1]))
+    O[has] = (P[has] @ Vh) / l[has, None]
+    lse = np.full(len(rows), -np.inf)
+    lse[has] = m[has] + np.log(l[has])
+    return O, lse
+
+
+def attention_bwd_rows(Qh, Kh, Vh, sel_h, blk, scale, rows, dOh_rows):
+    """Backward for a chunk of query rows of one head, mask held constant (reading 8).
+
+    With P the masked softmax, D_i = dO_i . O_i, dP = dO V^T,
+    dS = P * (dP - D), the chunk contributes dQ_rows = scale dS K,
+    dK += scale dS^T Q_rows, dV += P^T dO_rows.
+    Pinned: central finite differences of sum(dO * O) in fp64 and torch
+    autograd through SDPA with the same boolean mask.
+    Returns (dQ_rows, dK_part, dV_part).
+    """
+    A = scale * (Qh[rows] @ Kh.T)
+    allow = allowed_keys(sel_h, blk, rows)
+    A = np.where(allow, A, -np.inf)
+    has = allow.any(axis=1)
+    m = np.where(has, A.max(axis=1), 0.0)
+    P = np.exp(A - m[:, None])
+    l = P.sum(axis=1)
+    P[has] /= l[has, None]
+    P[~has] = 0.0
+    O = P @ Vh
+    D = np.sum(dOh_rows * O, axis=1)
+    dP = dOh_rows @ Vh.T
+    dS = P * (dP - D[:, None])
+    dQ = scale * (dS @ Kh)
+    dK = scale * (dS.T @ Qh[rows])
+    dV = P.T @ dOh_rows
+    return dQ, dK, dV
+
+
+def _row_chunks(s: int, chunk: int):
+    for r0 in range(0, s, chunk):
+        yield np.arange(r0, min(s, r0 + chunk))
+
+
+def attention_fwd(Q, K, V, sel, blk, scale, chunk: int = 1024):
+    """Masked attention forward for all heads: O [s][n_h][d], LSE [n_h][s]."""
+    s, n_h, d = Q.shape
+    O = np.zeros_like(Q)
+    lse = np.zeros((n_h, s))
+    for h in range(n_h):
+        for rows in _row_chunks(s, chunk):
+            o, l_ = attention_fwd_rows(Q[:, h], K[:, h], V[:, h], sel[h], blk, scale, rows)
+            O[rows, h] = o
+            lse[h, rows] = l_
+    return O, lse
+
+
+def attention_bwd(Q, K, V, sel, blk, scale, dO, chunk: int = 1024):
+    """Masked attention backward for all heads: dQ, dK, dV in [s][n_h][d]."""
+    s, n_h, d = Q.shape
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for h in range(n_h):
+        for rows in _row_chunks(s, chunk):
+            dq, dk, dv = attention_bwd_rows(Q[:, h], K[:, h], V[:, h], sel[h], blk,
+                                            scale, rows, dO[rows, h])
+            dQ[rows, h] = dq
+            dK[:, h] += dk
+            dV[:, h] += dv
+    return dQ, dK, dV
+
+
+# --------------------------------------------------------------------------
+# The whole layer (notes, overall framework flowchart; digest 3.1)
+# --------------------------------------------------------------------------
+
+def vmoba_layer(Q, K, V, T, H, W, mode, box_cfg, tau, scale=None, dO=None,
+                chunk: int = 1024):
+    """Partition -> pool -> scores -> global threshold selection -> attention.
+
+    ``box_cfg`` is (bt, bh, bw); ``mode`` picks which of its axes apply
+    (mode_box).  Returns a dict with perm, blk, B, S, sel, stats, O, LSE and,
+    when dO is given, dQ, dK, dV.
+    """
+    s, n_h, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    box = mode_box(mode, T, H, W, *box_cfg)
+    perm = partition_order(T, H, W, box)
+    blk = block_of_token(T, H, W, box)
+    B = pool_blocks(K, T, H, W, box)
+    S = block_scores(Q, B, scale)
+    sel, stats = select_all_heads(S, tau)
+    O, lse = attention_fwd(Q, K, V, sel, blk, scale, chunk)
+    out = dict(box=box, perm=perm, blk=blk, B=B, S=S, sel=sel, stats=stats,
+               O=O, LSE=lse, scale=scale)
+    if dO is not None:
+        dQ, dK, dV = attention_bwd(Q, K, V, sel, blk, scale, dO, chunk)
+        out.update(dQ=dQ, dK=dK, dV=dV)
+    return out
+
+
+def selected_pair_density(sel_h: np.ndarray, L: int) -> float:
+    """Fraction of query-key token pairs attended in one head (the pages' "sparsity")."""
+    s = sel_h.shape[0]
+    return float(sel_h.sum()) * L / (s * s)

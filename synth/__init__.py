@@ -1,0 +1,16 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests/bench and the CPU oracle.
+
+This package holds input generation and workload tables only: no step of the
+attention method (no partition, pooling, scoring, selection or attention
+arithmetic) lives here.
+"""
+from .video_latents import (  # noqa: F401
+    splitmix64_stream,
+    uniform01,
+    standard_normal,
+    smooth_fields,
+    make_qkv,
+    make_dout,
+    seed_for,
+)
+from .workloads import WORKLOADS, Workload  # noqa: F401

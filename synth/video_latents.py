@@ -1,0 +1,207 @@
+"""Deterministic video-latent-shaped Q/K/V/dO generators.
+
+The real inputs of the method are projections of Wan-2.1 latents of
+Koala-36M clips (VMoBA, page 2 section 4.1), which are not available here.
+These generators stand in for them with the shapes of the pages' workloads
+and a spatio-temporally smooth component, so that block means carry signal
+the way they do in a trained video DiT.
+
+Recipe (all on the host, fp64, reproducible bit for bit on any machine):
+
+* Random bits: a counter-based splitmix64 stream.  Element ``n`` of the
+  stream with seed ``S`` is ``mix64(S + (n + 1) * 0x9E3779B97F4A7C15)``
+  (Steele, Lea, Flood, "Fast splittable pseudorandom number generators",
+  OOPSLA 2014).
+* Uniforms in (0, 1]: ``((z >> 11) + 1) * 2**-53``.
+* Normals: Box-Muller on consecutive uniform pairs (u1, u2):
+  ``sqrt(-2 ln u1) * cos(2 pi u2)``.
+* Smooth fields: ``r`` i.i.d. N(0,1) scalar fields on the (T, H, W) grid,
+  separable Gaussian blur with sigma = (1, 2, 2) tokens in (t, h, w),
+  clamp-to-edge, kernel radius ceil(3 sigma), each field rescaled to unit
+  variance.
+* Q/K per head h: ``W_Q,h ~ N(0, 1/r)^{r x d}``,
+  ``W_K,h = W_Q,h + 0.5 N(0, 1/r)``; ``X = (F W_X + 0.5 eps) / sqrt(1.25)``
+  with eps ~ N(0, 1); Q and K share the fields F.  V uses its own fields
+  and its own W_V ~ N(0, 1/r).  An optional per-head gain c_h ~ U[0.5, 2]
+  multiplies Q and K of head h.
+* The i.i.d. variant draws every element of Q, K, V from N(0, 1).
+
+Layout of every returned tensor: ``[s][n_heads][head_dim]``, token index
+``t*H*W + y*W + x`` (frame-major).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+# tensor ids inside one (workload, layer) seed family
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "dout": 4}
+# sub-stream ids inside one tensor family
+_PART_FIELDS = 1
+_PART_W = 2
+_PART_W_DELTA = 3
+_PART_EPS = 4
+_PART_GAIN = 5
+
+
+def seed_for(workload_id: int, layer: int, tensor: str, part: int = 0) -> int:
+    """Seed of one sub-stream: (workload*1000 + layer*10 + tensor_id) << 8 | part."""
+    base = workload_id * 1000 + layer * 10 + TENSOR_IDS[tensor]
+    return (base << 8) | part
+
+
+def splitmix64_stream(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    """Counter-based splitmix64: element i is mix64(seed + (offset+i+1)*golden)."""
+    z = np.arange(offset + 1, offset + n + 1, dtype=np.uint64)
+    t = np.empty_like(z)
+    with np.errstate(over="ignore"):
+        np.multiply(z, _GOLDEN, out=z)
+        np.add(z, np.uint64(seed & 0xFFFFFFFFFFFFFFFF), out=z)
+        for shift, mul in ((30, _M1), (27, _M2)):
+            np.right_shift(z, np.uint64(shift), out=t)
+            np.bitwise_xor(z, t, out=z)
+            np.multiply(z, mul, out=z)
+        np.right_shift(z, np.uint64(31), out=t)
+        np.bitwise_xor(z, t, out=z)
+    return z
+
+
+def uniform01(seed: int, n: int) -> np.ndarray:
+    """n uniforms in (0, 1] as float64."""
+    z = splitmix64_stream(seed, n)
+    np.right_shift(z, np.uint64(11), out=z)
+    u = z.astype(np.float64)
+    u += 1.0
+    u *= 2.0 ** -53
+    return u
+
+
+def standard_normal(seed: int, n: int) -> np.ndarray:
+    """n N(0,1) float64 draws by Box-Muller on uniform pairs."""
+    u = uniform01(seed, 2 * n).reshape(n, 2)
+    r = np.log(u[:, 0])
+    r *= -2.0
+    np.sqrt(r, out=r)
+    c = u[:, 1] * (2.0 * math.pi)
+    np.cos(c, out=c)
+    r *= c
+    return r
+
+
+def _gauss_kernel(sigma: float) -> np.ndarray:
+    r = int(math.ceil(3.0 * sigma))
+    x = np.arange(-r, r + 1, dtype=np.float64)
+    k = np.exp(-0.5 * (x / sigma) ** 2)
+    return k / k.sum()
+
+
+def _blur_axis(a: np.ndarray, axis: int, sigma: float) -> np.ndarray:
+    if sigma <= 0:
+        return a
+    k = _gauss_kernel(sigma)
+    r = (k.size - 1) // 2
+    n = a.shape[axis]
+    idx = np.clip(np.arange(-r, n + r), 0, n - 1)  # clamp-to-edge
+    padded = np.take(a, idx, axis=axis)
+    out = np.zeros_like(a)
+    for t, w in enumerate(k):
+        sl = [slice(None)] * a.ndim
+        sl[axis] = slice(t, t + n)
+        out += w * padded[tuple(sl)]
+    return out
+
+
+def smooth_fields(T: int, H: int, W: int, r: int, seed: int,
+                  sigma=(1.0, 2.0, 2.0)) -> np.ndarray:
+    """r blurred unit-variance scalar fields on the grid, returned as [s][r] float64."""
+    g = standard_normal(seed, r * T * H * W).reshape(r, T, H, W)
+    g = _blur_axis(g, 1, sigma[0])
+    g = _blur_axis(g, 2, sigma[1])
+    g = _blur_axis(g, 3, sigma[2])
+    g = g.reshape(r, -1)
+    g = (g - g.mean(axis=1, keepdims=True)) / g.std(axis=1, keepdims=True)
+    return np.ascontiguousarray(g.T)
+
+
+def _project(F: np.ndarray, Wx: np.ndarray) -> np.ndarray:
+    """[s][r] fields times per-head [h][r][d] weights -> [s][h][d]."""
+    return np.ascontiguousarray(np.matmul(F[None], Wx).transpose(1, 0, 2))
+
+
+def _iid(seed: int, s: int, n_heads: int, d: int) -> np.ndarray:
+    return standard_normal(seed, s * n_heads * d).reshape(s, n_heads, d)
+
+
+def make_qkv(workload_id: int, layer: int, T: int, H: int, W: int,
+             n_heads: int, head_dim: int, kind: str = "smooth",
+             head_gain: bool = False, rank: int = 8):
+    """Q, K, V as float64 arrays [s][n_heads][head_dim] (see module doc).
+
+    ``kind`` is "iid" or "smooth"; ``head_gain`` draws c_h ~ U[0.5, 2] per head.
+    """
+    s = T * H * W
+    d = head_dim
+    if kind == "iid":
+        return (_iid(seed_for(workload_id, layer, "q", _PART_EPS), s, n_heads, d),
+                _iid(seed_for(workload_id, layer, "k", _PART_EPS), s, n_heads, d),
+                _iid(seed_for(workload_id, layer, "v", _PART_EPS), s, n_heads, d))
+    if kind != "smooth":
+        raise ValueError(f"unknown input kind {kind!r}")
+    sd = math.sqrt(1.0 / rank)
+    F = smooth_fields(T, H, W, rank, seed_for(workload_id, layer, "q", _PART_FIELDS))
+    Wq = standard_normal(seed_for(workload_id, layer, "q", _PART_W),
+                         n_heads * rank * d).reshape(n_heads, rank, d) * sd
+    Wk = Wq + 0.5 * sd * standard_normal(seed_for(workload_id, layer, "k", _PART_W_DELTA),
+                                         n_heads * rank * d).reshape(n_heads, rank, d)
+    Fv = smooth_fields(T, H, W, rank, seed_for(workload_id, layer, "v", _PART_FIELDS))
+    Wv = standard_normal(seed_for(workload_id, layer, "v", _PART_W),
+                         n_heads * rank * d).reshape(n_heads, rank, d) * sd
+    norm = 1.0 / math.sqrt(1.25)
+    q = (_project(F, Wq)
+         + 0.5 * _iid(seed_for(workload_id, layer, "q", _PART_EPS), s, n_heads, d)) * norm
+    k = (_project(F, Wk)
+         + 0.5 * _iid(seed_for(workload_id, layer, "k", _PART_EPS), s, n_heads, d)) * norm
+    v = (_project(Fv, Wv)
+         + 0.5 * _iid(seed_for(workload_id, layer, "v", _PART_EPS), s, n_heads, d)) * norm
+    if head_gain:
+        c = 0.5 + 1.5 * uniform01(seed_for(workload_id, layer, "q", _PART_GAIN), n_heads)
+        q = q * c[None, :, None]
+        k = k * c[None, :, None]
+    return q, k, v
+
+
+def make_dout(workload_id: int, layer: int, s: int, n_heads: int, head_dim: int) -> np.ndarray:
+    """Upstream gradient dO ~ N(0,1), [s][n_heads][head_dim] float64."""
+    return _iid(seed_for(workload_id, layer, "dout", _PART_EPS), s, n_heads, head_dim)
+
+
+def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float64 values to the I/O dtype and return them as float64 again.
+
+    fp32: IEEE round-to-nearest-even.  bf16: round the fp32 value to the upper
+    16 bits with round-to-nearest-even (no NaNs occur in these inputs).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    if dtype == "f32":
+        return x32.astype(np.float64)
+    if dtype != "bf16":
+        raise ValueError(dtype)
+    return bf16_bits_to_f64(f32_to_bf16_bits(x32))
+
+
+def f32_to_bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns (uint16), round-to-nearest-even."""
+    b = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
+    lsb = (b >> np.uint32(16)) & np.uint32(1)
+    with np.errstate(over="ignore"):
+        rounded = b + np.uint32(0x7FFF) + lsb
+    return (rounded >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)

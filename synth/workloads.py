@@ -1,0 +1,54 @@
+"""The five VMoBA layer workloads (shapes, block boxes, thresholds).
+
+Grids follow the pages' video sizes after a 4x temporal / 16x16 spatial latent
+compression (e.g. 93x576x1024 frames -> a 24x36x64 latent), 12 heads of
+head_dim 128 (the Wan 2.1 1.3B attention shape), and block counts near the
+paper's "8-48-72" setting (VMoBA page 1, training strategy).
+
+``boxes[mode]`` is the full (bt, bh, bw) block box of each partition mode,
+stored as plain data: mode 0 = 1D temporal, 1 = 2D spatial, 2 = 3D local.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+
+@dataclass(frozen=True)
+class Workload:
+    wid: int
+    name: str
+    T: int
+    H: int
+    W: int
+    n_heads: int
+    head_dim: int
+    dtype: str                      # "f32" or "bf16" (I/O and storage type)
+    kind: str                       # "iid" or "smooth"
+    boxes: tuple                    # full (bt, bh, bw) for modes 0, 1, 2
+    taus: tuple
+    backward: bool
+    head_gain: bool = False
+    layers: int = 3
+    notes: str = field(default="", compare=False)
+
+    @property
+    def s(self) -> int:
+        return self.T * self.H * self.W
+
+
+WORKLOADS = {
+    1: Workload(1, "tiny-256tok", 4, 8, 8, 2, 64, "f32", "iid",
+                ((1, 8, 8), (4, 4, 4), (2, 4, 4)), (0.5,), False,
+                notes="oracle-scale case, fp32 I/O, forward only"),
+    2: Workload(2, "small-2048tok", 8, 16, 16, 4, 64, "bf16", "smooth",
+                ((1, 16, 16), (8, 4, 4), (2, 4, 4)), (0.25, 0.5, 0.75), True),
+    3: Workload(3, "wan1.3b-32760tok", 21, 30, 52, 12, 128, "bf16", "smooth",
+                ((1, 30, 52), (21, 5, 4), (3, 5, 4)), (0.25,), False,
+                notes="inference setting, forward only"),
+    4: Workload(4, "train-55296tok", 24, 36, 64, 12, 128, "bf16", "smooth",
+                ((1, 36, 64), (24, 6, 8), (4, 6, 8)), (0.25,), True,
+                notes="headline: 93x576x1024 video, batch 1, fwd+bwd"),
+    5: Workload(5, "stack30-75600tok", 21, 45, 80, 12, 128, "bf16", "smooth",
+                ((1, 45, 80), (21, 9, 8), (3, 9, 8)), (0.1, 0.25, 0.5), True,
+                head_gain=True, layers=30, notes="30-layer sweep, mode = layer mod 3"),
+}
