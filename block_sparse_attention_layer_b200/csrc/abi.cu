@@ -1,0 +1,189 @@
+// The extern "C" boundary: argument validation, problem geometry, workspace
+// layout and kernel launches.  Every entry point validates synchronously and
+// launches nothing on invalid input; see include/vmoba.h for the contract.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+using namespace vmoba;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Fills P from the public shape; returns VMOBA_OK or a status.
+int make_prob(const vmoba_shape* sh, Prob* P) {
+  if (!sh) return VMOBA_ERR_ARG;
+  if (sh->dtype != VMOBA_BF16 && sh->dtype != VMOBA_F32) return VMOBA_ERR_DTYPE;
+  if (sh->T < 1 || sh->H < 1 || sh->W < 1 || sh->n_heads < 1 || sh->n_heads > 128)
+    return VMOBA_ERR_SHAPE;
+  if (sh->head_dim != 64 && sh->head_dim != 128) return VMOBA_ERR_SHAPE;
+  if (sh->mode < 0 || sh->mode > 2) return VMOBA_ERR_ARG;
+  int bt, bh, bw;
+  if (sh->mode == 0) { bt = sh->bt; bh = sh->H; bw = sh->W; }
+  else if (sh->mode == 1) { bt = sh->T; bh = sh->bh; bw = sh->bw; }
+  else { bt = sh->bt; bh = sh->bh; bw = sh->bw; }
+  if (bt < 1 || bh < 1 || bw < 1) return VMOBA_ERR_SHAPE;
+  if (sh->T % bt || sh->H % bh || sh->W % bw) return VMOBA_ERR_SHAPE;
+  const long long s = (long long)sh->T * sh->H * sh->W;
+  if (s > (long long)kMaxTiles * kTile) return VMOBA_ERR_SHAPE;
+  Prob p{};
+  p.T = sh->T; p.H = sh->H; p.W = sh->W; p.s = (int)s;
+  p.n_h = sh->n_heads; p.d = sh->head_dim; p.mode = sh->mode; p.dtype = sh->dtype;
+  p.bt = bt; p.bh = bh; p.bw = bw;
+  p.nbt = sh->T / bt; p.nbh = sh->H / bh; p.nbw = sh->W / bw;
+  p.Nb = p.nbt * p.nbh * p.nbw;
+  p.L = bt * bh * bw;
+  if (p.Nb > kMaxBlocks) return VMOBA_ERR_SHAPE;
+  if ((long long)p.s * p.Nb >= (1LL << 31)) return VMOBA_ERR_SHAPE;
+  p.Wb = (p.Nb + 31) / 32;
+  p.n_qt = (p.s + kTile - 1) / kTile;
+  p.Wqt = (p.n_qt + 31) / 32;
+  *P = p;
+  return VMOBA_OK;
+}
+
+int check_ws(const Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = ws_layout(P);
+  if (!ws || ws_bytes < L->total || !aligned16(ws)) return VMOBA_ERR_WORKSPACE;
+  return VMOBA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? VMOBA_OK : VMOBA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int vmoba_mode_for_layer(int layer_idx) { return layer_idx < 0 ? -1 : layer_idx % 3; }
+
+int vmoba_num_blocks(const vmoba_shape* shape) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  return rc == VMOBA_OK ? P.Nb : rc;
+}
+
+size_t vmoba_workspace_size(const vmoba_shape* shape) {
+  Prob P;
+  if (make_prob(shape, &P) != VMOBA_OK) return 0;
+  return ws_layout(P).total;
+}
+
+size_t vmoba_bwd_workspace_size(const vmoba_shape* shape) {
+  Prob P;
+  if (make_prob(shape, &P) != VMOBA_OK) return 0;
+  return align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
+}
+
+int vmoba_partition(const vmoba_shape* shape, const void* k, const void* v, void* k_perm,
+                    void* v_perm, float* blocks, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!k || !v || !k_perm || !v_perm || !blocks) return VMOBA_ERR_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_perm) || !aligned16(v_perm) ||
+      !aligned16(blocks))
+    return VMOBA_ERR_ARG;
+  return cuda_status(launch_partition(P, k, v, k_perm, v_perm, blocks, stream));
+}
+
+int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blocks, float tau,
+                       float scale, uint32_t* sel_bits, vmoba_head_stats* stats, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (!(tau > 0.0f) || std::isnan(tau)) return VMOBA_ERR_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
+  WsLayout L;
+  if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  // tau at or above the whole pool keeps every pair; 2 can never be reached
+  const float tau_dev = tau >= 1.0f ? 2.0f : tau;
+  return cuda_status(
+      launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
+}
+
+int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!sel_bits) return VMOBA_ERR_ARG;
+  WsLayout L;
+  if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  return cuda_status(launch_plan(P, sel_bits, ws, L, stream));
+}
+
+int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
+                   const void* v_perm, const uint32_t* sel_bits, void* ws, size_t ws_bytes,
+                   float scale, void* out, float* lse, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!q || !k_perm || !v_perm || !sel_bits || !out || !lse) return VMOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(out))
+    return VMOBA_ERR_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
+  WsLayout L;
+  if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  return cuda_status(
+      launch_attn_fwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
+}
+
+int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
+                   const void* v_perm, const uint32_t* sel_bits, void* ws, size_t ws_bytes,
+                   float scale, const void* out, const float* lse, const void* dout, void* dq,
+                   void* dk, void* dv, void* ws_bwd, size_t ws_bwd_bytes, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!q || !k_perm || !v_perm || !sel_bits || !out || !lse || !dout || !dq || !dk || !dv)
+    return VMOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(out) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return VMOBA_ERR_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
+  WsLayout L;
+  if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  if (!ws_bwd || ws_bwd_bytes < vmoba_bwd_workspace_size(shape) || !aligned16(ws_bwd))
+    return VMOBA_ERR_WORKSPACE;
+  if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  return cuda_status(launch_attn_bwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out,
+                                          lse, dout, dq, dk, dv, static_cast<float*>(ws_bwd),
+                                          stream));
+}
+
+int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream) {
+  if (!ws || !device_status) return VMOBA_ERR_ARG;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return VMOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VMOBA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyAsync(ws, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return VMOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VMOBA_ERR_CUDA;
+  *device_status = v;
+  return VMOBA_OK;
+}
+
+const char* vmoba_status_string(int status) {
+  switch (status) {
+    case VMOBA_OK: return "ok";
+    case VMOBA_ERR_ARG: return "invalid argument";
+    case VMOBA_ERR_SHAPE: return "unsupported shape (box must divide T,H,W; head_dim 64 or 128)";
+    case VMOBA_ERR_DTYPE: return "unsupported dtype";
+    case VMOBA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case VMOBA_ERR_CUDA: return "CUDA runtime error";
+    case VMOBA_ERR_TIMEOUT: return "bounded device wait timed out";
+    case VMOBA_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case VMOBA_ERR_DEVICE: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,438 @@
+// Steps 2-3 of the layer: the per-head score pool S = scale * q_i b_i^T and
+// the global threshold selection over it.
+//
+// VMoBA notes, key design 2 (global block selection: one pool of all s x N_b
+// query-block pairs per head) and key design 3 (k = min{k' : cumulative
+// normalised similarity >= tau}); digest sections 3.3 and 3.4.
+//
+// "Normalised" is read as p = exp(S - max S) / Z over the head's whole pool,
+// Z = sum exp(S - max S).  The cut is found without sorting: an exact radix
+// select over the 32-bit order-preserving key of each fp32 score, three
+// passes of 11/11/10 bits.  Each pass histograms (count, sum of exp(S - m))
+// per digit for the elements still in the candidate bucket; a one-warp scan
+// per head walks the digits from the top until the mass reaches tau * Z.
+// Exact ties at the cut are ranked by flat index i*N_b + j (ascending) with
+// three more count-only radix passes that return at once unless needed.
+//
+// Kernels, in stream order: init -> score -> {hist, scan} x 3 ->
+// {tie_hist, tie_scan} x 3 -> emit (bitmap) -> stats.
+#include "common.cuh"
+
+namespace vmoba {
+namespace {
+
+constexpr int kSel_Search = 0, kSel_Resolved = 1, kSel_All = 2, kSel_Ties = 3;
+
+__device__ __forceinline__ float ld_f(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_h * kHistBins;
+       i += gridDim.x * blockDim.x) {
+    hc[i] = 0u;
+    hm[i] = 0.0;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < n_h) {
+    SelState s{};
+    s.max_key = 0u;
+    s.idx_cut = 0xFFFFFFFFu;
+    s.state = kSel_Search;
+    st[threadIdx.x] = s;
+  }
+}
+
+// ---------------------------------------------------------------- scores
+// 64 queries x 64 blocks per CTA step, 256 threads, 4x4 outputs per thread,
+// fp32 FMA over d.  Q tile and B chunk staged transposed in shared memory.
+constexpr int kSQ = 64, kSB = 64, kSPad = 68;
+
+template <typename E, int D>
+__global__ void __launch_bounds__(256)
+k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scale,
+        float* __restrict__ S, SelState* __restrict__ st) {
+  extern __shared__ __align__(16) float sm[];
+  float* Qs = sm;                  // [D][kSPad]
+  float* Bs = sm + D * kSPad;      // [D][kSPad]
+  const int i0 = blockIdx.x * kSQ, h = blockIdx.y;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+
+  for (int idx = threadIdx.x; idx < kSQ * D; idx += 256) {
+    int r = idx / D, c = idx - r * D;
+    int i = i0 + r;
+    Qs[c * kSPad + r] = (i < P.s) ? ld_f(q + ((size_t)i * P.n_h + h) * D + c) : 0.f;
+  }
+  float vmax = -INFINITY;
+  const float* Bh = B + (size_t)h * P.Nb * D;
+  for (int j0 = 0; j0 < P.Nb; j0 += kSB) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kSB * D; idx += 256) {
+      int r = idx / D, c = idx - r * D;
+      int j = j0 + r;
+      Bs[c * kSPad + r] = (j < P.Nb) ? __ldg(Bh + (size_t)j * D + c) : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      float4 qa = *reinterpret_cast<const float4*>(Qs + c * kSPad + 4 * ty);
+      float4 bb = *reinterpret_cast<const float4*>(Bs + c * kSPad + 4 * tx);
+      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], bv[b], acc[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      int i = i0 + 4 * ty + a;
+      if (i >= P.s) continue;
+      float* row = S + ((size_t)h * P.s + i) * P.Nb;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        int j = j0 + 4 * tx + b;
+        if (j < P.Nb) {
+          float x = acc[a][b] * scale;
+          row[j] = x;
+          vmax = fmaxf(vmax, x);
+        }
+      }
+    }
+  }
+  // per-head maximum -> ordered key, one atomic per warp
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  if ((threadIdx.x & 31) == 0 && vmax > -INFINITY) atomicMax(&st[h].max_key, f2key(vmax));
+}
+
+// ------------------------------------------------------------- histograms
+constexpr int kHistThreads = 256;
+constexpr int kHistChunk = 64 * 1024;   // pool elements per CTA
+
+template <int PASS>
+__device__ __forceinline__ bool digit_of(uint32_t key, uint32_t prefix, uint32_t& dig) {
+  if (PASS == 0) { dig = key >> 21; return true; }
+  if (PASS == 1) { dig = (key >> 10) & 2047u; return (key >> 21) == prefix; }
+  dig = key & 1023u;
+  return (key >> 10) == prefix;
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kHistThreads)
+k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t* __restrict__ hc,
+       double* __restrict__ hm) {
+  __shared__ uint32_t cnt[kHistBins];
+  __shared__ float mass[kHistBins];
+  const int h = blockIdx.y;
+  if (st[h].state != kSel_Search) return;
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) { cnt[b] = 0u; mass[b] = 0.f; }
+  __syncthreads();
+  const float m = key2f(st[h].max_key);
+  const uint32_t prefix = st[h].prefix;
+  const size_t pool = (size_t)P.s * P.Nb;
+  const float* base = S + (size_t)h * pool;
+  const size_t beg = (size_t)blockIdx.x * kHistChunk;
+  const size_t end = min(beg + (size_t)kHistChunk, pool);
+  for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) {
+    float x = __ldg(base + f);
+    uint32_t dig;
+    if (digit_of<PASS>(f2key(x), prefix, dig)) {
+      atomicAdd(&cnt[dig], 1u);
+      atomicAdd(&mass[dig], expf(x - m));
+    }
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
+    if (cnt[b]) {
+      atomicAdd(&hc[h * kHistBins + b], cnt[b]);
+      atomicAdd(&hm[h * kHistBins + b], (double)mass[b]);
+    }
+  }
+}
+
+// One warp per head: walk the digits from the top, stop where the mass
+// reaches the target, record the bucket and the mass/count strictly above.
+template <int PASS>
+__global__ void __launch_bounds__(32)
+k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __restrict__ hm,
+       float tau) {
+  const int h = blockIdx.x, lane = threadIdx.x;
+  SelState& S = st[h];
+  if (S.state != kSel_Search) return;
+  uint32_t* c = hc + h * kHistBins;
+  double* mm = hm + h * kHistBins;
+  const int nb = (PASS == 2) ? 1024 : 2048;
+  const int per = nb / 32;
+  // lane l owns digits nb-1-l*per ... nb-per-l*per (descending)
+  double lm = 0.0;
+  unsigned long long lc = 0;
+  for (int k = 0; k < per; ++k) {
+    int d = nb - 1 - lane * per - k;
+    lm += mm[d];
+    lc += c[d];
+  }
+  double above = S.mass_above, target = S.target;
+  unsigned long long cabove = S.count_above;
+  if (PASS == 0) {
+    double tot = lm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    above = 0.0;
+    cabove = 0;
+    target = (double)tau * tot;
+    if (lane == 0) { S.Z = tot; S.target = target; }
+  }
+  double incl = lm;
+  unsigned long long cincl = lc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double y = __shfl_up_sync(0xffffffffu, incl, o);
+    unsigned long long yc = __shfl_up_sync(0xffffffffu, cincl, o);
+    if (lane >= o) { incl += y; cincl += yc; }
+  }
+  const unsigned ball = __ballot_sync(0xffffffffu, above + incl >= target);
+  const unsigned nz = __ballot_sync(0xffffffffu, lc > 0);
+  if (ball == 0u && PASS == 0) {
+    // tau reaches the whole pool: every pair is selected
+    if (lane == 0) {
+      S.state = kSel_All;
+      S.n_selected = (unsigned long long)P.s * P.Nb;
+      S.mass_selected = S.Z;
+    }
+    return;
+  }
+  // deciding lane: first lane whose running mass reaches the target (or, on a
+  // rounding shortfall, the last lane holding elements), moved forward to a
+  // lane that holds elements
+  int fl = ball ? (__ffs(ball) - 1) : (31 - __clz(nz));
+  const unsigned later = nz & (0xffffffffu << fl);
+  fl = later ? (__ffs(later) - 1) : (31 - __clz(nz));
+  int chosen = -1;
+  double acc = 0.0;
+  unsigned long long cacc = 0;
+  if (lane == fl) {
+    acc = above + (incl - lm);
+    cacc = cabove + (cincl - lc);
+    int last = -1;
+    double acc_last = 0.0;
+    unsigned long long cacc_last = 0;
+    for (int k = 0; k < per; ++k) {
+      int d = nb - 1 - lane * per - k;
+      if (c[d]) {
+        if (acc + mm[d] >= target) { chosen = d; break; }
+        last = d;
+        acc_last = acc;
+        cacc_last = cacc;
+      }
+      acc += mm[d];
+      cacc += c[d];
+    }
+    if (chosen < 0) { chosen = last; acc = acc_last; cacc = cacc_last; }
+  }
+  chosen = __shfl_sync(0xffffffffu, chosen, fl);
+  acc = __shfl_sync(0xffffffffu, acc, fl);
+  cacc = __shfl_sync(0xffffffffu, cacc, fl);
+  if (lane == 0) {
+    const uint32_t pre = (PASS == 0) ? (uint32_t)chosen
+                                     : ((S.prefix << (PASS == 1 ? 11 : 10)) | (uint32_t)chosen);
+    S.prefix = pre;
+    S.mass_above = acc;
+    S.count_above = cacc;
+    if (PASS == 2) {
+      const uint32_t nt = c[chosen];
+      const double e = mm[chosen] / (double)nt;
+      const double need = target - acc;
+      const double rr = (need > 0.0 && e > 0.0) ? ceil(need / e) : 1.0;
+      const uint32_t r = (rr < 1.0) ? 1u : (rr >= (double)nt ? nt : (uint32_t)rr);
+      S.cut_key = pre;
+      S.tie_count = nt;
+      S.n_selected = cacc + r;
+      S.mass_selected = acc + (double)r * e;
+      if (r == nt) {
+        S.state = kSel_Resolved;
+        S.idx_cut = 0xFFFFFFFFu;
+      } else {
+        S.state = kSel_Ties;
+        S.tie_take = r;
+        S.prefix = 0u;
+      }
+    }
+  }
+  __syncwarp();
+  for (int d = lane; d < kHistBins; d += 32) { c[d] = 0u; mm[d] = 0.0; }
+}
+
+// ---- ties at the cut: rank by flat index (count-only radix select) ----
+template <int TP>
+__global__ void __launch_bounds__(kHistThreads)
+k_tie_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t* __restrict__ hc) {
+  __shared__ uint32_t cnt[kHistBins];
+  const int h = blockIdx.y;
+  if (st[h].state != kSel_Ties) return;
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) cnt[b] = 0u;
+  __syncthreads();
+  const uint32_t cut = st[h].cut_key, prefix = st[h].prefix;
+  const size_t pool = (size_t)P.s * P.Nb;
+  const float* base = S + (size_t)h * pool;
+  const size_t beg = (size_t)blockIdx.x * kHistChunk;
+  const size_t end = min(beg + (size_t)kHistChunk, pool);
+  for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) {
+    if (f2key(__ldg(base + f)) != cut) continue;
+    uint32_t idx = (uint32_t)f, dig;
+    if (digit_of<TP>(idx, prefix, dig)) atomicAdd(&cnt[dig], 1u);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads)
+    if (cnt[b]) atomicAdd(&hc[h * kHistBins + b], cnt[b]);
+}
+
+template <int TP>
+__global__ void __launch_bounds__(32)
+k_tie_scan(SelState* __restrict__ st, uint32_t* __restrict__ hc) {
+  const int h = blockIdx.x, lane = threadIdx.x;
+  SelState& S = st[h];
+  if (S.state != kSel_Ties) return;
+  uint32_t* c = hc + h * kHistBins;
+  const int nb = (TP == 2) ? 1024 : 2048;
+  const int per = nb / 32;
+  unsigned long long lc = 0;
+  for (int k = 0; k < per; ++k) lc += c[lane * per + k];       // ascending digits
+  unsigned long long incl = lc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned long long take = S.tie_take;
+  unsigned ball = __ballot_sync(0xffffffffu, incl >= take);
+  const int fl = ball ? (__ffs(ball) - 1) : 31;
+  int chosen = -1;
+  unsigned long long before = 0;
+  if (lane == fl) {
+    unsigned long long acc = incl - lc;
+    for (int k = 0; k < per; ++k) {
+      int d = lane * per + k;
+      if (acc + c[d] >= take) { chosen = d; break; }
+      acc += c[d];
+    }
+    if (chosen < 0) chosen = lane * per + per - 1;
+    before = acc;
+  }
+  chosen = __shfl_sync(0xffffffffu, chosen, fl);
+  before = __shfl_sync(0xffffffffu, before, fl);
+  if (lane == 0) {
+    const uint32_t pre = (TP == 0) ? (uint32_t)chosen
+                                   : ((S.prefix << (TP == 1 ? 11 : 10)) | (uint32_t)chosen);
+    S.prefix = pre;
+    S.tie_take = (uint32_t)(take - before);
+    if (TP == 2) {
+      S.idx_cut = pre;
+      S.state = kSel_Resolved;
+    }
+  }
+  __syncwarp();
+  for (int d = lane; d < kHistBins; d += 32) c[d] = 0u;
+}
+
+// ------------------------------------------------------------------ emit
+// One warp per (row, 32-block word): bit j set iff pair (i, j) is selected.
+__global__ void __launch_bounds__(256)
+k_emit(Prob P, const float* __restrict__ S, const SelState* __restrict__ st,
+       uint32_t* __restrict__ sel) {
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int state = st[h].state;
+  const uint32_t cut = st[h].cut_key, idx_cut = st[h].idx_cut;
+  const int rows_per_cta = 8 * 4;
+  for (int rr = warp; rr < rows_per_cta; rr += 8) {
+    const int i = blockIdx.x * rows_per_cta + rr;
+    if (i >= P.s) break;
+    const float* row = S + ((size_t)h * P.s + i) * P.Nb;
+    for (int w = 0; w < P.Wb; ++w) {
+      const int j = w * 32 + lane;
+      bool on = false;
+      if (j < P.Nb) {
+        if (state == kSel_All) {
+          on = true;
+        } else {
+          uint32_t key = f2key(__ldg(row + j));
+          uint32_t idx = (uint32_t)((size_t)i * P.Nb + j);
+          on = key > cut || (key == cut && idx <= idx_cut);
+        }
+      }
+      unsigned bits = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) sel[((size_t)h * P.s + i) * P.Wb + w] = bits;
+    }
+  }
+}
+
+__global__ void k_stats(Prob P, const SelState* __restrict__ st, vmoba_head_stats* __restrict__ out) {
+  const int h = threadIdx.x;
+  if (h >= P.n_h) return;
+  const SelState S = st[h];
+  vmoba_head_stats o;
+  o.n_selected = (long long)S.n_selected;
+  o.mass = S.Z > 0.0 ? S.mass_selected / S.Z : 0.0;
+  o.all_selected = S.state == kSel_All ? 1 : 0;
+  o.cut_score = S.state == kSel_All ? -INFINITY : key2f(S.cut_key);
+  out[h] = o;
+}
+
+template <typename E, int D>
+cudaError_t launch_score(const Prob& P, const void* q, const float* B, float scale, float* S,
+                         SelState* st, cudaStream_t stream) {
+  const size_t smem = sizeof(float) * 2 * D * kSPad;
+  cudaError_t e = cudaFuncSetAttribute(k_score<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((P.s + kSQ - 1) / kSQ, P.n_h);
+  k_score<E, D><<<grid, 256, smem, stream>>>(P, static_cast<const E*>(q), B, scale, S, st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_select(const Prob& P, const void* q, const float* blocks, float tau,
+                                float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
+                                const WsLayout& L, cudaStream_t stream) {
+  SelState* st = ws_ptr<SelState>(ws, L.sel_state);
+  uint32_t* hc = ws_ptr<uint32_t>(ws, L.hist_count);
+  double* hm = ws_ptr<double>(ws, L.hist_mass);
+  float* S = ws_ptr<float>(ws, L.scores);
+
+  k_init<<<64, 256, 0, stream>>>(st, hc, hm, P.n_h);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (P.dtype == VMOBA_BF16)
+    e = (P.d == 128) ? launch_score<__nv_bfloat16, 128>(P, q, blocks, scale, S, st, stream)
+                     : launch_score<__nv_bfloat16, 64>(P, q, blocks, scale, S, st, stream);
+  else
+    e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
+                     : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
+  if (e != cudaSuccess) return e;
+
+  const size_t pool = (size_t)P.s * P.Nb;
+  dim3 hgrid((unsigned)((pool + kHistChunk - 1) / kHistChunk), P.n_h);
+  k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  k_tie_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  k_tie_scan<0><<<P.n_h, 32, 0, stream>>>(st, hc);
+  k_tie_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  k_tie_scan<1><<<P.n_h, 32, 0, stream>>>(st, hc);
+  k_tie_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  k_tie_scan<2><<<P.n_h, 32, 0, stream>>>(st, hc);
+  dim3 egrid((P.s + 31) / 32, P.n_h);
+  k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
+  k_stats<<<1, 128, 0, stream>>>(P, st, stats);
+  return cudaGetLastError();
+}
+
+}  // namespace vmoba

@@ -1,0 +1,169 @@
+/*
+ * vmoba.h -- C ABI of the B200 (sm_100a) VMoBA per-layer sparse attention.
+ *
+ * The method (VMoBA: Mixture-of-Block Attention for Video Diffusion Models;
+ * papernotes.org ICLR 2026 notes, "overall framework" and key designs 1-3;
+ * paperlayer.ai digest, sections 3.1-3.4) replaces one full self-attention of
+ * a video DiT.  Q/K/V of a (T, H, W) video latent go in; an output of
+ * full-attention shape comes out.  Per layer l it
+ *   1. rearranges the keys into blocks of the layer's partition mode
+ *      (l mod 3: 1D temporal, 2D spatial across all frames, 3D local patch)
+ *      and mean-pools every block into B                  -> vmoba_partition
+ *   2. scores every query of a head against every block, S = scale*q.b,
+ *   3. ranks the head's whole s x N_b pool and keeps pairs in descending
+ *      order until the normalised cumulative similarity reaches tau
+ *                                                          -> vmoba_score_select
+ *   4. runs attention over the selected (query, block) pairs only
+ *                                         -> vmoba_build_plan, vmoba_attn_fwd,
+ *                                            vmoba_attn_bwd
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tokens are frame-major: token n = t*H*W + y*W + x.  s = T*H*W.
+ * Q, K, V, O, dO, dQ, dK, dV are [s][n_heads][head_dim] row-major (one
+ * sample; loop or offset pointers for a batch).  K', V' (keys/values in
+ * partition order) are [n_heads][s][head_dim].  Blocks are numbered
+ * row-major over the (T/bt', H/bh', W/bw') box grid; inside a block tokens
+ * keep (t, y, x) order.  dtype VMOBA_BF16 = bf16 storage, VMOBA_F32 = fp32;
+ * all accumulation is fp32 or wider.
+ * Selection bitmap sel_bits: [n_heads][s][ceil(N_b/32)] uint32, bit (j%32)
+ * of word (j/32) of row i set iff query i (original order) attends block j.
+ * Normalisation of the pool (the pages name it but print no formula; the
+ * reading taken): p = exp(S - max S) / sum exp(S - max S) over the head's
+ * whole pool; ties rank by (query asc, block asc); ">=" tau stops.
+ *
+ * Ownership: the caller allocates every buffer (device memory unless noted);
+ * the library never allocates, frees or synchronises.  Every compute call
+ * is asynchronous on the given stream.
+ * Errors: invalid arguments return a negative vmoba_status synchronously,
+ * before anything is launched.  A launch failure returns VMOBA_ERR_CUDA.
+ * Faults detected on the device (a bounded wait that ran out) are latched in
+ * a status word inside the workspace: read it with vmoba_get_status.
+ * Workspace contents are private; the same workspace must be passed to
+ * vmoba_score_select, vmoba_build_plan, vmoba_attn_fwd and vmoba_attn_bwd of
+ * one layer, and no two calls may use one workspace concurrently.
+ */
+#ifndef VMOBA_H_
+#define VMOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vmoba_status {
+  VMOBA_OK = 0,
+  VMOBA_ERR_ARG = -1,             /* null pointer, bad tau/scale, misaligned pointer */
+  VMOBA_ERR_SHAPE = -2,           /* box does not divide (T,H,W); unsupported head_dim */
+  VMOBA_ERR_DTYPE = -3,           /* dtype not VMOBA_BF16 / VMOBA_F32 */
+  VMOBA_ERR_WORKSPACE = -4,       /* workspace pointer null or smaller than required */
+  VMOBA_ERR_CUDA = -5,            /* a CUDA runtime call or launch failed */
+  VMOBA_ERR_TIMEOUT = -6,         /* a bounded device wait ran out (device status) */
+  VMOBA_ERR_NOT_IMPLEMENTED = -7, /* combination not built (e.g. this dtype/head_dim) */
+  VMOBA_ERR_DEVICE = -8           /* current device is not sm_100 */
+} vmoba_status;
+
+enum { VMOBA_BF16 = 0, VMOBA_F32 = 1 };
+
+/* One layer's problem.  mode: 0 = 1D (box bt x H x W), 1 = 2D (T x bh x bw),
+ * 2 = 3D (bt x bh x bw); the fields the mode does not use are ignored.
+ * head_dim must be 64 or 128. */
+typedef struct vmoba_shape {
+  int T, H, W;
+  int n_heads, head_dim;
+  int mode;
+  int bt, bh, bw;
+  int dtype;
+} vmoba_shape;
+
+/* Per-head selection result (written to device memory by vmoba_score_select).
+ * n_selected = k*, the number of (query, block) pairs kept; mass = their
+ * normalised cumulative similarity (>= tau unless every pair is kept);
+ * cut_score = S of the last pair kept. */
+typedef struct vmoba_head_stats {
+  long long n_selected;
+  double mass;
+  float cut_score;
+  int all_selected;               /* 1 when tau reached the whole pool */
+} vmoba_head_stats;
+
+/* Partition mode of layer l: l mod 3 (notes, key design 1).  -1 if l < 0. */
+int vmoba_mode_for_layer(int layer_idx);
+
+/* N_b of the shape's mode, or a negative vmoba_status. */
+int vmoba_num_blocks(const vmoba_shape* shape);
+
+/* Bytes of workspace for score_select / build_plan / attn_fwd / attn_bwd
+ * (one buffer serves them all), or 0 for an invalid shape. */
+size_t vmoba_workspace_size(const vmoba_shape* shape);
+
+/* Bytes of the extra backward workspace (row terms D = rowsum(dO*O)), or 0. */
+size_t vmoba_bwd_workspace_size(const vmoba_shape* shape);
+
+/* Step 1 (notes, key design 1: "rearrange K in (T H W), B = mean(K')").
+ * k, v: [s][n_heads][d] (dtype).  Writes k_perm, v_perm: [n_heads][s][d]
+ * (dtype; exact copies in partition order) and blocks: [n_heads][N_b][d]
+ * fp32 block means (fp64 accumulation).  All pointers 16-byte aligned. */
+int vmoba_partition(const vmoba_shape* shape, const void* k, const void* v,
+                    void* k_perm, void* v_perm, float* blocks, cudaStream_t stream);
+
+/* Steps 2-3 (notes, key design 2: per-head global pool q_i b_i^T; key design
+ * 3: k = min{k' : cumulative normalised similarity >= tau}; digest 3.3-3.4).
+ * q: [s][n_heads][d] (dtype); blocks from vmoba_partition.  tau in (0, 1]
+ * (tau >= the pool's total keeps every pair; tau <= 0 or NaN ->
+ * VMOBA_ERR_ARG).  scale <= 0 selects 1/sqrt(head_dim).  Writes sel_bits
+ * (layout above, fully overwritten) and stats[n_heads] (device).  The pool
+ * is ranked by an exact on-device radix select over (score desc, index asc);
+ * no host sort and no host round trip. */
+int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blocks,
+                       float tau, float scale, uint32_t* sel_bits,
+                       vmoba_head_stats* stats, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Step 4a: from any selection bitmap (vmoba_score_select's, or one the
+ * caller built), build the tile work lists the attention kernels walk:
+ * per 128-query tile (queries in partition order) the key tiles its rows
+ * touch, and per key tile the query tiles that touch it. */
+int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Step 4b (notes, overall framework: attention only over the selected
+ * blocks, output of full-attention shape, heads concatenated).
+ * For query i: LSE_i = log sum_{n : block(n) selected for i} exp(scale q_i.k_n),
+ * O_i = softmax-weighted sum of v_n; a row with no selected block gets
+ * O = 0 and LSE = -inf.  q: [s][n_heads][d]; k_perm, v_perm from
+ * vmoba_partition; sel_bits the bitmap the plan was built from.  Writes
+ * out [s][n_heads][d] (dtype) and lse [n_heads][s] fp32 (natural log). */
+int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
+                   const void* v_perm, const uint32_t* sel_bits, void* ws,
+                   size_t ws_bytes, float scale, void* out, float* lse,
+                   cudaStream_t stream);
+
+/* Step 4c: gradients through the selected pairs, mask held constant (the
+ * pages add no loss and route no gradient through selection).
+ * D_i = dO_i.O_i, dS = P*(dP - D), dQ = scale dS K, dK = scale dS^T Q,
+ * dV = P^T dO.  out, lse from vmoba_attn_fwd; dout [s][n_heads][d].
+ * Writes dq, dk, dv [s][n_heads][d] (dtype, original token order; rows
+ * with no attended query get zeros).  ws_bwd: vmoba_bwd_workspace_size
+ * bytes. */
+int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
+                   const void* v_perm, const uint32_t* sel_bits, void* ws,
+                   size_t ws_bytes, float scale, const void* out, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
+                   size_t ws_bwd_bytes, cudaStream_t stream);
+
+/* Reads the workspace's device status word (synchronises the stream) into
+ * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it. */
+int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream);
+
+/* Static text of a vmoba_status code. */
+const char* vmoba_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VMOBA_H_ */
