@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""VMoBA layer benchmark: attention fwd+bwd throughput on selected pairs.
+
+One step = one synthetic 55296-token sample (T24 x H36 x W64 latent, 12 heads
+of 128, bf16, tau = 0.25) pushed through three VMoBA layers l = 0, 1, 2, i.e.
+one layer of each partition mode (1D temporal frame blocks, 2D 6x8 spatial
+blocks across all frames, 3D 4x6x8 blocks), each layer running the whole hot
+path through the C ABI: partition + pool, score + global threshold select,
+plan, sparse attention forward and backward.
+
+value = FLOPs on selected pairs (4d fwd + 10d bwd per attended token pair
+and head) / device time, summed over ranks / max time over ranks.
+Inputs (170 MB per tensor) are larger than the 126 MB L2, so no flush runs
+between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "VMoBA attn fwd+bwd ms/layer & TFLOP/s (selected pairs) at 55K tokens, 1 B200"
+WORKLOAD_ID = 4
+TAU = 0.25
+LAYERS = (0, 1, 2)
+CALLS = ("partition", "score_select", "build_plan", "attn_fwd", "attn_bwd")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sus=p.get("bf16_tflops_sustained", p["bf16_tflops"]), src="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# --------------------------------------------------------------- clocks
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------- distributed
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------- inputs
+def host_inputs(sample: int):
+    """bf16 host tensors (pinned) of one synthetic sample: q, k, v, dout."""
+    import numpy as np
+    import torch
+
+    import synth
+    from synth.video_latents import round_to
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    q, k, v = synth.make_qkv(w.wid, sample, w.T, w.H, w.W, w.n_heads, w.head_dim, kind=w.kind)
+    dout = synth.make_dout(w.wid, sample, w.s, w.n_heads, w.head_dim)
+    out = []
+    for x in (q, k, v, dout):
+        t = torch.from_numpy(round_to(x, "bf16").astype(np.float32)).to(torch.bfloat16)
+        out.append(t.pin_memory())
+    return out
+
+
+def layer_shapes():
+    import synth
+    from block_sparse_attention_layer_b200 import LayerShape
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    shapes = []
+    for l in LAYERS:
+        mode = l % 3
+        bt, bh, bw = w.boxes[mode]
+        shapes.append(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, bt, bh, bw, "bf16"))
+    return w, shapes
+
+
+# ------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_layer_b200 as V
+    from block_sparse_attention_layer_b200 import metrics
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    w, shapes = layer_shapes()
+    peaks = load_peaks()
+    t0 = time.time()
+    hq, hk, hv, hdo = host_inputs(sample=rank)
+    gen_s = time.time() - t0
+    q, k, v, dout = (x.cuda(non_blocking=False) for x in (hq, hk, hv, hdo))
+    layers = [VMoBALayer(sh) for sh in shapes]
+    stream = torch.cuda.current_stream()
+
+    def one_step(events=None):
+        for li, L in enumerate(layers):
+            ev = events[li] if events is not None else None
+            if ev: ev[0].record(stream)
+            V.partition(L.shape, k, v, L.k_perm, L.v_perm, L.blocks)
+            if ev: ev[1].record(stream)
+            V.score_select(L.shape, q, L.blocks, TAU, 0.0, L.sel, L.stats, L.ws)
+            if ev: ev[2].record(stream)
+            V.build_plan(L.shape, L.sel, L.ws)
+            if ev: ev[3].record(stream)
+            L.forward(q)
+            if ev: ev[4].record(stream)
+            L.backward(q, dout)
+            if ev: ev[5].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        one_step()
+    torch.cuda.synchronize()
+
+    # selected pairs (deterministic for these inputs) -> FLOPs per step
+    pairs = []
+    density = []
+    for L in layers:
+        st = L.head_stats()
+        p = metrics.token_pairs_from_stats(st["n_selected"], L.block_len)
+        pairs.append(p)
+        density.append(p / (L.shape.s * L.shape.s * L.shape.n_heads))
+    d = w.head_dim
+    flops_step = sum(metrics.attention_flops(p, d, True, True) for p in pairs)
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in layers]
+           for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n_launch0 = V.kernel_launches()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for kstep in range(K):
+            one_step(evs[kstep])
+        end.record(stream)
+        torch.cuda.synchronize()
+    launches = V.kernel_launches() - n_launch0
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+
+    # per-call device times (ms, summed over layers, averaged over steps)
+    call_ms = {c: 0.0 for c in CALLS}
+    layer_call_ms = [[0.0] * len(CALLS) for _ in layers]
+    for kstep in range(K):
+        for li in range(len(layers)):
+            e = evs[kstep][li]
+            for ci, c in enumerate(CALLS):
+                t = e[ci].elapsed_time(e[ci + 1])
+                call_ms[c] += t / K
+                layer_call_ms[li][ci] += t / K
+
+    total_flops = flops_step * K
+    if world > 1:
+        tt = torch.tensor([elapsed_ms, total_flops], dtype=torch.float64, device="cuda")
+        mx = tt.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tt, op=dist.ReduceOp.SUM)
+        elapsed_max = float(mx[0])
+        total_flops = float(tt[1])
+    else:
+        elapsed_max = elapsed_ms
+    value = total_flops / (elapsed_max * 1e-3) / 1e12
+
+    # roofline: the dominant call of the step
+    s, nh = w.s, w.n_heads
+    fwd_flops = sum(metrics.attention_flops(p, d, True, False) for p in pairs)
+    bwd_flops = sum(metrics.attention_flops(p, d, False, True) for p in pairs)
+    achieved = {
+        "attn_bwd": (bwd_flops / (call_ms["attn_bwd"] * 1e-3) / 1e12, "TFLOP/s", "tensor"),
+        "attn_fwd": (fwd_flops / (call_ms["attn_fwd"] * 1e-3) / 1e12, "TFLOP/s", "tensor"),
+    }
+    part_bytes = sum(metrics.partition_bytes(s, nh, d, 2, V.num_blocks(sh)) for sh in shapes)
+    sel_bytes = sum(metrics.select_bytes(s, nh, V.num_blocks(sh)) for sh in shapes)
+    achieved["partition"] = (part_bytes / (call_ms["partition"] * 1e-3) / 1e9, "GB/s", "hbm")
+    achieved["score_select"] = (sel_bytes / (call_ms["score_select"] * 1e-3) / 1e9, "GB/s", "hbm")
+    dom = max(("attn_bwd", "attn_fwd"), key=lambda c: call_ms[c])
+    a, unit, bound = achieved[dom]
+    peak = peaks["bf16_sus"] if bound == "tensor" else peaks["hbm"]
+    roofline = {"bound": bound, "achieved": round(a, 3), "peak": peak, "unit": unit,
+                "frac": round(a / peak, 5), "traffic": None, "kernel": dom,
+                "peak_source": f"{peaks['src']} (sustained bf16)" if bound == "tensor"
+                else f"{peaks['src']} hbm"}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, layers, (hq, hk, hv, hdo), flops_step, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(elapsed_max / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded smooth+noise video-latent Q/K/V, dO ~ N(0,1))",
+            "config": {
+                "workload": "train-55296tok: T24xH36xW64 latent, 12 heads x 128, bf16, "
+                            "tau 0.25, layers l=0,1,2 (1D 1-frame / 2D 6x8 / 3D 4x6x8 blocks), "
+                            "fwd+bwd, batch 1 per GPU",
+                "global_batch": world, "seq_len": w.s, "parallelism": f"dp{world}",
+                "l2": "inputs larger than L2 (170 MB per tensor), no flush"},
+            "ms_per_layer": round(elapsed_max / K / len(layers), 4),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "detail": {
+                "call_ms_per_step": {c: round(call_ms[c], 4) for c in CALLS},
+                "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
+                                  for i, l in enumerate(LAYERS)},
+                "achieved": {c: [round(x[0], 3), x[1]] for c, x in achieved.items()},
+                "density": [round(x, 5) for x in density],
+                "selected_token_pairs": pairs,
+                "flops_per_step": flops_step,
+                "input_gen_s": round(gen_s, 2),
+            },
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, layers, host, flops_step, world):
+    """Same metric through the public API with host buffers: per layer, H2D of
+    q, k, v, dO from pinned memory, the ABI calls, D2H of O, dQ, dK, dV."""
+    import torch
+    hq, hk, hv, hdo = host
+    stream = torch.cuda.current_stream()
+    outs = [torch.empty_like(hq).pin_memory() for _ in range(4)]
+    dq_in, dk_in, dv_in, ddo_in = (torch.empty_like(x, device="cuda") for x in host)
+
+    def step():
+        for L in layers:
+            for dst, src in ((dq_in, hq), (dk_in, hk), (dv_in, hv), (ddo_in, hdo)):
+                dst.copy_(src, non_blocking=True)
+            L.step(dq_in, dk_in, dv_in, TAU, dout=ddo_in)
+            for dst, src in zip(outs, (L.out, L.dq, L.dk, L.dv)):
+                dst.copy_(src, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K = max(1, args.steps)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    nbytes = hq.numel() * hq.element_size()
+    return {"value": round(flops_step * K * world / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": 4 * nbytes * len(layers),
+            "d2h_bytes_per_step": 4 * nbytes * len(layers),
+            "ms_per_step": round(ms / K, 3)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def _oracle_sample(seconds: float, seed_rows: int = 0):
+    """Run the fp64 oracle on a bounded sample of the workload: the 3D layer of
+    one sample, head 0: partition + pool, scores, global threshold selection,
+    then masked attention forward + backward over chunks of 128 query rows
+    until ``seconds`` have elapsed.  Returns (selected-pair FLOPs, seconds, rows)."""
+    import numpy as np
+
+    import oracle as O
+    import synth
+    from synth.video_latents import round_to
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    mode = 2
+    t0 = time.perf_counter()
+    q, k, v = synth.make_qkv(w.wid, 0, w.T, w.H, w.W, 1, w.head_dim, kind=w.kind)
+    dout = synth.make_dout(w.wid, 0, w.s, 1, w.head_dim)
+    q, k, v, dout = (round_to(x, "bf16") for x in (q, k, v, dout))
+    t_gen = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    box = O.mode_box(mode, w.T, w.H, w.W, *w.boxes[mode])
+    B = O.pool_blocks(k, w.T, w.H, w.W, box)
+    S = O.block_scores(q, B, 1.0 / math.sqrt(w.head_dim))
+    sel, _ = O.threshold_select(S[0], TAU)
+    blk = O.block_of_token(w.T, w.H, w.W, box)
+    L = box[0] * box[1] * box[2]
+    scale = 1.0 / math.sqrt(w.head_dim)
+    rng = np.random.default_rng(seed_rows)
+    order = rng.permutation(w.s // 128)
+    pairs = 0
+    rows_done = 0
+    for c in order:
+        rows = np.arange(c * 128, (c + 1) * 128)
+        O.attention_bwd_rows(q[:, 0], k[:, 0], v[:, 0], sel, blk, scale, rows, dout[rows, 0])
+        O.attention_fwd_rows(q[:, 0], k[:, 0], v[:, 0], sel, blk, scale, rows)
+        pairs += int(sel[rows].sum()) * L
+        rows_done += len(rows)
+        if time.perf_counter() - t0 > seconds:
+            break
+    el = time.perf_counter() - t0
+    flops = pairs * 14 * w.head_dim
+    return flops, el, rows_done, t_gen
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds: float):
+    flops, el, rows, _ = _oracle_sample(seconds)
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": _cpu_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle, 3D layer (4x6x8 blocks), head 0 of 12: partition+pool, "
+                      f"scores, global threshold select, then masked attention fwd+bwd on "
+                      f"{rows} of 55296 query rows ({el:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    K = max(1, args.steps)
+    per_step = max(2.0, min(20.0, 120.0 / (K + args.warmup)))
+    for _ in range(args.warmup):
+        _oracle_sample(per_step / 4)
+    tot_flops = 0.0
+    tot_s = 0.0
+    rows_tot = 0
+    for kstep in range(K):
+        f, el, rows, _ = _oracle_sample(per_step, seed_rows=kstep + 1)
+        tot_flops += f
+        tot_s += el
+        rows_tot += rows
+    value = tot_flops / tot_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(tot_s / K * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "train-55296tok: T24xH36xW64 latent, 12 heads x 128, tau 0.25, "
+                               "3D layer sample", "global_batch": 1, "seq_len": 55296,
+                   "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: 3D layer head 0 partition/pool/score/select + "
+                                   f"masked attention fwd+bwd on ~{rows_tot // K} query rows"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

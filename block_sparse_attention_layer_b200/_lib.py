@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, P, Z, P]),
         "vmoba_get_status": (I, [P, ctypes.POINTER(I), P]),
         "vmoba_status_string": (ctypes.c_char_p, [I]),
+        "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -177,8 +178,29 @@ def partition(shape, k, v, k_perm, v_perm, blocks, stream=None):
         _stream(stream)))
 
 
+def _check_common(shape, q=None, k_perm=None, v_perm=None, sel_bits=None, ws=None):
+    import torch
+    dt = _torch_dtype(shape)
+    s, h, d = shape.s, shape.n_heads, shape.head_dim
+    if q is not None:
+        _expect(q, (s, h, d), dt, "q")
+    if k_perm is not None:
+        _expect(k_perm, (h, s, d), dt, "k_perm")
+    if v_perm is not None:
+        _expect(v_perm, (h, s, d), dt, "v_perm")
+    if sel_bits is not None:
+        _expect(sel_bits, (h, s, sel_words(shape)), torch.int32, "sel_bits")
+    if ws is not None and ws.numel() * ws.element_size() < workspace_size(shape):
+        raise ValueError("workspace smaller than vmoba_workspace_size")
+
+
 def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None):
     """Steps 2-3: scores, global threshold selection -> bitmap + per-head stats."""
+    import torch
+    _check_common(shape, q=q, sel_bits=sel_bits, ws=ws)
+    _expect(blocks, (shape.n_heads, num_blocks(shape), shape.head_dim), torch.float32, "blocks")
+    if stats.numel() * stats.element_size() < shape.n_heads * HEAD_STATS_DTYPE.itemsize:
+        raise ValueError("stats buffer too small")
     _check("vmoba_score_select", lib().vmoba_score_select(
         ctypes.byref(shape.c()), _ptr(q), _ptr(blocks), float(tau), float(scale),
         _ptr(sel_bits), _ptr(stats), _ptr(ws), ws.numel() * ws.element_size(),
@@ -186,12 +208,17 @@ def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None)
 
 
 def build_plan(shape, sel_bits, ws, stream=None):
+    _check_common(shape, sel_bits=sel_bits, ws=ws)
     _check("vmoba_build_plan", lib().vmoba_build_plan(
         ctypes.byref(shape.c()), _ptr(sel_bits), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
 def attn_fwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, out, lse, stream=None):
+    import torch
+    _check_common(shape, q, k_perm, v_perm, sel_bits, ws)
+    _expect(out, (shape.s, shape.n_heads, shape.head_dim), _torch_dtype(shape), "out")
+    _expect(lse, (shape.n_heads, shape.s), torch.float32, "lse")
     _check("vmoba_attn_fwd", lib().vmoba_attn_fwd(
         ctypes.byref(shape.c()), _ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(sel_bits), _ptr(ws),
         ws.numel() * ws.element_size(), float(scale), _ptr(out), _ptr(lse), _stream(stream)))
@@ -199,6 +226,14 @@ def attn_fwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, out, lse, stream=Non
 
 def attn_bwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, out, lse, dout, dq, dk, dv, ws_bwd,
              stream=None):
+    import torch
+    _check_common(shape, q, k_perm, v_perm, sel_bits, ws)
+    full = (shape.s, shape.n_heads, shape.head_dim)
+    for name, t in (("out", out), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _expect(t, full, _torch_dtype(shape), name)
+    _expect(lse, (shape.n_heads, shape.s), torch.float32, "lse")
+    if ws_bwd.numel() * ws_bwd.element_size() < bwd_workspace_size(shape):
+        raise ValueError("backward workspace smaller than vmoba_bwd_workspace_size")
     _check("vmoba_attn_bwd", lib().vmoba_attn_bwd(
         ctypes.byref(shape.c()), _ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(sel_bits), _ptr(ws),
         ws.numel() * ws.element_size(), float(scale), _ptr(out), _ptr(lse), _ptr(dout),
@@ -210,6 +245,11 @@ def get_status(ws, stream=None) -> int:
     v = ctypes.c_int(0)
     _check("vmoba_get_status", lib().vmoba_get_status(_ptr(ws), ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def kernel_launches() -> int:
+    """Kernels libvmoba has launched since load (its own host-side counter)."""
+    return int(lib().vmoba_kernel_launches())
 
 
 def decode_stats(stats_tensor) -> np.ndarray:

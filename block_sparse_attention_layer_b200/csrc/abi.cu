@@ -1,6 +1,7 @@
 // The extern "C" boundary: argument validation, problem geometry, workspace
 // layout and kernel launches.  Every entry point validates synchronously and
 // launches nothing on invalid input; see include/vmoba.h for the contract.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -9,6 +10,8 @@
 using namespace vmoba;
 
 namespace {
+
+std::atomic<unsigned long long> g_launches{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -54,7 +57,14 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? VMOBA_OK : VMOBA_ERR_
 
 }  // namespace
 
+namespace vmoba {
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
+}  // namespace vmoba
+
 extern "C" {
+
+unsigned long long vmoba_kernel_launches(void) { return g_launches.load(); }
+
 
 int vmoba_mode_for_layer(int layer_idx) { return layer_idx < 0 ? -1 : layer_idx % 3; }
 

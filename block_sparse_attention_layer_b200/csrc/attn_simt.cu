@@ -365,6 +365,7 @@ cudaError_t fwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
   k_fwd_simt<E, D><<<grid, kTile * (D / 32), smem, st>>>(
       P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
       qt_kt, scale, static_cast<E*>(out), lse);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -398,6 +399,7 @@ cudaError_t bwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
       P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
       kt_qt, scale, lse, static_cast<const E*>(dout), rowD, static_cast<E*>(dk),
       static_cast<E*>(dv));
+  count_launches(3);
   return cudaGetLastError();
 }
 

@@ -45,8 +45,10 @@ __host__ __device__ __forceinline__ int perm_token(const Prob& P, int p) {
   return (t * P.H + y) * P.W + x;
 }
 
-// Order-preserving map float -> uint32 (larger float <=> larger key).
+// Order-preserving map float -> uint32 (larger float <=> larger key); -0 and
+// +0 map to one key.
 __host__ __device__ __forceinline__ uint32_t f2key(float f) {
+  f = f + 0.0f;
   uint32_t b;
 #ifdef __CUDA_ARCH__
   b = __float_as_uint(f);
@@ -113,6 +115,10 @@ inline WsLayout ws_layout(const Prob& P) {
 
 template <typename T>
 inline T* ws_ptr(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+// Kernels launched by this library since load (diagnostics; see
+// vmoba_kernel_launches).  Every launch wrapper adds what it launched.
+void count_launches(int n);
 
 // ---- launch wrappers (one per kernel family; defined in the .cu files) ----
 cudaError_t launch_partition(const Prob& P, const void* k, const void* v, void* kp, void* vp,

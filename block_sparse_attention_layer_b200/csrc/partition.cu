@@ -92,6 +92,7 @@ cudaError_t launch_t(const Prob& P, const void* k, const void* v, void* kp, void
   k_partition_pool<E, D><<<grid, kWarps * 32, 0, st>>>(
       P, static_cast<const E*>(k), static_cast<const E*>(v), static_cast<E*>(kp),
       static_cast<E*>(vp), blocks);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -93,6 +93,7 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw);
   dim3 grid(P.n_qt, P.n_h);
   k_plan_tiles<<<grid, kTile, 0, st>>>(P, sel, qt_kt, qt_work, kt_qt, kt_work);
+  count_launches(2);
   return cudaGetLastError();
 }
 

@@ -196,7 +196,7 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
   }
   const unsigned ball = __ballot_sync(0xffffffffu, above + incl >= target);
   const unsigned nz = __ballot_sync(0xffffffffu, lc > 0);
-  if (ball == 0u && PASS == 0) {
+  if (nz == 0u || (ball == 0u && PASS == 0)) {
     // tau reaches the whole pool: every pair is selected
     if (lane == 0) {
       S.state = kSel_All;
@@ -432,6 +432,7 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   dim3 egrid((P.s + 31) / 32, P.n_h);
   k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
   k_stats<<<1, 128, 0, stream>>>(P, st, stats);
+  count_launches(16);
   return cudaGetLastError();
 }
 

@@ -159,6 +159,10 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
  * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it. */
 int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream);
 
+/* Number of CUDA kernels this library has launched since it was loaded
+ * (host-side counter, thread-safe; diagnostics for launch accounting). */
+unsigned long long vmoba_kernel_launches(void);
+
 /* Static text of a vmoba_status code. */
 const char* vmoba_status_string(int status);
 

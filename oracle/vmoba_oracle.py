@@ -29,6 +29,11 @@ step open, the reading taken is stated in the function's docstring:
    tokens inside a block are in (t, y, x) order.
 8. The selection mask is a constant for the backward pass (no gradient
    flows through the pooled blocks or the threshold).
+9. O, dQ, dK, dV are returned in the I/O dtype, rounded to nearest-even from
+   the exact values (round_io); LSE stays fp32.  Tolerances compare a
+   kernel's stored output with round_io of the fp64 result, since the
+   storage rounding itself (half an ulp: 0.03 at |x| = 8 in bf16) is not an
+   error of the computation.
 
 Pins (what ties each function to something other than itself) are in
 ``tests/test_oracle_pins.py``; each function's docstring lists them.
@@ -312,6 +317,22 @@ def vmoba_layer(Q, K, V, T, H, W, mode, box_cfg, tau, scale=None, dO=None,
         dQ, dK, dV = attention_bwd(Q, K, V, sel, blk, scale, dO, chunk)
         out.update(dQ=dQ, dK=dK, dV=dV)
     return out
+
+
+def round_io(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round exact results to the layer's I/O dtype (reading 9), back as float64.
+
+    fp32: IEEE round-to-nearest-even.  bf16: the fp32 value's upper 16 bits
+    rounded to nearest-even.  Pinned against torch's float -> bfloat16 cast.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    if dtype == "f32":
+        return x32.astype(np.float64)
+    bits = np.ascontiguousarray(x32).view(np.uint32).astype(np.uint64)
+    keep = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16
+    finite = np.isfinite(x32)
+    out = np.where(finite, keep, bits >> 16).astype(np.uint32) << 16
+    return out.view(np.float32).astype(np.float64)
 
 
 def selected_pair_density(sel_h: np.ndarray, L: int) -> float:

@@ -361,3 +361,13 @@ def test_layer_full_threshold_is_dense_attention_on_workload_inputs():
             ref = _sdpa(q[:, h], k[:, h], v[:, h], np.ones((w.s, w.s), bool),
                         1 / math.sqrt(w.head_dim)).numpy()
             np.testing.assert_allclose(out["O"][:, h], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_round_io_matches_torch_casts():
+    rng = np.random.default_rng(21)
+    x = np.concatenate([rng.standard_normal(4096) * 10.0 ** rng.integers(-6, 6, 4096),
+                        [0.0, -0.0, 1.0, 2.0 ** -130, 3.0e38, -np.inf, np.inf]])
+    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        ref = torch.from_numpy(x).to(torch.float32).to(tdt).to(torch.float64).numpy()
+        got = O.round_io(x, dt)
+        np.testing.assert_array_equal(got, ref)
