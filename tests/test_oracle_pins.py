@@ -371,3 +371,14 @@ def test_round_io_matches_torch_casts():
         ref = torch.from_numpy(x).to(torch.float32).to(tdt).to(torch.float64).numpy()
         got = O.round_io(x, dt)
         np.testing.assert_array_equal(got, ref)
+
+
+def test_half_ulp_bounds_the_rounding_of_torch_casts():
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal(20000) * 10.0 ** rng.integers(-5, 5, 20000)
+    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        stored = torch.from_numpy(x).to(torch.float32).to(tdt).to(torch.float64).numpy()
+        assert O.io_excess_error(stored, x, dt) == 0.0
+        # one ulp off is detected
+        bumped = stored + 4.0 * O.io_half_ulp(x, dt)
+        assert O.io_excess_error(bumped, x, dt) > 0.0
