@@ -91,7 +91,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_score_select": (I, [S, P, P, F, F, P, P, P, Z, P]),
         "vmoba_build_plan": (I, [S, P, P, Z, P]),
         "vmoba_attn_fwd": (I, [S, P, P, P, P, P, Z, F, P, P, P]),
-        "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, P, Z, P]),
+        "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, Z, P]),
         "vmoba_get_status": (I, [P, ctypes.POINTER(I), P]),
         "vmoba_status_string": (ctypes.c_char_p, [I]),
         "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
@@ -224,19 +224,20 @@ def attn_fwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, out, lse, stream=Non
         ws.numel() * ws.element_size(), float(scale), _ptr(out), _ptr(lse), _stream(stream)))
 
 
-def attn_bwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, out, lse, dout, dq, dk, dv, ws_bwd,
+def attn_bwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, lse, dout, dq, dk, dv, ws_bwd,
              stream=None):
+    """Step 4c; ``ws`` must hold the preceding attn_fwd's fp32 output copy."""
     import torch
     _check_common(shape, q, k_perm, v_perm, sel_bits, ws)
     full = (shape.s, shape.n_heads, shape.head_dim)
-    for name, t in (("out", out), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+    for name, t in (("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         _expect(t, full, _torch_dtype(shape), name)
     _expect(lse, (shape.n_heads, shape.s), torch.float32, "lse")
     if ws_bwd.numel() * ws_bwd.element_size() < bwd_workspace_size(shape):
         raise ValueError("backward workspace smaller than vmoba_bwd_workspace_size")
     _check("vmoba_attn_bwd", lib().vmoba_attn_bwd(
         ctypes.byref(shape.c()), _ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(sel_bits), _ptr(ws),
-        ws.numel() * ws.element_size(), float(scale), _ptr(out), _ptr(lse), _ptr(dout),
+        ws.numel() * ws.element_size(), float(scale), _ptr(lse), _ptr(dout),
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws_bwd), ws_bwd.numel() * ws_bwd.element_size(),
         _stream(stream)))
 

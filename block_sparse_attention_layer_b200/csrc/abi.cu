@@ -146,15 +146,15 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
 
 int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    const void* v_perm, const uint32_t* sel_bits, void* ws, size_t ws_bytes,
-                   float scale, const void* out, const float* lse, const void* dout, void* dq,
-                   void* dk, void* dv, void* ws_bwd, size_t ws_bwd_bytes, cudaStream_t stream) {
+                   float scale, const float* lse, const void* dout, void* dq, void* dk,
+                   void* dv, void* ws_bwd, size_t ws_bwd_bytes, cudaStream_t stream) {
   Prob P;
   int rc = make_prob(shape, &P);
   if (rc != VMOBA_OK) return rc;
-  if (!q || !k_perm || !v_perm || !sel_bits || !out || !lse || !dout || !dq || !dk || !dv)
+  if (!q || !k_perm || !v_perm || !sel_bits || !lse || !dout || !dq || !dk || !dv)
     return VMOBA_ERR_ARG;
-  if (!aligned16(q) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(out) ||
-      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+  if (!aligned16(q) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return VMOBA_ERR_ARG;
   if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
   WsLayout L;
@@ -162,8 +162,8 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (!ws_bwd || ws_bwd_bytes < vmoba_bwd_workspace_size(shape) || !aligned16(ws_bwd))
     return VMOBA_ERR_WORKSPACE;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
-  return cuda_status(launch_attn_bwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out,
-                                          lse, dout, dq, dk, dv, static_cast<float*>(ws_bwd),
+  return cuda_status(launch_attn_bwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, lse,
+                                          dout, dq, dk, dv, static_cast<float*>(ws_bwd),
                                           stream));
 }
 

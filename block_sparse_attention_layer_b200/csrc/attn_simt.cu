@@ -81,7 +81,7 @@ template <typename E, int D>
 __global__ void __launch_bounds__(kTile * (D / 32))
 k_fwd_simt(Prob P, const E* __restrict__ q, const E* __restrict__ kp, const E* __restrict__ vp,
            const uint32_t* __restrict__ sel, const uint32_t* __restrict__ qt_kt, float scale,
-           E* __restrict__ out, float* __restrict__ lse) {
+           E* __restrict__ out, float* __restrict__ o32, float* __restrict__ lse) {
   constexpr int TPR = D / 32;
   extern __shared__ __align__(16) float sm[];
   float* Ks = sm;
@@ -156,22 +156,28 @@ k_fwd_simt(Prob P, const E* __restrict__ q, const E* __restrict__ kp, const E* _
   if (!valid) return;
   const float inv = l > 0.f ? 1.f / l : 0.f;
   E* orow = out + ((size_t)i * P.n_h + h) * D + part * 32;
+  float* frow = o32 + ((size_t)i * P.n_h + h) * D + part * 32;
 #pragma unroll
-  for (int x = 0; x < 32; ++x) orow[x] = from_f<E>(o[x] * inv);
+  for (int x = 0; x < 32; ++x) {
+    orow[x] = from_f<E>(o[x] * inv);
+    frow[x] = o[x] * inv;
+  }
   if (part == 0) lse[(size_t)h * P.s + i] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
 }
 
 // ------------------------------------------------------------- bwd: D_i
+// D_i = dO_i . O_i with the forward's fp32 output (the stored bf16 output
+// would put its rounding, 2^-9 relative, into every dS of the row).
 template <typename E, int D>
-__global__ void k_bwd_rowdot(Prob P, const E* __restrict__ o, const E* __restrict__ dout,
+__global__ void k_bwd_rowdot(Prob P, const float* __restrict__ o, const E* __restrict__ dout,
                              float* __restrict__ rowD) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= P.s * P.n_h) return;
   const int i = warp / P.n_h, h = warp - i * P.n_h;
-  const E* a = o + (size_t)warp * D;
+  const float* a = o + (size_t)warp * D;
   const E* b = dout + (size_t)warp * D;
   float acc = 0.f;
-  for (int x = lane; x < D; x += 32) acc = fmaf(to_f(a[x]), to_f(b[x]), acc);
+  for (int x = lane; x < D; x += 32) acc = fmaf(a[x], to_f(b[x]), acc);
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   if (lane == 0) rowD[(size_t)h * P.s + i] = acc;
@@ -355,8 +361,8 @@ size_t dkdv_smem(const Prob& P) {
 
 template <typename E, int D>
 cudaError_t fwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
-                  const uint32_t* sel, const uint32_t* qt_kt, float scale, void* out, float* lse,
-                  cudaStream_t st) {
+                  const uint32_t* sel, const uint32_t* qt_kt, float scale, void* out, float* o32,
+                  float* lse, cudaStream_t st) {
   const size_t smem = fwd_smem<D>(P);
   cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<E, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -364,7 +370,7 @@ cudaError_t fwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
   dim3 grid(P.n_qt, P.n_h);
   k_fwd_simt<E, D><<<grid, kTile * (D / 32), smem, st>>>(
       P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
-      qt_kt, scale, static_cast<E*>(out), lse);
+      qt_kt, scale, static_cast<E*>(out), o32, lse);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -372,11 +378,11 @@ cudaError_t fwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
 template <typename E, int D>
 cudaError_t bwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
                   const uint32_t* sel, const uint32_t* qt_kt, const uint32_t* kt_qt, float scale,
-                  const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                  const float* o32, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, float* rowD, cudaStream_t st) {
   const int warps = P.s * P.n_h;
-  k_bwd_rowdot<E, D><<<(warps + 7) / 8, 256, 0, st>>>(P, static_cast<const E*>(out),
-                                                       static_cast<const E*>(dout), rowD);
+  k_bwd_rowdot<E, D><<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const E*>(dout),
+                                                       rowD);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t s1 = fwd_smem<D>(P);
@@ -409,27 +415,30 @@ cudaError_t launch_attn_fwd_simt(const Prob& P, const void* q, const void* kp, c
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
                                  void* out, float* lse, cudaStream_t st) {
   const uint32_t* qt_kt = ws_ptr<uint32_t>(ws, L.qt_kt_bits);
+  float* o32 = ws_ptr<float>(ws, L.o32);
   if (P.dtype == VMOBA_BF16)
-    return P.d == 128 ? fwd_t<__nv_bfloat16, 128>(P, q, kp, vp, sel, qt_kt, scale, out, lse, st)
-                      : fwd_t<__nv_bfloat16, 64>(P, q, kp, vp, sel, qt_kt, scale, out, lse, st);
-  return P.d == 128 ? fwd_t<float, 128>(P, q, kp, vp, sel, qt_kt, scale, out, lse, st)
-                    : fwd_t<float, 64>(P, q, kp, vp, sel, qt_kt, scale, out, lse, st);
+    return P.d == 128
+               ? fwd_t<__nv_bfloat16, 128>(P, q, kp, vp, sel, qt_kt, scale, out, o32, lse, st)
+               : fwd_t<__nv_bfloat16, 64>(P, q, kp, vp, sel, qt_kt, scale, out, o32, lse, st);
+  return P.d == 128 ? fwd_t<float, 128>(P, q, kp, vp, sel, qt_kt, scale, out, o32, lse, st)
+                    : fwd_t<float, 64>(P, q, kp, vp, sel, qt_kt, scale, out, o32, lse, st);
 }
 
 cudaError_t launch_attn_bwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
-                                 const void* out, const float* lse, const void* dout, void* dq,
-                                 void* dk, void* dv, float* rowD, cudaStream_t st) {
+                                 const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                 float* rowD, cudaStream_t st) {
   const uint32_t* qt_kt = ws_ptr<uint32_t>(ws, L.qt_kt_bits);
   const uint32_t* kt_qt = ws_ptr<uint32_t>(ws, L.kt_qt_bits);
+  const float* o32 = ws_ptr<float>(ws, L.o32);
   if (P.dtype == VMOBA_BF16)
-    return P.d == 128 ? bwd_t<__nv_bfloat16, 128>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, out,
+    return P.d == 128 ? bwd_t<__nv_bfloat16, 128>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, o32,
                                                   lse, dout, dq, dk, dv, rowD, st)
-                      : bwd_t<__nv_bfloat16, 64>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, out,
+                      : bwd_t<__nv_bfloat16, 64>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, o32,
                                                  lse, dout, dq, dk, dv, rowD, st);
-  return P.d == 128 ? bwd_t<float, 128>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, out, lse, dout,
+  return P.d == 128 ? bwd_t<float, 128>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, o32, lse, dout,
                                         dq, dk, dv, rowD, st)
-                    : bwd_t<float, 64>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, out, lse, dout,
+                    : bwd_t<float, 64>(P, q, kp, vp, sel, qt_kt, kt_qt, scale, o32, lse, dout,
                                        dq, dk, dv, rowD, st);
 }
 

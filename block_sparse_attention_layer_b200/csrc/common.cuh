@@ -91,6 +91,7 @@ struct SelState {
 struct WsLayout {
   size_t status, sel_state, hist_count, hist_mass, scores;
   size_t qt_kt_bits, qt_work, kt_qt_bits, kt_work;
+  size_t o32;            // fp32 copy of the forward output, [s][n_h][d]
   size_t total;
 };
 
@@ -109,6 +110,7 @@ inline WsLayout ws_layout(const Prob& P) {
   w.qt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
   w.kt_qt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
   w.kt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
+  w.o32 = take(sizeof(float) * (size_t)P.n_h * P.s * P.d);
   w.total = off;
   return w;
 }
@@ -133,7 +135,7 @@ cudaError_t launch_attn_fwd_simt(const Prob& P, const void* q, const void* kp, c
                                  void* out, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
-                                 const void* out, const float* lse, const void* dout, void* dq,
-                                 void* dk, void* dv, float* rowD, cudaStream_t st);
+                                 const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                 float* rowD, cudaStream_t st);
 
 }  // namespace vmoba

@@ -61,7 +61,7 @@ class VMoBALayer:
 
     def backward(self, q, dout, scale=0.0):
         _lib.attn_bwd(self.shape, q, self.k_perm, self.v_perm, self.sel, self.ws, scale,
-                      self.out, self.lse, dout, self.dq, self.dk, self.dv, self.ws_bwd)
+                      self.lse, dout, self.dq, self.dk, self.dv, self.ws_bwd)
         return self.dq, self.dk, self.dv
 
     def step(self, q, k, v, tau, dout=None, scale=0.0):

@@ -136,7 +136,8 @@ int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits,
  * O_i = softmax-weighted sum of v_n; a row with no selected block gets
  * O = 0 and LSE = -inf.  q: [s][n_heads][d]; k_perm, v_perm from
  * vmoba_partition; sel_bits the bitmap the plan was built from.  Writes
- * out [s][n_heads][d] (dtype) and lse [n_heads][s] fp32 (natural log). */
+ * out [s][n_heads][d] (dtype) and lse [n_heads][s] fp32 (natural log), and
+ * keeps an fp32 copy of O in the workspace for vmoba_attn_bwd. */
 int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    const void* v_perm, const uint32_t* sel_bits, void* ws,
                    size_t ws_bytes, float scale, void* out, float* lse,
@@ -145,15 +146,17 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
 /* Step 4c: gradients through the selected pairs, mask held constant (the
  * pages add no loss and route no gradient through selection).
  * D_i = dO_i.O_i, dS = P*(dP - D), dQ = scale dS K, dK = scale dS^T Q,
- * dV = P^T dO.  out, lse from vmoba_attn_fwd; dout [s][n_heads][d].
- * Writes dq, dk, dv [s][n_heads][d] (dtype, original token order; rows
- * with no attended query get zeros).  ws_bwd: vmoba_bwd_workspace_size
- * bytes. */
+ * dV = P^T dO.  D is taken from the fp32 output copy the preceding
+ * vmoba_attn_fwd left in ws (the same ws, sel_bits and inputs are
+ * required), so the bf16 rounding of the stored output does not enter the
+ * gradients.  lse from vmoba_attn_fwd; dout [s][n_heads][d].  Writes dq, dk,
+ * dv [s][n_heads][d] (dtype, original token order; a key no selected query
+ * attends gets zeros).  ws_bwd: vmoba_bwd_workspace_size bytes. */
 int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    const void* v_perm, const uint32_t* sel_bits, void* ws,
-                   size_t ws_bytes, float scale, const void* out, const float* lse,
-                   const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
-                   size_t ws_bwd_bytes, cudaStream_t stream);
+                   size_t ws_bytes, float scale, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, void* ws_bwd, size_t ws_bwd_bytes,
+                   cudaStream_t stream);
 
 /* Reads the workspace's device status word (synchronises the stream) into
  * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it. */

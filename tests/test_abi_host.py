@@ -114,7 +114,7 @@ def test_small_workspace_rejected():
     assert rc == -4
     rc = L.vmoba_build_plan(ctypes.byref(sh.c()), BAD, None, need, None)
     assert rc == -4
-    rc = L.vmoba_attn_bwd(ctypes.byref(sh.c()), BAD, BAD, BAD, BAD, BAD, need, 0.0, BAD, BAD,
+    rc = L.vmoba_attn_bwd(ctypes.byref(sh.c()), BAD, BAD, BAD, BAD, BAD, need, 0.0, BAD,
                           BAD, BAD, BAD, BAD, BAD, 0, None)
     assert rc == -4
 
