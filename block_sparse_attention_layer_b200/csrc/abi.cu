@@ -140,6 +140,11 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   WsLayout L;
   if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  // bf16 with head_dim 128 runs on the tensor cores; fp32 I/O (whose 1e-4
+  // bar rules out TF32) and head_dim 64 run on the CUDA cores
+  if (fwd_tc_supported(P))
+    return cuda_status(
+        launch_attn_fwd_tc(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
   return cuda_status(
       launch_attn_fwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
 }

@@ -133,6 +133,10 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
 cudaError_t launch_attn_fwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
                                  void* out, float* lse, cudaStream_t st);
+bool fwd_tc_supported(const Prob& P);
+cudaError_t launch_attn_fwd_tc(const Prob& P, const void* q, const void* kp, const void* vp,
+                               const uint32_t* sel, void* ws, const WsLayout& L, float scale,
+                               void* out, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
                                  const float* lse, const void* dout, void* dq, void* dk, void* dv,

@@ -20,10 +20,17 @@ Recipe (all on the host, fp64, reproducible bit for bit on any machine):
   clamp-to-edge, kernel radius ceil(3 sigma), each field rescaled to unit
   variance.
 * Q/K per head h: ``W_Q,h ~ N(0, 1/r)^{r x d}``,
-  ``W_K,h = W_Q,h + 0.5 N(0, 1/r)``; ``X = (F W_X + 0.5 eps) / sqrt(1.25)``
-  with eps ~ N(0, 1); Q and K share the fields F.  V uses its own fields
-  and its own W_V ~ N(0, 1/r).  An optional per-head gain c_h ~ U[0.5, 2]
-  multiplies Q and K of head h.
+  ``W_K,h = W_Q,h + 0.5 N(0, 1/r)``;
+  ``X = (a F W_X + eps) / sqrt(a^2 + 1)`` with eps ~ N(0, 1) and a the
+  weight of the smooth component (``coherence``); Q and K share the fields
+  F.  V uses its own fields and its own W_V ~ N(0, 1/r).  An optional
+  per-head gain c_h ~ U[0.5, 2] multiplies Q and K of head h.
+* a = 0.4 is calibrated on the 55296-token workload so that global threshold
+  selection at tau = 0.25 attends 22 % / 20 % / 14 % of the token pairs in the
+  1D / 2D / 3D layers (mean 0.19), the sparsity VMoBA's notes print for this
+  video size in Table 2.  A larger a makes block means coherent enough that a
+  handful of pairs carry most of a head's mass (a = 2: one pair per head in
+  the 3D layer).
 * The i.i.d. variant draws every element of Q, K, V from N(0, 1).
 
 Layout of every returned tensor: ``[s][n_heads][head_dim]``, token index
@@ -139,7 +146,7 @@ def _iid(seed: int, s: int, n_heads: int, d: int) -> np.ndarray:
 
 def make_qkv(workload_id: int, layer: int, T: int, H: int, W: int,
              n_heads: int, head_dim: int, kind: str = "smooth",
-             head_gain: bool = False, rank: int = 8):
+             head_gain: bool = False, rank: int = 8, coherence: float = 0.4):
     """Q, K, V as float64 arrays [s][n_heads][head_dim] (see module doc).
 
     ``kind`` is "iid" or "smooth"; ``head_gain`` draws c_h ~ U[0.5, 2] per head.
@@ -161,13 +168,14 @@ def make_qkv(workload_id: int, layer: int, T: int, H: int, W: int,
     Fv = smooth_fields(T, H, W, rank, seed_for(workload_id, layer, "v", _PART_FIELDS))
     Wv = standard_normal(seed_for(workload_id, layer, "v", _PART_W),
                          n_heads * rank * d).reshape(n_heads, rank, d) * sd
-    norm = 1.0 / math.sqrt(1.25)
-    q = (_project(F, Wq)
-         + 0.5 * _iid(seed_for(workload_id, layer, "q", _PART_EPS), s, n_heads, d)) * norm
-    k = (_project(F, Wk)
-         + 0.5 * _iid(seed_for(workload_id, layer, "k", _PART_EPS), s, n_heads, d)) * norm
-    v = (_project(Fv, Wv)
-         + 0.5 * _iid(seed_for(workload_id, layer, "v", _PART_EPS), s, n_heads, d)) * norm
+    a = float(coherence)
+    norm = 1.0 / math.sqrt(a * a + 1.0)
+    q = (a * _project(F, Wq)
+         + _iid(seed_for(workload_id, layer, "q", _PART_EPS), s, n_heads, d)) * norm
+    k = (a * _project(F, Wk)
+         + _iid(seed_for(workload_id, layer, "k", _PART_EPS), s, n_heads, d)) * norm
+    v = (a * _project(Fv, Wv)
+         + _iid(seed_for(workload_id, layer, "v", _PART_EPS), s, n_heads, d)) * norm
     if head_gain:
         c = 0.5 + 1.5 * uniform01(seed_for(workload_id, layer, "q", _PART_GAIN), n_heads)
         q = q * c[None, :, None]

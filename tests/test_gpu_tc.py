@@ -1,0 +1,150 @@
+"""Tensor-core path (bf16, head_dim 128) against the fp64 oracle.
+
+Small shapes are compared on every output element; the 32760- and 55296-token
+layers (ragged 60-token blocks; the headline shape) are compared on sampled
+query rows of two heads, with those heads attending the oracle's own
+selection, plus the full pair set of those heads.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+from synth.video_latents import round_to
+
+from .gpu_util import (TOL, from_device, out_err, pack_bits, pair_set_mismatch, sample_rows,
+                       to_device, unpack_bits)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from block_sparse_attention_layer_b200 import LayerShape  # noqa: E402
+from block_sparse_attention_layer_b200.layer import VMoBALayer  # noqa: E402
+
+# (name, T, H, W, heads, boxes per mode)
+SMALL = [
+    ("2048tok", 8, 16, 16, 2, ((1, 16, 16), (8, 4, 4), (2, 4, 4))),
+    ("360tok-ragged", 3, 10, 12, 2, ((1, 10, 12), (3, 5, 4), (1, 5, 4))),
+]
+
+
+def _inputs(seed, T, H, W, nh, with_dout=False):
+    q, k, v = synth.make_qkv(100 + seed, 0, T, H, W, nh, 128)
+    out = [round_to(x, "bf16") for x in (q, k, v)]
+    if with_dout:
+        out.append(round_to(synth.make_dout(100 + seed, 0, T * H * W, nh, 128), "bf16"))
+    return out
+
+
+def _oracle_sel(q, k, T, H, W, mode, box_cfg, tau):
+    box = O.mode_box(mode, T, H, W, *box_cfg)
+    S = O.block_scores(q, O.pool_blocks(k, T, H, W, box), 1 / math.sqrt(128))
+    sel, stats = O.select_all_heads(S, tau)
+    return box, S, sel, stats
+
+
+@pytest.mark.parametrize("case", range(len(SMALL)))
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("tau", [0.25, 0.6, 1.0])
+def test_tc_forward_small(case, mode, tau):
+    name, T, H, W, nh, boxes = SMALL[case]
+    q, k, v = _inputs(case, T, H, W, nh)
+    box, S, sel, _ = _oracle_sel(q, k, T, H, W, mode, boxes[mode], tau)
+    blk = O.block_of_token(T, H, W, box)
+    Oref, lse_ref = O.attention_fwd(q, k, v, sel, blk, 1 / math.sqrt(128))
+    sh = LayerShape(T, H, W, nh, 128, mode, *boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    L.partition_only(to_device(k, "bf16"), to_device(v, "bf16"))
+    L.use_selection(torch.from_numpy(pack_bits(sel)).cuda())
+    out, lse = L.forward(to_device(q, "bf16"))
+    torch.cuda.synchronize()
+    assert out_err(from_device(out), Oref, "bf16") <= TOL["bf16"]
+    lg = from_device(lse)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lg), fin)
+    if fin.any():
+        assert np.abs(lg[fin] - lse_ref[fin]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("case", range(len(SMALL)))
+@pytest.mark.parametrize("mode", [0, 2])
+def test_backward_after_tc_forward(case, mode):
+    name, T, H, W, nh, boxes = SMALL[case]
+    q, k, v, dout = _inputs(case, T, H, W, nh, with_dout=True)
+    tau = 0.4
+    box, S, sel, _ = _oracle_sel(q, k, T, H, W, mode, boxes[mode], tau)
+    blk = O.block_of_token(T, H, W, box)
+    dQ, dK, dV = O.attention_bwd(q, k, v, sel, blk, 1 / math.sqrt(128), dout)
+    sh = LayerShape(T, H, W, nh, 128, mode, *boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    qd = to_device(q, "bf16")
+    L.partition_only(to_device(k, "bf16"), to_device(v, "bf16"))
+    L.use_selection(torch.from_numpy(pack_bits(sel)).cuda())
+    L.forward(qd)
+    dq, dk, dv = L.backward(qd, to_device(dout, "bf16"))
+    torch.cuda.synchronize()
+    for name_, got, ref in (("dq", dq, dQ), ("dk", dk, dK), ("dv", dv, dV)):
+        assert out_err(from_device(got), ref, "bf16") <= TOL["bf16"], name_
+
+
+def test_tc_forward_empty_rows_and_single_pair():
+    name, T, H, W, nh, boxes = SMALL[0]
+    q, k, v = _inputs(7, T, H, W, nh)
+    sh = LayerShape(T, H, W, nh, 128, 2, *boxes[2], "bf16")
+    L = VMoBALayer(sh)
+    L.step(to_device(q, "bf16"), to_device(k, "bf16"), to_device(v, "bf16"), 1e-7)
+    torch.cuda.synchronize()
+    assert np.all(L.head_stats()["n_selected"] == 1)
+    g = unpack_bits(L.sel.cpu().numpy(), L.n_blocks)
+    rows_on = g.any(axis=2)
+    o = from_device(L.out).transpose(1, 0, 2)
+    assert np.all(o[~rows_on] == 0)
+    assert np.all(np.isneginf(from_device(L.lse)[~rows_on]))
+    box = O.mode_box(2, T, H, W, *boxes[2])
+    Oref, _ = O.attention_fwd(q, k, v, g, O.block_of_token(T, H, W, box), 1 / math.sqrt(128))
+    assert out_err(from_device(L.out), Oref, "bf16") <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("wid,mode", [(3, 0), (3, 1), (3, 2), (4, 0), (4, 1), (4, 2)])
+def test_tc_forward_full_size_sampled(wid, mode):
+    w = synth.WORKLOADS[wid]
+    heads = (0, w.n_heads - 1)
+    tau = 0.25
+    q, k, v = synth.make_qkv(w.wid, mode, w.T, w.H, w.W, w.n_heads, w.head_dim)
+    q, k, v = (round_to(x, "bf16") for x in (q, k, v))
+    sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *w.boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    qd = to_device(q, "bf16")
+    L.select(qd, to_device(k, "bf16"), to_device(v, "bf16"), tau)
+    torch.cuda.synchronize()
+    box = O.mode_box(mode, w.T, w.H, w.W, *w.boxes[mode])
+    B = O.pool_blocks(k, w.T, w.H, w.W, box)
+    blk = O.block_of_token(w.T, w.H, w.W, box)
+    bits = L.sel.cpu().numpy().copy()
+    g = unpack_bits(bits, L.n_blocks)
+    for h in heads:
+        S_h = O.block_scores(q[:, h:h + 1], B[h:h + 1], 1 / math.sqrt(128))[0]
+        m, st = O.threshold_select(S_h, tau)
+        assert pair_set_mismatch(g[h], S_h, m, st["cut_score"]) == 0
+        bits[h] = pack_bits(m)          # attend the oracle's own pairs on checked heads
+        g[h] = m
+    L.use_selection(torch.from_numpy(bits).cuda())
+    out, lse = L.forward(qd)
+    torch.cuda.synchronize()
+    got = from_device(out)
+    lg = from_device(lse)
+    for h in heads:
+        empty = np.flatnonzero(~g[h].any(axis=1))[:8]
+        rows = sample_rows(w.s, 192, seed=h, must=empty)
+        o_ref, l_ref = O.attention_fwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk,
+                                            1 / math.sqrt(128), rows)
+        assert out_err(got[rows, h], o_ref, "bf16") <= TOL["bf16"]
+        fin = np.isfinite(l_ref)
+        assert np.array_equal(np.isfinite(lg[h, rows]), fin)
+        if fin.any():
+            assert np.abs(lg[h, rows][fin] - l_ref[fin]).max() <= 1e-3
