@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "pairs.cuh"
 
 using namespace vmoba;
 
@@ -54,6 +55,14 @@ int check_ws(const Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? VMOBA_OK : VMOBA_ERR_CUDA; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
 
 }  // namespace
 
@@ -142,9 +151,11 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   // bf16 with head_dim 128 runs on the tensor cores; fp32 I/O (whose 1e-4
   // bar rules out TF32) and head_dim 64 run on the CUDA cores
-  if (fwd_tc_supported(P))
-    return cuda_status(
-        launch_attn_fwd_tc(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
+  if (uses_blk_path(P))
+    return cuda_status(launch_attn_fwd_blk(
+        P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
+        ws_ptr<char>(ws, L.part), scale, out, ws_ptr<float>(ws, L.o32), lse,
+        ws_ptr<int>(ws, L.status), num_sms(), stream));
   return cuda_status(
       launch_attn_fwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
 }

@@ -92,10 +92,18 @@ struct WsLayout {
   size_t status, sel_state, hist_count, hist_mass, scores;
   size_t qt_kt_bits, qt_work, kt_qt_bits, kt_work;
   size_t o32;            // fp32 copy of the forward output, [s][n_h][d]
+  size_t pairs;          // pair lists of the selection (pairs.cu)
+  size_t part;           // per-pair partial results of one head (block-major kernels)
   size_t total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t pairs_ws_bytes(const Prob& P);
+size_t blk_partial_bytes(const Prob& P);
+// bf16 with head_dim 128 runs the block-major tensor-core kernels; fp32 I/O
+// (whose 1e-4 bar rules out TF32) and head_dim 64 run on the CUDA cores.
+inline bool uses_blk_path(const Prob& P) { return P.dtype == VMOBA_BF16 && P.d == 128; }
 
 inline WsLayout ws_layout(const Prob& P) {
   WsLayout w{};
@@ -111,6 +119,8 @@ inline WsLayout ws_layout(const Prob& P) {
   w.kt_qt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
   w.kt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
   w.o32 = take(sizeof(float) * (size_t)P.n_h * P.s * P.d);
+  w.pairs = take(pairs_ws_bytes(P));
+  w.part = take(uses_blk_path(P) ? blk_partial_bytes(P) : 0);
   w.total = off;
   return w;
 }
@@ -133,10 +143,6 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
 cudaError_t launch_attn_fwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
                                  void* out, float* lse, cudaStream_t st);
-bool fwd_tc_supported(const Prob& P);
-cudaError_t launch_attn_fwd_tc(const Prob& P, const void* q, const void* kp, const void* vp,
-                               const uint32_t* sel, void* ws, const WsLayout& L, float scale,
-                               void* out, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,
                                  const uint32_t* sel, void* ws, const WsLayout& L, float scale,
                                  const float* lse, const void* dout, void* dq, void* dk, void* dv,

@@ -1,0 +1,209 @@
+// Pair lists of the selection bitmap (the (query, block) mask of VMoBA notes,
+// key design 2), built on the device for the block-major attention kernels.
+//
+// For every head h:
+//   row_cnt[i]   number of blocks query i selected;
+//   row_off[i]   exclusive prefix of row_cnt: the pairs of query i occupy
+//                slots row_off[i] .. row_off[i]+row_cnt[i]-1, in block order
+//                ("CSR"); partial results of the attention kernels live there;
+//   col_off[j]   start of block j's query list in col_rows ("CSC"), queries
+//                in ascending order (deterministic);
+//   item_off[j]  first work item of block j: its query list cut into tiles of
+//                128 queries; item_off[N_b] = number of work items.
+// Rows are processed in chunks of 256 (8 warps x 32 rows); per-chunk column
+// counts give each chunk's base inside every block list, and warp ballots
+// give each row's rank inside the chunk.
+#include "common.cuh"
+#include "pairs.cuh"
+
+namespace vmoba {
+namespace {
+
+constexpr int kChunkRows = 256;
+
+// Per (chunk, head): column counts of the chunk and the row popcounts.
+__global__ void __launch_bounds__(kChunkRows)
+k_pairs_count(Prob P, const uint32_t* __restrict__ sel, uint32_t* __restrict__ row_cnt,
+              uint32_t* __restrict__ chunk_cnt, int n_chunks) {
+  __shared__ uint32_t cc[kMaxBlocks];
+  const int c = blockIdx.x, h = blockIdx.y;
+  for (int j = threadIdx.x; j < P.Nb; j += blockDim.x) cc[j] = 0u;
+  __syncthreads();
+  const int i = c * kChunkRows + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  uint32_t n = 0;
+  for (int w = 0; w < P.Wb; ++w) {
+    const uint32_t bits = (i < P.s) ? __ldg(sel + ((size_t)h * P.s + i) * P.Wb + w) : 0u;
+    n += __popc(bits);
+    // column counts of this warp's 32 rows, one ballot per column of the word
+    const int jmax = min(32, P.Nb - w * 32);
+    for (int b = 0; b < jmax; ++b) {
+      const unsigned m = __ballot_sync(0xffffffffu, (bits >> b) & 1u);
+      if (lane == 0 && m) atomicAdd(&cc[w * 32 + b], (uint32_t)__popc(m));
+    }
+  }
+  if (i < P.s) row_cnt[(size_t)h * P.s + i] = n;
+  __syncthreads();
+  for (int j = threadIdx.x; j < P.Nb; j += blockDim.x)
+    chunk_cnt[((size_t)h * n_chunks + c) * P.Nb + j] = cc[j];
+}
+
+// Block-wide exclusive scan helper (blockDim.x == 1024).
+__device__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t s = sh[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;
+  }
+  __syncthreads();
+  const uint32_t before = (warp > 0 ? sh[warp - 1] : 0u) + x - v;
+  *total = sh[31];
+  __syncthreads();
+  return before;
+}
+
+// One CTA (1024 threads) per head: column totals and offsets, chunk bases,
+// work-item offsets, and the row offsets (CSR).
+__global__ void __launch_bounds__(1024)
+k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict__ chunk_cnt,
+             int n_chunks, uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_off,
+             uint32_t* __restrict__ item_off, uint32_t* __restrict__ head_totals) {
+  __shared__ uint32_t sh[32];
+  const int h = blockIdx.x, t = threadIdx.x;
+  uint32_t* cc = chunk_cnt + (size_t)h * n_chunks * P.Nb;
+  // column totals (one thread per block)
+  uint32_t tot = 0;
+  if (t < P.Nb)
+    for (int c = 0; c < n_chunks; ++c) tot += cc[(size_t)c * P.Nb + t];
+  uint32_t all;
+  const uint32_t off = block_excl_scan(t < P.Nb ? tot : 0u, sh, &all);
+  const uint32_t tiles = t < P.Nb ? (tot + kTile - 1) / kTile : 0u;
+  uint32_t n_items;
+  const uint32_t ioff = block_excl_scan(tiles, sh, &n_items);
+  if (t < P.Nb) {
+    col_off[(size_t)h * (P.Nb + 1) + t] = off;
+    item_off[(size_t)h * (P.Nb + 1) + t] = ioff;
+    // chunk bases in place: base of chunk c in block t's list
+    uint32_t run = off;
+    for (int c = 0; c < n_chunks; ++c) {
+      const uint32_t v = cc[(size_t)c * P.Nb + t];
+      cc[(size_t)c * P.Nb + t] = run;
+      run += v;
+    }
+  }
+  if (t == 0) {
+    col_off[(size_t)h * (P.Nb + 1) + P.Nb] = all;
+    item_off[(size_t)h * (P.Nb + 1) + P.Nb] = n_items;
+    head_totals[2 * h] = all;
+    head_totals[2 * h + 1] = n_items;
+  }
+  // row offsets: exclusive scan of row_cnt over s rows, 1024 at a time
+  uint32_t carry = 0;
+  for (int base = 0; base < P.s; base += 1024) {
+    const int i = base + t;
+    const uint32_t v = i < P.s ? row_cnt[(size_t)h * P.s + i] : 0u;
+    uint32_t sum;
+    const uint32_t ex = block_excl_scan(v, sh, &sum);
+    if (i < P.s) row_off[(size_t)h * (P.s + 1) + i] = carry + ex;
+    carry += sum;
+  }
+  if (t == 0) row_off[(size_t)h * (P.s + 1) + P.s] = carry;
+}
+
+// Per (chunk, head): write every row of the chunk into the lists of the
+// blocks it selected, at chunk base + rank among the chunk's rows.
+__global__ void __launch_bounds__(kChunkRows)
+k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restrict__ chunk_base,
+             int n_chunks, uint32_t* __restrict__ col_rows) {
+  __shared__ uint32_t wcnt[kChunkRows / 32][32];
+  const int c = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = c * kChunkRows + threadIdx.x;
+  const uint32_t* cb = chunk_base + ((size_t)h * n_chunks + c) * P.Nb;
+  uint32_t* rows = col_rows + (size_t)h * P.s * P.Nb;
+  for (int w = 0; w < P.Wb; ++w) {
+    const uint32_t bits = (i < P.s) ? __ldg(sel + ((size_t)h * P.s + i) * P.Wb + w) : 0u;
+    const int jmax = min(32, P.Nb - w * 32);
+    // counts of each warp for the 32 columns of this word
+    for (int b = 0; b < jmax; ++b) {
+      const unsigned m = __ballot_sync(0xffffffffu, (bits >> b) & 1u);
+      if (lane == b) wcnt[warp][b] = __popc(m);
+    }
+    __syncthreads();
+    // prefix over warps -> base of each warp for each column
+    if (warp == 0 && lane < jmax) {
+      uint32_t run = cb[w * 32 + lane];
+      for (int ww = 0; ww < kChunkRows / 32; ++ww) {
+        const uint32_t v = wcnt[ww][lane];
+        wcnt[ww][lane] = run;
+        run += v;
+      }
+    }
+    __syncthreads();
+    for (int b = 0; b < jmax; ++b) {
+      const unsigned m = __ballot_sync(0xffffffffu, (bits >> b) & 1u);
+      if ((bits >> b) & 1u) {
+        const uint32_t rank = __popc(m & ((1u << lane) - 1u));
+        rows[wcnt[warp][b] + rank] = (uint32_t)i;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t pairs_ws_bytes(const Prob& P) {
+  const int n_chunks = (P.s + kChunkRows - 1) / kChunkRows;
+  size_t b = 0;
+  auto take = [&](size_t x) { b += align_up(x, 256); };
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.s);                 // row_cnt
+  take(sizeof(uint32_t) * (size_t)P.n_h * (P.s + 1));           // row_off
+  take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // col_off
+  take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // item_off
+  take(sizeof(uint32_t) * 2 * P.n_h);                           // head totals
+  take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);     // chunk counts / bases
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_rows (worst case)
+  return b;
+}
+
+PairsView pairs_view(const Prob& P, void* base) {
+  const int n_chunks = (P.s + kChunkRows - 1) / kChunkRows;
+  PairsView v{};
+  char* p = static_cast<char*>(base);
+  auto take = [&](size_t x) { char* r = p; p += align_up(x, 256); return reinterpret_cast<uint32_t*>(r); };
+  v.row_cnt = take(sizeof(uint32_t) * (size_t)P.n_h * P.s);
+  v.row_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.s + 1));
+  v.col_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
+  v.item_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
+  v.head_totals = take(sizeof(uint32_t) * 2 * P.n_h);
+  v.chunk = take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);
+  v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
+  v.n_chunks = n_chunks;
+  return v;
+}
+
+cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, cudaStream_t st) {
+  dim3 g(v.n_chunks, P.n_h);
+  k_pairs_count<<<g, kChunkRows, 0, st>>>(P, sel, v.row_cnt, v.chunk, v.n_chunks);
+  k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
+                                       v.item_off, v.head_totals);
+  k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.col_rows);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+}  // namespace vmoba

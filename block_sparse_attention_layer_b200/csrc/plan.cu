@@ -10,6 +10,7 @@
 // the key-stationary backward walks.  Per-row masking inside a tile is done
 // by the attention kernels from the bitmap itself.
 #include "common.cuh"
+#include "pairs.cuh"
 
 namespace vmoba {
 namespace {
@@ -94,7 +95,9 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   dim3 grid(P.n_qt, P.n_h);
   k_plan_tiles<<<grid, kTile, 0, st>>>(P, sel, qt_kt, qt_work, kt_qt, kt_work);
   count_launches(2);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_pairs(P, sel, pairs_view(P, ws_ptr<char>(ws, L.pairs)), st);
 }
 
 }  // namespace vmoba

@@ -146,7 +146,8 @@ def _iid(seed: int, s: int, n_heads: int, d: int) -> np.ndarray:
 
 def make_qkv(workload_id: int, layer: int, T: int, H: int, W: int,
              n_heads: int, head_dim: int, kind: str = "smooth",
-             head_gain: bool = False, rank: int = 8, coherence: float = 0.4):
+             head_gain: bool = False, rank: int = 8, coherence: float = 0.4,
+             qk_gain: float = 1.0):
     """Q, K, V as float64 arrays [s][n_heads][head_dim] (see module doc).
 
     ``kind`` is "iid" or "smooth"; ``head_gain`` draws c_h ~ U[0.5, 2] per head.
@@ -176,6 +177,9 @@ def make_qkv(workload_id: int, layer: int, T: int, H: int, W: int,
          + _iid(seed_for(workload_id, layer, "k", _PART_EPS), s, n_heads, d)) * norm
     v = (a * _project(Fv, Wv)
          + _iid(seed_for(workload_id, layer, "v", _PART_EPS), s, n_heads, d)) * norm
+    if qk_gain != 1.0:
+        q = q * qk_gain
+        k = k * qk_gain
     if head_gain:
         c = 0.5 + 1.5 * uniform01(seed_for(workload_id, layer, "q", _PART_GAIN), n_heads)
         q = q * c[None, :, None]
