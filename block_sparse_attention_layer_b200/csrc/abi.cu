@@ -92,7 +92,7 @@ size_t vmoba_workspace_size(const vmoba_shape* shape) {
 size_t vmoba_bwd_workspace_size(const vmoba_shape* shape) {
   Prob P;
   if (make_prob(shape, &P) != VMOBA_OK) return 0;
-  return align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
+  return bwd_blk_ws_bytes(P);   // rowD and LSE*log2(e), [n_h][s] fp32 each
 }
 
 int vmoba_partition(const vmoba_shape* shape, const void* k, const void* v, void* k_perm,
@@ -178,6 +178,11 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (!ws_bwd || ws_bwd_bytes < vmoba_bwd_workspace_size(shape) || !aligned16(ws_bwd))
     return VMOBA_ERR_WORKSPACE;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  if (uses_blk_path(P))
+    return cuda_status(launch_attn_bwd_blk(
+        P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
+        ws_ptr<char>(ws, L.part), ws_ptr<float>(ws, L.o32), lse, dout, dq, dk, dv, ws_bwd,
+        scale, ws_ptr<int>(ws, L.status), num_sms(), stream));
   return cuda_status(launch_attn_bwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, lse,
                                           dout, dq, dk, dv, static_cast<float*>(ws_bwd),
                                           stream));

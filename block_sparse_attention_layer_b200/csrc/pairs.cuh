@@ -25,6 +25,13 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
                                 float scale, void* out, float* o32, float* lse, int* status,
                                 int num_sms, cudaStream_t st);
 
+size_t bwd_blk_ws_bytes(const Prob& P);
+cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
+                                const uint32_t* sel, const PairsView& pv, void* part,
+                                const float* o32, const float* lse, const void* dout, void* dq,
+                                void* dk, void* dv, void* ws_bwd, float scale, int* status,
+                                int num_sms, cudaStream_t st);
+
 // Pair slot of (query i, block j) for a selected pair: CSR offset of the row
 // plus the number of blocks below j the row selected.
 __device__ __forceinline__ uint32_t pair_slot(const uint32_t* __restrict__ row_off_h,

@@ -148,3 +148,59 @@ def test_tc_forward_full_size_sampled(wid, mode):
         assert np.array_equal(np.isfinite(lg[h, rows]), fin)
         if fin.any():
             assert np.abs(lg[h, rows][fin] - l_ref[fin]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_tc_backward_full_size(mode):
+    """55296-token layer, fwd + bwd on the tensor cores.  Two heads attend the
+    oracle's own pairs; dQ is compared on sampled rows, dK/dV on every key of
+    the blocks with the fewest selecting queries (only those queries reach
+    them, so the oracle needs just those rows), and keys of blocks nobody
+    selected must get exact zeros."""
+    w = synth.WORKLOADS[4]
+    heads = (0, w.n_heads - 1)
+    tau = 0.25
+    scale = 1 / math.sqrt(128)
+    q, k, v = synth.make_qkv(w.wid, 10 + mode, w.T, w.H, w.W, w.n_heads, w.head_dim)
+    dout = synth.make_dout(w.wid, 10 + mode, w.s, w.n_heads, w.head_dim)
+    q, k, v, dout = (round_to(x, "bf16") for x in (q, k, v, dout))
+    sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *w.boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    qd = to_device(q, "bf16")
+    L.select(qd, to_device(k, "bf16"), to_device(v, "bf16"), tau)
+    torch.cuda.synchronize()
+    box = O.mode_box(mode, w.T, w.H, w.W, *w.boxes[mode])
+    B = O.pool_blocks(k, w.T, w.H, w.W, box)
+    blk = O.block_of_token(w.T, w.H, w.W, box)
+    bits = L.sel.cpu().numpy().copy()
+    g = unpack_bits(bits, L.n_blocks)
+    for h in heads:
+        S_h = O.block_scores(q[:, h:h + 1], B[h:h + 1], scale)[0]
+        m, _ = O.threshold_select(S_h, tau)
+        bits[h] = pack_bits(m)
+        g[h] = m
+    L.use_selection(torch.from_numpy(bits).cuda())
+    L.forward(qd)
+    dq, dk, dv = L.backward(qd, to_device(dout, "bf16"))
+    torch.cuda.synchronize()
+    gq, gk, gv = from_device(dq), from_device(dk), from_device(dv)
+    for h in heads:
+        empty = np.flatnonzero(~g[h].any(axis=1))[:8]
+        rows = sample_rows(w.s, 128, seed=100 + h, must=empty)
+        dq_ref, _, _ = O.attention_bwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows,
+                                            dout[rows, h])
+        assert out_err(gq[rows, h], dq_ref, "bf16") <= TOL["bf16"]
+        counts = g[h].sum(axis=0)
+        for j in np.flatnonzero(counts == 0):
+            keys = np.flatnonzero(blk == j)
+            assert np.all(gk[keys, h] == 0) and np.all(gv[keys, h] == 0)
+        order = [j for j in np.argsort(counts, kind="stable") if counts[j] > 0]
+        for j in order[:2]:
+            if counts[j] > 1024:
+                break
+            qrows = np.flatnonzero(g[h][:, j])
+            _, dk_ref, dv_ref = O.attention_bwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale,
+                                                     qrows, dout[qrows, h])
+            keys = np.flatnonzero(blk == j)
+            assert out_err(gk[keys, h], dk_ref[keys], "bf16") <= TOL["bf16"]
+            assert out_err(gv[keys, h], dv_ref[keys], "bf16") <= TOL["bf16"]
