@@ -269,35 +269,36 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         tc_fence_after();
         const int lim = P.L - c * kTile;
         const bool full = lim >= kTile;
-        float p[128];
+        // S row: four loads, one wait; P in place
+        uint32_t xr[128];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t xr[32];
-          tmem_ld32(tS + lane_off + c4 * 32, xr);
-          tmem_ld_wait();
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + lane_off + c4 * 32, xr + c4 * 32);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const bool on = valid && (full || c4 * 32 + e < lim);
-            p[c4 * 32 + e] = on ? exp2f(fmaf(__uint_as_float(xr[e]), sl2, -l2)) : 0.f;
-          }
+        for (int e = 0; e < 128; ++e) {
+          const bool on = valid && (full || e < lim);
+          xr[e] = __float_as_uint(on ? exp2f(fmaf(__uint_as_float(xr[e]), sl2, -l2)) : 0.f);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free);       // S may be overwritten now
         const uint32_t tdP = tmem + 128 + b * 128 + lane_off;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t xr[32];
-          tmem_ld32(tdP + c4 * 32, xr);
+        for (int hh = 0; hh < 2; ++hh) {                  // dP in two halves of 64 columns
+          uint32_t dp[64];
+          tmem_ld32(tdP + hh * 64, dp);
+          tmem_ld32(tdP + hh * 64 + 32, dp + 32);
           tmem_ld_wait();
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float d0 = p[c4 * 32 + e] * (__uint_as_float(xr[e]) - Di);
-            const float d1 = p[c4 * 32 + e + 1] * (__uint_as_float(xr[e + 1]) - Di);
+          for (int e = 0; e < 64; e += 2) {
+            const float d0 = __uint_as_float(xr[hh * 64 + e]) * (__uint_as_float(dp[e]) - Di);
+            const float d1 =
+                __uint_as_float(xr[hh * 64 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di);
             pk[e >> 1] = pack_bf16x2(d0, d1);
           }
-          tmem_st16(tdP + c4 * 16, pk);
+          // dS columns [32 hh, 32 hh + 32): dP columns already read
+          tmem_st32(tdP + hh * 32, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -512,18 +513,20 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const float* L2 = sL + b * kTile;
       const float* Dq = sD + b * kTile;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t xs[32], xp[32];
-        tmem_ld32(tS + lane_off + c4 * 32, xs);
-        tmem_ld32(tP + lane_off + c4 * 32, xp);
+      for (int hh = 0; hh < 2; ++hh) {                 // 64 query columns per wait
+        uint32_t xs[64], xp[64];
+        tmem_ld32(tS + lane_off + hh * 64, xs);
+        tmem_ld32(tS + lane_off + hh * 64 + 32, xs + 32);
+        tmem_ld32(tP + lane_off + hh * 64, xp);
+        tmem_ld32(tP + lane_off + hh * 64 + 32, xp + 32);
         tmem_ld_wait();
-        uint32_t pp[16], pd[16];
+        uint32_t pp[32], pd[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 64; e += 2) {
           float pv2[2], dv2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qi = c4 * 32 + e + u;
+            const int qi = hh * 64 + e + u;
             const float pr = kvalid ? exp2f(fmaf(__uint_as_float(xs[e + u]), sl2, -L2[qi])) : 0.f;
             pv2[u] = pr;
             dv2[u] = pr * (__uint_as_float(xp[e + u]) - Dq[qi]);
@@ -531,8 +534,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           pp[e >> 1] = pack_bf16x2(pv2[0], pv2[1]);
           pd[e >> 1] = pack_bf16x2(dv2[0], dv2[1]);
         }
-        tmem_st16(tS + lane_off + c4 * 16, pp);
-        tmem_st16(tP + lane_off + c4 * 16, pd);
+        // P^T, dS^T columns [32 hh, 32 hh + 32): S^T / dP^T columns already read
+        tmem_st32(tS + lane_off + hh * 32, pp);
+        tmem_st32(tP + lane_off + hh * 32, pd);
       }
       tmem_st_wait();
       tc_fence_before();

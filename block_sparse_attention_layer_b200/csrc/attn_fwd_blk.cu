@@ -237,18 +237,15 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         const uint32_t tS = tmem + sb * 128 + lane_off;
         const int lim = P.L - c * kTile;        // keys of this chunk inside block j
         const bool full = lim >= kTile;         // uniform over the CTA
+        // the whole S row in registers: four loads, one wait
+        uint32_t xr[128];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, xr + c4 * 32);
+        tmem_ld_wait();
         float mt = -INFINITY;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t xr[32];
-          tmem_ld32(tS + c4 * 32, xr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = __uint_as_float(xr[e]);
-            mt = fmaxf(mt, (full || c4 * 32 + e < lim) ? x : -INFINITY);
-          }
-        }
+        for (int e = 0; e < 128; ++e)
+          mt = fmaxf(mt, (full || e < lim) ? __uint_as_float(xr[e]) : -INFINITY);
         const float mt2 = mt * sl2;
         const bool grows = m_run == -INFINITY || mt2 > m_run + kRescaleLog2;
         const bool rescale = grows && m_run > -INFINITY;
@@ -275,16 +272,14 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         float lsum = 0.f;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t xr[32];
-          tmem_ld32(tS + c4 * 32, xr);
-          tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float a = (full || c4 * 32 + e < lim)
-                                ? exp2f(fmaf(__uint_as_float(xr[e]), sl2, -m_run)) : 0.f;
-            const float b = (full || c4 * 32 + e + 1 < lim)
-                                ? exp2f(fmaf(__uint_as_float(xr[e + 1]), sl2, -m_run)) : 0.f;
+            const int col = c4 * 32 + e;
+            const float a = (full || col < lim)
+                                ? exp2f(fmaf(__uint_as_float(xr[col]), sl2, -m_run)) : 0.f;
+            const float b = (full || col + 1 < lim)
+                                ? exp2f(fmaf(__uint_as_float(xr[col + 1]), sl2, -m_run)) : 0.f;
             lsum += a + b;
             pk[e >> 1] = pack_bf16x2(a, b);
           }
