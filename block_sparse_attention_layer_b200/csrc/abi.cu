@@ -56,6 +56,20 @@ int check_ws(const Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? VMOBA_OK : VMOBA_ERR_CUDA; }
 
+ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
+  ItemBufs b{};
+  b.rows = item_rows_capacity(P);
+  char* p = ws_ptr<char>(ws, L.items);
+  b.qg = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align_up(b.rows * 128 * sizeof(__nv_bfloat16), 256);
+  b.dog = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align_up(b.rows * 128 * sizeof(__nv_bfloat16), 256);
+  b.l2g = reinterpret_cast<float*>(p);
+  p += align_up(b.rows * sizeof(float), 256);
+  b.dg = reinterpret_cast<float*>(p);
+  return b;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -154,8 +168,8 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (uses_blk_path(P))
     return cuda_status(launch_attn_fwd_blk(
         P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
-        ws_ptr<char>(ws, L.part), scale, out, ws_ptr<float>(ws, L.o32), lse,
-        ws_ptr<int>(ws, L.status), num_sms(), stream));
+        ws_ptr<char>(ws, L.part), item_bufs(P, ws, L), scale, out, ws_ptr<float>(ws, L.o32),
+        lse, ws_ptr<int>(ws, L.status), num_sms(), stream));
   return cuda_status(
       launch_attn_fwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, out, lse, stream));
 }
@@ -181,8 +195,8 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (uses_blk_path(P))
     return cuda_status(launch_attn_bwd_blk(
         P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
-        ws_ptr<char>(ws, L.part), ws_ptr<float>(ws, L.o32), lse, dout, dq, dk, dv, ws_bwd,
-        scale, ws_ptr<int>(ws, L.status), num_sms(), stream));
+        ws_ptr<char>(ws, L.part), item_bufs(P, ws, L), ws_ptr<float>(ws, L.o32), lse, dout, dq,
+        dk, dv, ws_bwd, scale, ws_ptr<int>(ws, L.status), num_sms(), stream));
   return cuda_status(launch_attn_bwd_simt(P, q, k_perm, v_perm, sel_bits, ws, L, scale, lse,
                                           dout, dq, dk, dv, static_cast<float*>(ws_bwd),
                                           stream));

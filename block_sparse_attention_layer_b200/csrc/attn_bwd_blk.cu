@@ -70,27 +70,11 @@ __device__ __forceinline__ QItem decode_qitem(const Prob& P, int n, const uint32
   return it;
 }
 
-// Gather `count` rows (indices rows[]) of a [s][n_h][128] bf16 tensor into a
-// 128B-swizzled K-major tile; rows past count are zero.  64 threads.
-__device__ __forceinline__ void gather_rows64(uint8_t* dst, const __nv_bfloat16* __restrict__ src,
-                                              const uint32_t* __restrict__ rows, int count,
-                                              int n_h, int h, int t) {
-#pragma unroll 4
-  for (int idx = t; idx < kTile * 16; idx += 64) {
-    const int r = idx >> 4, c = idx & 15;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r < count) {
-      const uint32_t i = __ldg(rows + r);
-      val = __ldg(reinterpret_cast<const uint4*>(src + ((size_t)i * n_h + h) * kD) + c);
-    }
-    *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalf + sw128_off(r, c & 7)) = val;
-  }
-}
-
 // =====================================================================
 // dQ pass.  TMEM: S [0,128), dP0 [128,256), dP1 [256,384), dQ [384,512).
-// Roles: warp 0 TMA (K, V chunks), warp 1 MMA, warps 2-3 gather Q and dO
-// (one buffer each), warps 4-7 softmax rows + epilogue.
+// Roles: warp 0 TMA (the item's Q and dO tiles from the item-ordered copies,
+// then the block's K, V chunks), warp 1 MMA, warps 4-7 softmax rows +
+// epilogue (warps 2-3 idle).
 // =====================================================================
 struct DqBars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
@@ -103,10 +87,10 @@ constexpr size_t kDqSmem = 1024 + 2 * kTileB /*Q,dO*/ + 4 * kTileB /*K,V x2*/ + 
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-             Prob P, int h, const __nv_bfloat16* __restrict__ q,
-             const __nv_bfloat16* __restrict__ dout, const uint32_t* __restrict__ sel,
-             PairsView pv, const float* __restrict__ rowD, const float* __restrict__ lse2,
-             float sl2, float* __restrict__ part_dq, int* __restrict__ status) {
+             const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+             Prob P, int h, const uint32_t* __restrict__ sel, PairsView pv,
+             const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
+             float* __restrict__ part_dq, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -133,7 +117,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->ds_full[i], 4);
     }
     mbar_init(&bars->s_free, 4);
-    mbar_init(&bars->qd_full, 64);
+    mbar_init(&bars->qd_full, 1);
     mbar_init(&bars->qd_empty, 1);
     mbar_init(&bars->dq_final, 1);
     mbar_init(&bars->dq_free, 4);
@@ -154,10 +138,19 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int J = 0;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_o);
+      int J = 0, it_local = 0;
       bool ok = true;
-      for (int n = blockIdx.x; n < n_items && ok; n += G) {
+      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
         const QItem it = decode_qitem(P, n, item_off, col_off, col_rows);
+        if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, status, abort);
+        if (!ok) break;
+        mbar_expect_tx(&bars->qd_full, 2 * kTileB);
+        tma_load_2d(sQ, &tm_q, &bars->qd_full, 0, n * kTile);
+        tma_load_2d(sQ + kHalf, &tm_q, &bars->qd_full, 64, n * kTile);
+        tma_load_2d(sO, &tm_o, &bars->qd_full, 0, n * kTile);
+        tma_load_2d(sO + kHalf, &tm_o, &bars->qd_full, 64, n * kTile);
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + it.j * P.L + c * kTile;
           const int st = J & 1;
@@ -232,21 +225,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       }
       if (ok && J > 0) issue_dq(J - 1, prev_c, prev_it);
     }
-  } else if (warp < 4) {
-    const int t = threadIdx.x - 64;
-    int it_local = 0;
-    for (int n = blockIdx.x; n < n_items; n += G, ++it_local) {
-      if (it_local >= 1) {
-        const bool ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, status, abort);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      const QItem it = decode_qitem(P, n, item_off, col_off, col_rows);
-      gather_rows64(sQ, q, it.rows, it.count, P.n_h, h, t);
-      gather_rows64(sO, dout, it.rows, it.count, P.n_h, h, t);
-      fence_proxy_async();
-      mbar_arrive(&bars->qd_full);
-    }
-  } else {
+  } else if (warp >= 4) {
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -259,8 +238,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       float l2 = 0.f, Di = 0.f;
       if (valid) {
         i = __ldg(it.rows + r);
-        l2 = __ldg(lse2 + (size_t)h * P.s + i);
-        Di = __ldg(rowD + (size_t)h * P.s + i);
+        l2 = __ldg(l2g + (size_t)n * kTile + r);
+        Di = __ldg(dg + (size_t)n * kTile + r);
       }
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
@@ -360,9 +339,10 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
 // =====================================================================
 // dK/dV pass.  Item = (key tile kt of block j, head h), one CTA each.
 // TMEM: S^T [0,128) (then P^T), dP^T [128,256) (then dS^T), dV [256,384),
-// dK [384,512).  Roles: warp 0 loads the K/V tile once (TMA), warp 1 MMA,
-// warps 2-3 gather Q, dO, lse2 and D of each query tile (2 buffers),
-// warps 4-7 softmax rows (one key per thread) + epilogue.
+// dK [384,512).  Roles: warp 0 loads the K/V tile once, then each query
+// tile's Q and dO (TMA, item-ordered copies) and LSE*log2e, D (bulk copies)
+// into two buffers; warp 1 MMA; warps 4-7 softmax rows (one key per thread)
+// + epilogue (warps 2-3 idle).
 // =====================================================================
 struct KvBars {
   uint64_t kv_full;
@@ -376,10 +356,10 @@ constexpr size_t kKvSmem = 1024 + 2 * kTileB /*K,V*/ + 4 * kTileB /*Q,dO x2*/ +
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               Prob P, const __nv_bfloat16* __restrict__ q,
-               const __nv_bfloat16* __restrict__ dout, PairsView pv,
-               const float* __restrict__ rowD, const float* __restrict__ lse2, float sl2,
-               float scale, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+               const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+               Prob P, int h, PairsView pv, const float* __restrict__ dg,
+               const float* __restrict__ l2g, float sl2, float scale,
+               __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -394,10 +374,10 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   volatile int* abort = &bars->abort;
 
   const int nkt = (P.L + kTile - 1) / kTile;
-  const int j = blockIdx.x / nkt, kt = blockIdx.x - j * nkt, h = blockIdx.y;
+  const int j = blockIdx.x / nkt, kt = blockIdx.x - j * nkt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
+  const int item0 = (int)__ldg(pv.item_off + (size_t)h * (P.Nb + 1) + j);
   const int c0 = (int)__ldg(col_off + j), c1 = (int)__ldg(col_off + j + 1);
   const int nq = c1 - c0;
   const int ng = (nq + kTile - 1) / kTile;           // query tiles of block j
@@ -406,7 +386,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 64); mbar_init(&bars->qd_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->pd_full, 4);
     mbar_init(&bars->acc_final, 1);
@@ -431,6 +411,20 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       tma_load_2d(sK + kHalf, &tm_k, &bars->kv_full, 64, row);
       tma_load_2d(sV, &tm_v, &bars->kv_full, 0, row);
       tma_load_2d(sV + kHalf, &tm_v, &bars->kv_full, 64, row);
+      bool ok = true;
+      for (int g = 0; g < ng && ok; ++g) {
+        const int b = g & 1;
+        if (g >= 2) ok = mbar_wait(&bars->qd_empty[b], ((g >> 1) - 1) & 1, status, abort);
+        if (!ok) break;
+        const int qrow = (item0 + g) * kTile;
+        mbar_expect_tx(&bars->qd_full[b], 2 * kTileB + 2 * kTile * sizeof(float));
+        tma_load_2d(sQ + b * kTileB, &tm_q, &bars->qd_full[b], 0, qrow);
+        tma_load_2d(sQ + b * kTileB + kHalf, &tm_q, &bars->qd_full[b], 64, qrow);
+        tma_load_2d(sO + b * kTileB, &tm_o, &bars->qd_full[b], 0, qrow);
+        tma_load_2d(sO + b * kTileB + kHalf, &tm_o, &bars->qd_full[b], 64, qrow);
+        bulk_load(sL + b * kTile, l2g + qrow, kTile * sizeof(float), &bars->qd_full[b]);
+        bulk_load(sD + b * kTile, dg + qrow, kTile * sizeof(float), &bars->qd_full[b]);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && ng > 0) {
@@ -471,32 +465,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       }
       if (ok) mma_commit(&bars->acc_final);
     }
-  } else if (warp < 4) {
-    const int t = threadIdx.x - 64;
-    for (int g = 0; g < ng; ++g) {
-      const int b = g & 1;
-      if (g >= 2) {
-        const bool ok = mbar_wait(&bars->qd_empty[b], ((g >> 1) - 1) & 1, status, abort);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      const uint32_t* rows = col_rows + c0 + g * kTile;
-      const int count = min(kTile, nq - g * kTile);
-      gather_rows64(sQ + b * kTileB, q, rows, count, P.n_h, h, t);
-      gather_rows64(sO + b * kTileB, dout, rows, count, P.n_h, h, t);
-      for (int r = t; r < kTile; r += 64) {
-        float l = INFINITY, d = 0.f;          // padding queries: P = exp2(x - inf) = 0
-        if (r < count) {
-          const uint32_t i = __ldg(rows + r);
-          l = __ldg(lse2 + (size_t)h * P.s + i);
-          d = __ldg(rowD + (size_t)h * P.s + i);
-        }
-        sL[b * kTile + r] = l;
-        sD[b * kTile + r] = d;
-      }
-      fence_proxy_async();
-      mbar_arrive(&bars->qd_full[b]);
-    }
-  } else {
+  } else if (warp >= 4) {
     const int wq = warp - 4;
     const int c = wq * 32 + lane;                     // key row of this thread
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -504,7 +473,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool ok = true;
     for (int g = 0; g < ng && ok; ++g) {
       const int b = g & 1;
-      // qd_full also publishes sL / sD of this tile to the softmax warps
+      // qd_full also covers sL / sD of this tile
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, status, abort));
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, status, abort));
@@ -598,12 +567,14 @@ size_t bwd_blk_ws_bytes(const Prob& P) {
 
 cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
-                                const float* o32, const float* lse, const void* dout, void* dq,
-                                void* dk, void* dv, void* ws_bwd, float scale, int* status,
-                                int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv;
+                                const ItemBufs& ib, const float* o32, const float* lse,
+                                const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
+                                float scale, int* status, int num_sms, cudaStream_t st) {
+  CUtensorMap tk, tv, tq, to;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
-  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128))
+  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
+      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128) ||
+      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, kD, 128))
     return cudaErrorInvalidValue;
   float* rowD = static_cast<float*>(ws_bwd);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws_bwd) +
@@ -619,20 +590,22 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
   if (e != cudaSuccess) return e;
   const float sl2 = scale * kLog2e;
   float* part_dq = static_cast<float*>(part);
+  const int nkt = (P.L + kTile - 1) / kTile;
   for (int h = 0; h < P.n_h; ++h) {
-    k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(
-        tk, tv, P, h, static_cast<const __nv_bfloat16*>(q),
-        static_cast<const __nv_bfloat16*>(dout), sel, pv, rowD, lse2, sl2, part_dq, status);
+    // padding rows get LSE = +inf, so their P is exactly 0
+    e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q),
+                            static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, lse2, rowD,
+                            ib.l2g, ib.dg, INFINITY, num_sms, st);
+    if (e != cudaSuccess) return e;
+    k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, sel, pv, ib.dg,
+                                                      ib.l2g, sl2, part_dq, status);
     k_bwd_dq_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
                                                   static_cast<__nv_bfloat16*>(dq));
+    k_bwd_dkdv_blk<<<P.Nb * nkt, kThreads, kKvSmem, st>>>(
+        tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv), status);
   }
-  const int nkt = (P.L + kTile - 1) / kTile;
-  dim3 grid(P.Nb * nkt, P.n_h);
-  k_bwd_dkdv_blk<<<grid, kThreads, kKvSmem, st>>>(
-      tk, tv, P, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout),
-      pv, rowD, lse2, sl2, scale, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), status);
-  count_launches(1 + 2 * P.n_h + 1);
+  count_launches(1 + 3 * P.n_h);
   return cudaGetLastError();
 }
 

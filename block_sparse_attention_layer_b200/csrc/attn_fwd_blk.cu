@@ -17,8 +17,9 @@
 //   warp 0      TMA producer of the block's K / V chunks (2-stage rings);
 //   warp 1      TMEM owner (512 columns) and single-thread MMA issuer:
 //               S = Q K^T into two S buffers; O += P V with P read from TMEM;
-//   warps 2-3   gather the next item's 128 query rows into the free one of
-//               two Q buffers (128B-swizzled, K-major);
+//   (warps 2-3 idle: the softmax warpgroup must start at a multiple of 4)
+// Query tiles come by TMA from the item-ordered copy of Q (gather.cu) into
+// two Q buffers, loaded by the producer ahead of the item.
 //   warps 4-7   softmax: one query row per thread, lazy 2^8 rescale of O,
 //               then the item's epilogue (partials out).
 // TMEM columns: S0 [0,128), S1 [128,256), O [256,384).
@@ -73,7 +74,8 @@ __device__ __forceinline__ Item decode_item(const Prob& P, int n, const uint32_t
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-          Prob P, int h, const __nv_bfloat16* __restrict__ q, const uint32_t* __restrict__ sel,
+          const __grid_constant__ CUtensorMap tm_q, Prob P, int h,
+          const uint32_t* __restrict__ sel,
           PairsView pv, float sl2, float* __restrict__ part_o, float2* __restrict__ part_ml,
           int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -100,7 +102,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       mbar_init(&bars->full_v[i], 1); mbar_init(&bars->empty_v[i], 1);
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 4);
       mbar_init(&bars->o_done[i], 1);
-      mbar_init(&bars->q_full[i], 64); mbar_init(&bars->q_empty[i], 1);
+      mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 1);
     }
     mbar_init(&bars->o_final, 1);
     mbar_init(&bars->o_free, 4);
@@ -122,10 +124,18 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int J = 0;
+      tma_prefetch_desc(&tm_q);
+      int J = 0, it_local = 0;
       bool ok = true;
-      for (int n = blockIdx.x; n < n_items && ok; n += G) {
+      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
         const Item it = decode_item(P, n, item_off, col_off, col_rows);
+        const int qb = it_local & 1;
+        if (it_local >= 2)
+          ok = mbar_wait(&bars->q_empty[qb], ((it_local >> 1) - 1) & 1, status, abort);
+        if (!ok) break;
+        mbar_expect_tx(&bars->q_full[qb], kTileB);
+        tma_load_2d(sQ + qb * kTileB, &tm_q, &bars->q_full[qb], 0, n * kTile);
+        tma_load_2d(sQ + qb * kTileB + kHalf, &tm_q, &bars->q_full[qb], 64, n * kTile);
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + it.j * P.L + c * kTile;
           const int st = J & 1;
@@ -194,32 +204,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       }
       if (ok && J > 0) issue_pv(J - 1, prev_c, prev_it);
     }
-  } else if (warp < 4) {
-    // -------------------------------------------------------- Q gatherers
-    const int t = threadIdx.x - 64;          // 0..63
-    int it_local = 0;
-    for (int n = blockIdx.x; n < n_items; n += G, ++it_local) {
-      const int qb = it_local & 1;
-      if (it_local >= 2) {
-        const bool ok = mbar_wait(&bars->q_empty[qb], ((it_local >> 1) - 1) & 1, status, abort);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      const Item it = decode_item(P, n, item_off, col_off, col_rows);
-      uint8_t* dst = sQ + qb * kTileB;
-#pragma unroll 4
-      for (int idx = t; idx < kTile * 16; idx += 64) {
-        const int r = idx >> 4, c = idx & 15;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (r < it.count) {
-          const uint32_t i = __ldg(it.rows + r);
-          val = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)i * P.n_h + h) * kD) + c);
-        }
-        *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalf + sw128_off(r, c & 7)) = val;
-      }
-      fence_proxy_async();
-      mbar_arrive(&bars->q_full[qb]);
-    }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
@@ -374,11 +359,12 @@ size_t blk_partial_bytes(const Prob& P) {
 
 cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
-                                float scale, void* out, float* o32, float* lse, int* status,
-                                int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv;
+                                const ItemBufs& ib, float scale, void* out, float* o32,
+                                float* lse, int* status, int num_sms, cudaStream_t st) {
+  CUtensorMap tk, tv, tq;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
-  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128))
+  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
+      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_fwd_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
@@ -388,9 +374,11 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
       static_cast<char*>(part) + align_up((size_t)P.s * P.Nb * 128 * sizeof(float), 256));
   const float sl2 = scale * 1.4426950408889634f;
   for (int h = 0; h < P.n_h; ++h) {
-    k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(
-        tk, tv, P, h, static_cast<const __nv_bfloat16*>(q), sel, pv, sl2, part_o, part_ml,
-        status);
+    e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q), nullptr, ib.qg,
+                            nullptr, nullptr, nullptr, nullptr, nullptr, 0.f, num_sms, st);
+    if (e != cudaSuccess) return e;
+    k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, sel, pv, sl2, part_o,
+                                                      part_ml, status);
     k_fwd_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_o, part_ml,
                                                static_cast<__nv_bfloat16*>(out), o32, lse);
   }

@@ -94,6 +94,7 @@ struct WsLayout {
   size_t o32;            // fp32 copy of the forward output, [s][n_h][d]
   size_t pairs;          // pair lists of the selection (pairs.cu)
   size_t part;           // per-pair partial results of one head (block-major kernels)
+  size_t items;          // item-ordered Q / dO / LSE / D copies of one head
   size_t total;
 };
 
@@ -101,6 +102,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t pairs_ws_bytes(const Prob& P);
 size_t blk_partial_bytes(const Prob& P);
+size_t item_bufs_bytes(const Prob& P);
 // bf16 with head_dim 128 runs the block-major tensor-core kernels; fp32 I/O
 // (whose 1e-4 bar rules out TF32) and head_dim 64 run on the CUDA cores.
 inline bool uses_blk_path(const Prob& P) { return P.dtype == VMOBA_BF16 && P.d == 128; }
@@ -121,6 +123,7 @@ inline WsLayout ws_layout(const Prob& P) {
   w.o32 = take(sizeof(float) * (size_t)P.n_h * P.s * P.d);
   w.pairs = take(pairs_ws_bytes(P));
   w.part = take(uses_blk_path(P) ? blk_partial_bytes(P) : 0);
+  w.items = take(uses_blk_path(P) ? item_bufs_bytes(P) : 0);
   w.total = off;
   return w;
 }

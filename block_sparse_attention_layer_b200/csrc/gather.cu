@@ -1,0 +1,101 @@
+// Item-ordered copies of the rows the block-major kernels read as tiles.
+//
+// Work item n of a head (block j, query tile g of block j's list) covers rows
+// [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
+// rows past the list end are zero.  The attention kernels then fetch query
+// tiles with plain 2-D TMA instead of scattered loads.  One warp per item;
+// each lane moves 8 bytes of a 256-byte row, eight rows in flight.
+#include "common.cuh"
+#include "pairs.cuh"
+
+namespace vmoba {
+namespace {
+
+constexpr int kRowsInFlight = 8;
+
+__global__ void __launch_bounds__(256)
+k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
+               const __nv_bfloat16* __restrict__ b, __nv_bfloat16* __restrict__ ag,
+               __nv_bfloat16* __restrict__ bg, const float* __restrict__ fa,
+               const float* __restrict__ fb, float* __restrict__ fag, float* __restrict__ fbg,
+               float fa_pad) {
+  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
+  const int n_items = (int)__ldg(pv.head_totals + 2 * h + 1);
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < n_items; n += warps) {
+    int lo = 0, hi = P.Nb;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
+    }
+    const int g = n - (int)__ldg(item_off + lo);
+    const int c0 = (int)__ldg(col_off + lo), c1 = (int)__ldg(col_off + lo + 1);
+    const int count = min(kTile, c1 - c0 - g * kTile);
+    const uint32_t* rows = col_rows + c0 + g * kTile;
+    const size_t base = (size_t)n * kTile;
+    for (int r0 = 0; r0 < kTile; r0 += kRowsInFlight) {
+      uint2 va[kRowsInFlight], vb[kRowsInFlight];
+#pragma unroll
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const int r = r0 + u;
+        va[u] = make_uint2(0u, 0u);
+        vb[u] = make_uint2(0u, 0u);
+        if (r < count) {
+          const size_t src = ((size_t)__ldg(rows + r) * P.n_h + h) * 128;
+          va[u] = __ldg(reinterpret_cast<const uint2*>(a + src) + lane);
+          if (b) vb[u] = __ldg(reinterpret_cast<const uint2*>(b + src) + lane);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const size_t dst = (base + r0 + u) * 128;
+        reinterpret_cast<uint2*>(ag + dst)[lane] = va[u];
+        if (b) reinterpret_cast<uint2*>(bg + dst)[lane] = vb[u];
+      }
+    }
+    if (fa) {
+      for (int r = lane; r < kTile; r += 32) {
+        float x = fa_pad, y = 0.f;
+        if (r < count) {
+          const uint32_t i = __ldg(rows + r);
+          x = __ldg(fa + (size_t)h * P.s + i);
+          y = __ldg(fb + (size_t)h * P.s + i);
+        }
+        fag[base + r] = x;
+        fbg[base + r] = y;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t item_rows_capacity(const Prob& P) {
+  // at most one partial tile per block beyond the pairs themselves
+  return (size_t)P.s * P.Nb + (size_t)kTile * P.Nb;
+}
+
+cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
+                                const __nv_bfloat16* a, const __nv_bfloat16* b,
+                                __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
+                                const float* fb, float* fag, float* fbg, float fa_pad,
+                                int num_sms, cudaStream_t st) {
+  k_gather_items<<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg, fa_pad);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace vmoba
+
+namespace vmoba {
+
+size_t item_bufs_bytes(const Prob& P) {
+  const size_t rows = item_rows_capacity(P);
+  return 2 * align_up(rows * 128 * sizeof(__nv_bfloat16), 256) +
+         2 * align_up(rows * sizeof(float), 256);
+}
+
+}  // namespace vmoba

@@ -16,21 +16,37 @@ struct PairsView {
   int n_chunks;
 };
 
+// Item-ordered copies (gather.cu): bf16 rows of Q and dO, fp32 LSE*log2e and D.
+struct ItemBufs {
+  __nv_bfloat16* qg;
+  __nv_bfloat16* dog;
+  float* l2g;
+  float* dg;
+  size_t rows;   // capacity
+};
+
 size_t pairs_ws_bytes(const Prob& P);
 PairsView pairs_view(const Prob& P, void* base);
 cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, cudaStream_t st);
 
 cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
-                                float scale, void* out, float* o32, float* lse, int* status,
+                                const ItemBufs& ib, float scale, void* out, float* o32,
+                                float* lse, int* status, int num_sms, cudaStream_t st);
+
+size_t item_rows_capacity(const Prob& P);
+cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
+                                const __nv_bfloat16* a, const __nv_bfloat16* b,
+                                __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
+                                const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st);
 
 size_t bwd_blk_ws_bytes(const Prob& P);
 cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
-                                const float* o32, const float* lse, const void* dout, void* dq,
-                                void* dk, void* dv, void* ws_bwd, float scale, int* status,
-                                int num_sms, cudaStream_t st);
+                                const ItemBufs& ib, const float* o32, const float* lse,
+                                const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
+                                float scale, int* status, int num_sms, cudaStream_t st);
 
 // Pair slot of (query i, block j) for a selected pair: CSR offset of the row
 // plus the number of blocks below j the row selected.
