@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libvmoba.so")
 
 VMOBA_BF16 = 0
 VMOBA_F32 = 1
+STATIC_SELECT_SCRATCH_BYTES = 16 << 20   # VMOBA_STATIC_SELECT_SCRATCH_BYTES
 
 STATUS = {
     0: "VMOBA_OK", -1: "VMOBA_ERR_ARG", -2: "VMOBA_ERR_SHAPE", -3: "VMOBA_ERR_DTYPE",
@@ -95,6 +96,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_get_status": (I, [P, ctypes.POINTER(I), P]),
         "vmoba_status_string": (ctypes.c_char_p, [I]),
         "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
+        "vmoba_score_select_static": (I, [S, P, P, F, F, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -205,6 +207,19 @@ def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None)
         ctypes.byref(shape.c()), _ptr(q), _ptr(blocks), float(tau), float(scale),
         _ptr(sel_bits), _ptr(stats), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def score_select_static(shape, q, blocks, tau, scale, sel_bits, stats, stream=None):
+    """Steps 2-3 with the library's fixed static scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/vmoba.h)."""
+    import torch
+    _check_common(shape, q=q, sel_bits=sel_bits)
+    _expect(blocks, (shape.n_heads, num_blocks(shape), shape.head_dim), torch.float32, "blocks")
+    if stats.numel() * stats.element_size() < shape.n_heads * HEAD_STATS_DTYPE.itemsize:
+        raise ValueError("stats buffer too small")
+    _check("vmoba_score_select_static", lib().vmoba_score_select_static(
+        ctypes.byref(shape.c()), _ptr(q), _ptr(blocks), float(tau), float(scale),
+        _ptr(sel_bits), _ptr(stats), _stream(stream)))
 
 
 def build_plan(shape, sel_bits, ws, stream=None):

@@ -232,3 +232,85 @@ const char* vmoba_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Selection without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc when they want a selection: an engine
+// that reserves all device memory into its own pool at start-up and forbids
+// later allocations (so it cannot hand out a workspace of its own), or a
+// plugin loaded into a host program that gives it no allocator.  For them
+// vmoba_score_select_static keeps the score pool, the radix histograms and
+// the per-head search state in a fixed array of device memory that belongs
+// to the library (kStaticSelectScratch bytes on every GPU whose copy of this
+// library's device code is loaded, held until the process exits).  Only this
+// entry point uses the array; every other call keeps using caller memory.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kStaticSelectScratch = VMOBA_STATIC_SELECT_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_select_scratch[kStaticSelectScratch];
+
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxStaticDevices] = {};
+
+// Device address of the scratch array on the current device.  Host code may
+// not pass g_select_scratch itself to a kernel: on the host that name is a
+// stand-in symbol, not a device address.  Resolved once per device.
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VMOBA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxStaticDevices) return VMOBA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr)
+      return VMOBA_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return VMOBA_OK;
+}
+
+// The selection's part of the workspace layout, packed into the static array.
+WsLayout static_select_layout(const Prob& P) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  w.sel_state = take(sizeof(SelState) * P.n_h);
+  w.hist_count = take(sizeof(uint32_t) * kHistBins * P.n_h);
+  w.hist_mass = take(sizeof(double) * kHistBins * P.n_h);
+  w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const float* blocks,
+                              float tau, float scale, uint32_t* sel_bits,
+                              vmoba_head_stats* stats, cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (!(tau > 0.0f) || std::isnan(tau)) return VMOBA_ERR_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
+  const WsLayout L = static_select_layout(P);
+  if (L.total > kStaticSelectScratch) return VMOBA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((rc = static_scratch(&scratch)) != VMOBA_OK) return rc;
+  if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  const float tau_dev = tau >= 1.0f ? 2.0f : tau;
+  // the first kernel of the selection clears the histograms and the search
+  // state; the score pool is fully overwritten before it is read
+  return cuda_status(
+      launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, scratch, L, stream));
+}
+
+}  // extern "C"

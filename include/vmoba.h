@@ -68,6 +68,9 @@ typedef enum vmoba_status {
 
 enum { VMOBA_BF16 = 0, VMOBA_F32 = 1 };
 
+/* Size of the library-owned device scratch of vmoba_score_select_static. */
+#define VMOBA_STATIC_SELECT_SCRATCH_BYTES ((size_t)16 << 20)
+
 /* One layer's problem.  mode: 0 = 1D (box bt x H x W), 1 = 2D (T x bh x bw),
  * 2 = 3D (bt x bh x bw); the fields the mode does not use are ignored.
  * head_dim must be 64 or 128. */
@@ -161,6 +164,32 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
 /* Reads the workspace's device status word (synchronises the stream) into
  * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it. */
 int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream);
+
+/* Selection for callers that cannot allocate device memory.
+ * Same contract and results as vmoba_score_select, but the score pool, the
+ * radix histograms and the per-head search state live in a fixed 16 MiB
+ * array of device memory owned by the library (reserved on every GPU where
+ * the library's device code is loaded, until the process exits), so no
+ * workspace is passed and nothing is allocated.  Meant for callers such as
+ * an engine that has pooled all device memory at start-up and forbids later
+ * cudaMalloc, or a plugin that is given no allocator.  This entry point has
+ * no counterpart in the paper: it only changes where scratch memory lives.
+ * - Problems whose scratch exceeds VMOBA_STATIC_SELECT_SCRATCH_BYTES return
+ *   VMOBA_ERR_WORKSPACE without launching anything.  The scratch is the fp32
+ *   score pool (4*n_heads*s*N_b bytes) plus about 24.6 KB per head of
+ *   histograms and search state; e.g. 4 heads x 2048 tokens x 64 blocks
+ *   (2.1 MB) fits, 12 heads x 55296 tokens x 24 blocks (64 MB) does not.
+ * - The first call on a device looks up the array's device address on that
+ *   device (a CUDA runtime query); make that first call before any stream
+ *   capture.
+ * - Every call on a device shares the one array: calls that may run at the
+ *   same time on the GPU (different streams, other host threads) race and
+ *   corrupt each other's results.  Serialise them.
+ * - Inputs and outputs (q, blocks, sel_bits, stats) are caller memory, as in
+ *   vmoba_score_select. */
+int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const float* blocks,
+                              float tau, float scale, uint32_t* sel_bits,
+                              vmoba_head_stats* stats, cudaStream_t stream);
 
 /* Number of CUDA kernels this library has launched since it was loaded
  * (host-side counter, thread-safe; diagnostics for launch accounting). */
