@@ -206,6 +206,8 @@ def run_ours(args, rank, world, local):
     K = args.steps
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in layers]
            for _ in range(K)]
+    V.trace_read()                 # drop anything traced before the timed region
+    V.trace_enable(True)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -218,6 +220,8 @@ def run_ours(args, rank, world, local):
         end.record(stream)
         torch.cuda.synchronize()
     launches = V.kernel_launches() - n_launch0
+    V.trace_enable(False)
+    trace = V.trace_read()         # per-kernel device time over the timed region
     if world > 1:
         dist.barrier()
     elapsed_ms = start.elapsed_time(end)
@@ -245,25 +249,37 @@ def run_ours(args, rank, world, local):
         elapsed_max = elapsed_ms
     value = total_flops / (elapsed_max * 1e-3) / 1e12
 
-    # roofline: the dominant call of the step
+    # roofline of the dominant kernel (by device time over the timed region):
+    # algorithmic work per launch summed over the step / its traced time
     s, nh = w.s, w.n_heads
-    fwd_flops = sum(metrics.attention_flops(p, d, True, False) for p in pairs)
-    bwd_flops = sum(metrics.attention_flops(p, d, False, True) for p in pairs)
-    achieved = {
-        "attn_bwd": (bwd_flops / (call_ms["attn_bwd"] * 1e-3) / 1e12, "TFLOP/s", "tensor"),
-        "attn_fwd": (fwd_flops / (call_ms["attn_fwd"] * 1e-3) / 1e12, "TFLOP/s", "tensor"),
-    }
+    flops_per_pair = {"k_fwd_blk": 4 * d, "k_bwd_dq_blk": 6 * d, "k_bwd_dkdv_blk": 8 * d}
+    tot_pairs = sum(pairs)
+    kern = {}
+    for name, (n_launch, ms) in trace.items():
+        kern[name] = {"launches_per_step": n_launch / K, "ms_per_step": round(ms / K, 4)}
+        if name in flops_per_pair and ms > 0:
+            kern[name]["tflops"] = round(flops_per_pair[name] * tot_pairs * K / (ms * 1e-3) / 1e12, 2)
+    dom = max(trace, key=lambda n: trace[n][1]) if trace else None
     part_bytes = sum(metrics.partition_bytes(s, nh, d, 2, V.num_blocks(sh)) for sh in shapes)
     sel_bytes = sum(metrics.select_bytes(s, nh, V.num_blocks(sh)) for sh in shapes)
-    achieved["partition"] = (part_bytes / (call_ms["partition"] * 1e-3) / 1e9, "GB/s", "hbm")
-    achieved["score_select"] = (sel_bytes / (call_ms["score_select"] * 1e-3) / 1e9, "GB/s", "hbm")
-    dom = max(("attn_bwd", "attn_fwd"), key=lambda c: call_ms[c])
-    a, unit, bound = achieved[dom]
-    peak = peaks["bf16_sus"] if bound == "tensor" else peaks["hbm"]
-    roofline = {"bound": bound, "achieved": round(a, 3), "peak": peak, "unit": unit,
-                "frac": round(a / peak, 5), "traffic": None, "kernel": dom,
-                "peak_source": f"{peaks['src']} (sustained bf16)" if bound == "tensor"
-                else f"{peaks['src']} hbm"}
+    achieved = {
+        "attn_bwd_call": (metrics.attention_flops(tot_pairs, d, False, True)
+                          / (call_ms["attn_bwd"] * 1e-3) / 1e12, "TFLOP/s"),
+        "attn_fwd_call": (metrics.attention_flops(tot_pairs, d, True, False)
+                          / (call_ms["attn_fwd"] * 1e-3) / 1e12, "TFLOP/s"),
+        "partition_call": (part_bytes / (call_ms["partition"] * 1e-3) / 1e9, "GB/s"),
+        "score_select_call": (sel_bytes / (call_ms["score_select"] * 1e-3) / 1e9, "GB/s"),
+    }
+    roofline = None
+    if dom in flops_per_pair:
+        a = kern[dom]["tflops"]
+        peak = peaks["bf16_sus"]
+        roofline = {"bound": "tensor", "achieved": a, "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(a / peak, 5), "traffic": kernel_traffic(dom, w),
+                    "kernel": dom,
+                    "algorithmic": f"{flops_per_pair[dom] // d}*d FLOPs per selected "
+                                   f"(query, key) pair, {tot_pairs} pairs per step",
+                    "peak_source": f"{peaks['src']} bf16 sustained (kernel timed inside a long step)"}
 
     e2e = None
     if not args.no_e2e:
@@ -296,6 +312,7 @@ def run_ours(args, rank, world, local):
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
                                   for i, l in enumerate(LAYERS)},
                 "achieved": {c: [round(x[0], 3), x[1]] for c, x in achieved.items()},
+                "kernels": kern,
                 "density": [round(x, 5) for x in density],
                 "selected_token_pairs": pairs,
                 "flops_per_step": flops_step,
@@ -305,6 +322,30 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def kernel_traffic(name, w):
+    """DRAM bytes per launch of ``name`` from the committed ncu summary, or None
+    when the kernel's source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "kernel_traffic.md")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = line.split("|")
+        if len(parts) < 6 or parts[1].strip() != name:
+            continue
+        src, digest, nbytes = parts[2].strip(), parts[3].strip(), parts[4].strip()
+        fpath = os.path.join(ROOT, "block_sparse_attention_layer_b200", "csrc", src)
+        if not os.path.exists(fpath):
+            return None
+        if hashlib.sha256(open(fpath, "rb").read()).hexdigest()[:16] != digest:
+            return None
+        try:
+            return float(nbytes)
+        except ValueError:
+            return None
+    return None
 
 
 def run_e2e(args, layers, host, flops_step, world):

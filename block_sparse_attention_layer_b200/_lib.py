@@ -41,6 +41,10 @@ class CShape(ctypes.Structure):
                 ("dtype", ctypes.c_int)]
 
 
+class TraceEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int), ("ms", ctypes.c_double)]
+
+
 HEAD_STATS_DTYPE = np.dtype([("n_selected", "<i8"), ("mass", "<f8"), ("cut_score", "<f4"),
                              ("all_selected", "<i4")])
 
@@ -97,6 +101,8 @@ def lib() -> ctypes.CDLL:
         "vmoba_status_string": (ctypes.c_char_p, [I]),
         "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
         "vmoba_score_select_static": (I, [S, P, P, F, F, P, P, P]),
+        "vmoba_trace_enable": (I, [I]),
+        "vmoba_trace_read": (I, [ctypes.POINTER(TraceEntry), I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -261,6 +267,18 @@ def get_status(ws, stream=None) -> int:
     v = ctypes.c_int(0)
     _check("vmoba_get_status", lib().vmoba_get_status(_ptr(ws), ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def trace_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (per-kernel timing)."""
+    lib().vmoba_trace_enable(1 if on else 0)
+
+
+def trace_read() -> dict:
+    """{kernel name: (launches, device ms)} since the last read; clears the trace."""
+    buf = (TraceEntry * 256)()
+    n = lib().vmoba_trace_read(buf, len(buf))
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].ms) for i in range(min(n, len(buf)))}
 
 
 def kernel_launches() -> int:

@@ -580,8 +580,11 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws_bwd) +
                                          align_up(sizeof(float) * (size_t)P.n_h * P.s, 256));
   const int warps = P.s * P.n_h;
-  k_bwd_rows<<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const __nv_bfloat16*>(dout),
-                                              lse, rowD, lse2);
+  {
+    VMOBA_TRACE("k_bwd_rows", st);
+    k_bwd_rows<<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const __nv_bfloat16*>(dout),
+                                                lse, rowD, lse2);
+  }
   cudaError_t e = cudaFuncSetAttribute(k_bwd_dq_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kDqSmem);
   if (e != cudaSuccess) return e;
@@ -597,13 +600,22 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
                             static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, lse2, rowD,
                             ib.l2g, ib.dg, INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
-    k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, sel, pv, ib.dg,
-                                                      ib.l2g, sl2, part_dq, status);
-    k_bwd_dq_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
-                                                  static_cast<__nv_bfloat16*>(dq));
-    k_bwd_dkdv_blk<<<P.Nb * nkt, kThreads, kKvSmem, st>>>(
-        tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), status);
+    {
+      VMOBA_TRACE("k_bwd_dq_blk", st);
+      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, sel, pv, ib.dg,
+                                                        ib.l2g, sl2, part_dq, status);
+    }
+    {
+      VMOBA_TRACE("k_bwd_dq_merge", st);
+      k_bwd_dq_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
+                                                    static_cast<__nv_bfloat16*>(dq));
+    }
+    {
+      VMOBA_TRACE("k_bwd_dkdv_blk", st);
+      k_bwd_dkdv_blk<<<P.Nb * nkt, kThreads, kKvSmem, st>>>(
+          tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
+          static_cast<__nv_bfloat16*>(dv), status);
+    }
   }
   count_launches(1 + 3 * P.n_h);
   return cudaGetLastError();

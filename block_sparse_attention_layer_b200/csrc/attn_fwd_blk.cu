@@ -377,10 +377,16 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
     e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q), nullptr, ib.qg,
                             nullptr, nullptr, nullptr, nullptr, nullptr, 0.f, num_sms, st);
     if (e != cudaSuccess) return e;
-    k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, sel, pv, sl2, part_o,
-                                                      part_ml, status);
-    k_fwd_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_o, part_ml,
-                                               static_cast<__nv_bfloat16*>(out), o32, lse);
+    {
+      VMOBA_TRACE("k_fwd_blk", st);
+      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, sel, pv, sl2, part_o,
+                                                        part_ml, status);
+    }
+    {
+      VMOBA_TRACE("k_fwd_merge", st);
+      k_fwd_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_o, part_ml,
+                                                 static_cast<__nv_bfloat16*>(out), o32, lse);
+    }
   }
   count_launches(2 * P.n_h);
   return cudaGetLastError();

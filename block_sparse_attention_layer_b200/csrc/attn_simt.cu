@@ -368,9 +368,12 @@ cudaError_t fwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(P.n_qt, P.n_h);
-  k_fwd_simt<E, D><<<grid, kTile * (D / 32), smem, st>>>(
-      P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
-      qt_kt, scale, static_cast<E*>(out), o32, lse);
+  {
+    VMOBA_TRACE("k_fwd_simt", st);
+    k_fwd_simt<E, D><<<grid, kTile * (D / 32), smem, st>>>(
+        P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
+        qt_kt, scale, static_cast<E*>(out), o32, lse);
+  }
   count_launches(1);
   return cudaGetLastError();
 }
@@ -381,8 +384,11 @@ cudaError_t bwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
                   const float* o32, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, float* rowD, cudaStream_t st) {
   const int warps = P.s * P.n_h;
-  k_bwd_rowdot<E, D><<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const E*>(dout),
-                                                       rowD);
+  {
+    VMOBA_TRACE("k_bwd_rowdot", st);
+    k_bwd_rowdot<E, D><<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const E*>(dout),
+                                                         rowD);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t s1 = fwd_smem<D>(P);
@@ -390,9 +396,12 @@ cudaError_t bwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
                            (int)s1);
   if (e != cudaSuccess) return e;
   dim3 grid(P.n_qt, P.n_h);
-  k_bwd_dq_simt<E, D><<<grid, kTile * (D / 32), s1, st>>>(
-      P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
-      qt_kt, scale, lse, static_cast<const E*>(dout), rowD, static_cast<E*>(dq));
+  {
+    VMOBA_TRACE("k_bwd_dq_simt", st);
+    k_bwd_dq_simt<E, D><<<grid, kTile * (D / 32), s1, st>>>(
+        P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
+        qt_kt, scale, lse, static_cast<const E*>(dout), rowD, static_cast<E*>(dq));
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr int KR = D == 128 ? 64 : 128;
@@ -401,10 +410,13 @@ cudaError_t bwd_t(const Prob& P, const void* q, const void* kp, const void* vp,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
   if (e != cudaSuccess) return e;
   dim3 kgrid(P.n_qt * (kTile / KR), P.n_h);
-  k_bwd_dkdv_simt<E, D, KR><<<kgrid, KR * (D / 32), s2, st>>>(
-      P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
-      kt_qt, scale, lse, static_cast<const E*>(dout), rowD, static_cast<E*>(dk),
-      static_cast<E*>(dv));
+  {
+    VMOBA_TRACE("k_bwd_dkdv_simt", st);
+    k_bwd_dkdv_simt<E, D, KR><<<kgrid, KR * (D / 32), s2, st>>>(
+        P, static_cast<const E*>(q), static_cast<const E*>(kp), static_cast<const E*>(vp), sel,
+        kt_qt, scale, lse, static_cast<const E*>(dout), rowD, static_cast<E*>(dk),
+        static_cast<E*>(dv));
+  }
   count_launches(3);
   return cudaGetLastError();
 }

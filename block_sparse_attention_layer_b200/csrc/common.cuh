@@ -131,6 +131,19 @@ inline WsLayout ws_layout(const Prob& P) {
 template <typename T>
 inline T* ws_ptr(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
+// Brackets one kernel launch with CUDA events on its stream while tracing is
+// enabled (vmoba_trace_enable); a no-op otherwise.
+class TraceScope {
+ public:
+  TraceScope(const char* name, cudaStream_t st);
+  ~TraceScope();
+ private:
+  cudaStream_t stream_;
+  void* a_;
+  const char* name_ = nullptr;
+};
+#define VMOBA_TRACE(name, st) ::vmoba::TraceScope _vmoba_trace_scope_((name), (st))
+
 // Kernels launched by this library since load (diagnostics; see
 // vmoba_kernel_launches).  Every launch wrapper adds what it launched.
 void count_launches(int n);

@@ -83,7 +83,10 @@ cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st) {
-  k_gather_items<<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg, fa_pad);
+  {
+    VMOBA_TRACE("k_gather_items", st);
+    k_gather_items<<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg, fa_pad);
+  }
   count_launches(1);
   return cudaGetLastError();
 }

@@ -198,10 +198,19 @@ PairsView pairs_view(const Prob& P, void* base) {
 
 cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, cudaStream_t st) {
   dim3 g(v.n_chunks, P.n_h);
-  k_pairs_count<<<g, kChunkRows, 0, st>>>(P, sel, v.row_cnt, v.chunk, v.n_chunks);
-  k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
-                                       v.item_off, v.head_totals);
-  k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.col_rows);
+  {
+    VMOBA_TRACE("k_pairs_count", st);
+    k_pairs_count<<<g, kChunkRows, 0, st>>>(P, sel, v.row_cnt, v.chunk, v.n_chunks);
+  }
+  {
+    VMOBA_TRACE("k_pairs_scan", st);
+    k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
+                                         v.item_off, v.head_totals);
+  }
+  {
+    VMOBA_TRACE("k_pairs_fill", st);
+    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.col_rows);
+  }
   count_launches(3);
   return cudaGetLastError();
 }

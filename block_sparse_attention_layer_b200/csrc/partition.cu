@@ -89,9 +89,12 @@ template <typename E, int D>
 cudaError_t launch_t(const Prob& P, const void* k, const void* v, void* kp, void* vp,
                      float* blocks, cudaStream_t st) {
   dim3 grid(P.Nb, P.n_h);
-  k_partition_pool<E, D><<<grid, kWarps * 32, 0, st>>>(
-      P, static_cast<const E*>(k), static_cast<const E*>(v), static_cast<E*>(kp),
-      static_cast<E*>(vp), blocks);
+  {
+    VMOBA_TRACE("k_partition_pool", st);
+    k_partition_pool<E, D><<<grid, kWarps * 32, 0, st>>>(
+        P, static_cast<const E*>(k), static_cast<const E*>(v), static_cast<E*>(kp),
+        static_cast<E*>(vp), blocks);
+  }
   count_launches(1);
   return cudaGetLastError();
 }

@@ -91,9 +91,15 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   uint32_t* kt_work = ws_ptr<uint32_t>(ws, L.kt_work);
   const size_t nbw = (size_t)P.n_h * P.n_qt * P.Wqt;
   const size_t nw = (size_t)P.n_h * P.n_qt;
-  k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw);
+  {
+    VMOBA_TRACE("k_plan_clear", st);
+    k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw);
+  }
   dim3 grid(P.n_qt, P.n_h);
-  k_plan_tiles<<<grid, kTile, 0, st>>>(P, sel, qt_kt, qt_work, kt_qt, kt_work);
+  {
+    VMOBA_TRACE("k_plan_tiles", st);
+    k_plan_tiles<<<grid, kTile, 0, st>>>(P, sel, qt_kt, qt_work, kt_qt, kt_work);
+  }
   count_launches(2);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -390,7 +390,10 @@ cudaError_t launch_score(const Prob& P, const void* q, const float* B, float sca
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((P.s + kSQ - 1) / kSQ, P.n_h);
-  k_score<E, D><<<grid, 256, smem, stream>>>(P, static_cast<const E*>(q), B, scale, S, st);
+  {
+    VMOBA_TRACE("k_score", stream);
+    k_score<E, D><<<grid, 256, smem, stream>>>(P, static_cast<const E*>(q), B, scale, S, st);
+  }
   return cudaGetLastError();
 }
 
@@ -404,7 +407,10 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   double* hm = ws_ptr<double>(ws, L.hist_mass);
   float* S = ws_ptr<float>(ws, L.scores);
 
-  k_init<<<64, 256, 0, stream>>>(st, hc, hm, P.n_h);
+  {
+    VMOBA_TRACE("k_init", stream);
+    k_init<<<64, 256, 0, stream>>>(st, hc, hm, P.n_h);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (P.dtype == VMOBA_BF16)
@@ -417,21 +423,63 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
 
   const size_t pool = (size_t)P.s * P.Nb;
   dim3 hgrid((unsigned)((pool + kHistChunk - 1) / kHistChunk), P.n_h);
-  k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-  k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
-  k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-  k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
-  k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-  k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
-  k_tie_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  k_tie_scan<0><<<P.n_h, 32, 0, stream>>>(st, hc);
-  k_tie_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  k_tie_scan<1><<<P.n_h, 32, 0, stream>>>(st, hc);
-  k_tie_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  k_tie_scan<2><<<P.n_h, 32, 0, stream>>>(st, hc);
+  {
+    VMOBA_TRACE("k_hist", stream);
+    k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  }
+  {
+    VMOBA_TRACE("k_scan", stream);
+    k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  }
+  {
+    VMOBA_TRACE("k_hist", stream);
+    k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  }
+  {
+    VMOBA_TRACE("k_scan", stream);
+    k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  }
+  {
+    VMOBA_TRACE("k_hist", stream);
+    k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  }
+  {
+    VMOBA_TRACE("k_scan", stream);
+    k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+  }
+  {
+    VMOBA_TRACE("k_tie_hist", stream);
+    k_tie_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  }
+  {
+    VMOBA_TRACE("k_tie_scan", stream);
+    k_tie_scan<0><<<P.n_h, 32, 0, stream>>>(st, hc);
+  }
+  {
+    VMOBA_TRACE("k_tie_hist", stream);
+    k_tie_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  }
+  {
+    VMOBA_TRACE("k_tie_scan", stream);
+    k_tie_scan<1><<<P.n_h, 32, 0, stream>>>(st, hc);
+  }
+  {
+    VMOBA_TRACE("k_tie_hist", stream);
+    k_tie_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+  }
+  {
+    VMOBA_TRACE("k_tie_scan", stream);
+    k_tie_scan<2><<<P.n_h, 32, 0, stream>>>(st, hc);
+  }
   dim3 egrid((P.s + 31) / 32, P.n_h);
-  k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
-  k_stats<<<1, 128, 0, stream>>>(P, st, stats);
+  {
+    VMOBA_TRACE("k_emit", stream);
+    k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
+  }
+  {
+    VMOBA_TRACE("k_stats", stream);
+    k_stats<<<1, 128, 0, stream>>>(P, st, stats);
+  }
   count_launches(16);
   return cudaGetLastError();
 }

@@ -195,6 +195,22 @@ int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const flo
  * (host-side counter, thread-safe; diagnostics for launch accounting). */
 unsigned long long vmoba_kernel_launches(void);
 
+/* Per-kernel device timing (diagnostics).  While enabled, every kernel the
+ * library launches is bracketed by two CUDA events on its own stream. */
+typedef struct vmoba_trace_entry {
+  char name[48];        /* kernel name */
+  int launches;         /* launches since the last read */
+  double ms;            /* summed device time of those launches */
+} vmoba_trace_entry;
+
+/* Turns tracing on (nonzero) or off.  Always VMOBA_OK. */
+int vmoba_trace_enable(int on);
+
+/* Waits for the traced launches, writes up to max_entries aggregated
+ * entries (one per kernel name) and clears the trace.  Returns the number of
+ * distinct kernel names (may exceed max_entries; out may be NULL). */
+int vmoba_trace_read(vmoba_trace_entry* out, int max_entries);
+
 /* Static text of a vmoba_status code. */
 const char* vmoba_status_string(int status);
 
