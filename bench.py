@@ -121,6 +121,25 @@ def dist_env():
     return rank, world, local
 
 
+def reduce_over_ranks(elapsed_ms: float, flops: float, device) -> tuple:
+    """(max elapsed over ranks, summed FLOPs over ranks): the job's time is the
+    slowest rank's and its work is every rank's sample (weak scaling)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(elapsed_ms), float(flops)
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    f = torch.tensor([flops], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(f[0])
+
+
+def rank_sample(rank: int) -> int:
+    """Synthetic sample (seed family) of a data-parallel rank: one per rank."""
+    return rank
+
+
 # ---------------------------------------------------------------- inputs
 def host_inputs(sample: int):
     """bf16 host tensors (pinned) of one synthetic sample: q, k, v, dout."""
@@ -167,7 +186,7 @@ def run_ours(args, rank, world, local):
     w, shapes = layer_shapes()
     peaks = load_peaks()
     t0 = time.time()
-    hq, hk, hv, hdo = host_inputs(sample=rank)
+    hq, hk, hv, hdo = host_inputs(sample=rank_sample(rank))
     gen_s = time.time() - t0
     q, k, v, dout = (x.cuda(non_blocking=False) for x in (hq, hk, hv, hdo))
     layers = [VMoBALayer(sh) for sh in shapes]
@@ -237,16 +256,7 @@ def run_ours(args, rank, world, local):
                 call_ms[c] += t / K
                 layer_call_ms[li][ci] += t / K
 
-    total_flops = flops_step * K
-    if world > 1:
-        tt = torch.tensor([elapsed_ms, total_flops], dtype=torch.float64, device="cuda")
-        mx = tt.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tt, op=dist.ReduceOp.SUM)
-        elapsed_max = float(mx[0])
-        total_flops = float(tt[1])
-    else:
-        elapsed_max = elapsed_ms
+    elapsed_max, total_flops = reduce_over_ranks(elapsed_ms, flops_step * K, "cuda")
     value = total_flops / (elapsed_max * 1e-3) / 1e12
 
     # roofline of the dominant kernel (by device time over the timed region):
@@ -376,11 +386,7 @@ def run_e2e(args, layers, host, flops_step, world):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    ms, _ = reduce_over_ranks(ms, 0.0, "cuda")
     nbytes = hq.numel() * hq.element_size()
     return {"value": round(flops_step * K * world / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
             "h2d_bytes_per_step": 4 * nbytes * len(layers),
