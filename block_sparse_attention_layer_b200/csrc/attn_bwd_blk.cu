@@ -25,7 +25,14 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr uint32_t kHalf = 128 * 64 * 2;
 constexpr uint32_t kTileB = 2 * kHalf;
-constexpr int kThreads = 256;
+// 384 threads: warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 two softmax
+// warpgroups that split each tile's 128 columns 64/64 (a warp reaches TMEM
+// lanes 32*(warp % 4) .. +32, so both groups cover all 128 rows).
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarps = 8;
+// Column of the packed bf16 operand (P, P^T, dS, dS^T) for 16-wide step kk:
+// group g writes its 64 columns, packed two per 32-bit column, at 64 g.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -114,13 +121,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->full_k[i], 1); mbar_init(&bars->empty_k[i], 1);
       mbar_init(&bars->full_v[i], 1); mbar_init(&bars->empty_v[i], 1);
-      mbar_init(&bars->s_full[i], 1); mbar_init(&bars->ds_full[i], 4);
+      mbar_init(&bars->s_full[i], 1); mbar_init(&bars->ds_full[i], kSoftmaxWarps);
     }
-    mbar_init(&bars->s_free, 4);
+    mbar_init(&bars->s_free, kSoftmaxWarps);
     mbar_init(&bars->qd_full, 1);
     mbar_init(&bars->qd_empty, 1);
     mbar_init(&bars->dq_final, 1);
-    mbar_init(&bars->dq_free, 4);
+    mbar_init(&bars->dq_free, kSoftmaxWarps);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -185,7 +192,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         const uint32_t tdS = tmem + 128 + b * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDQ, tdS + kk * 8, desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
+          mma_ts(tDQ, tdS + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
                  (cp > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty_k[b]);
         if (cp == nch - 1) mma_commit(&bars->dq_final);
@@ -226,8 +233,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       if (ok && J > 0) issue_dq(J - 1, prev_c, prev_it);
     }
   } else if (warp >= 4) {
-    const int wq = warp - 4;
+    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, column group
     const int r = wq * 32 + lane;
+    const int cb = 64 * wg;                         // this group's key columns
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     int J = 0, it_local = 0;
     bool ok = true;
@@ -246,38 +254,36 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, status, abort));
         if (!ok) break;
         tc_fence_after();
-        const int lim = P.L - c * kTile;
-        const bool full = lim >= kTile;
-        // S row: four loads, one wait; P in place
-        uint32_t xr[128];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + lane_off + c4 * 32, xr + c4 * 32);
+        const int lim = P.L - c * kTile - cb;       // valid columns of this group
+        const bool full = lim >= 64;
+        uint32_t xr[64];
+        tmem_ld32(tS + lane_off + cb, xr);
+        tmem_ld32(tS + lane_off + cb + 32, xr + 32);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
+        for (int e = 0; e < 64; ++e) {
           const bool on = valid && (full || e < lim);
-          xr[e] = __float_as_uint(on ? exp2f(fmaf(__uint_as_float(xr[e]), sl2, -l2)) : 0.f);
+          xr[e] = __float_as_uint(on ? fast_exp2(fmaf(__uint_as_float(xr[e]), sl2, -l2)) : 0.f);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free);       // S may be overwritten now
-        const uint32_t tdP = tmem + 128 + b * 128 + lane_off;
+        const uint32_t tdP = tmem + 128 + b * 128 + lane_off + cb;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {                  // dP in two halves of 64 columns
-          uint32_t dp[64];
-          tmem_ld32(tdP + hh * 64, dp);
-          tmem_ld32(tdP + hh * 64 + 32, dp + 32);
+        for (int hh = 0; hh < 2; ++hh) {                  // 32 dP columns per wait
+          uint32_t dp[32];
+          tmem_ld32(tdP + hh * 32, dp);
           tmem_ld_wait();
-          uint32_t pk[32];
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const float d0 = __uint_as_float(xr[hh * 64 + e]) * (__uint_as_float(dp[e]) - Di);
+          for (int e = 0; e < 32; e += 2) {
+            const float d0 = __uint_as_float(xr[hh * 32 + e]) * (__uint_as_float(dp[e]) - Di);
             const float d1 =
-                __uint_as_float(xr[hh * 64 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di);
+                __uint_as_float(xr[hh * 32 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di);
             pk[e >> 1] = pack_bf16x2(d0, d1);
           }
-          // dS columns [32 hh, 32 hh + 32): dP columns already read
-          tmem_st32(tdP + hh * 32, pk);
+          // dS into the group's columns [cb + 16 hh, +16): dP columns already read
+          tmem_st16(tdP + hh * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -292,12 +298,12 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       if (valid)
         slot = pair_slot(row_off, sel + ((size_t)h * P.s + i) * P.Wb, P.Wb, (int)i, it.j);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {               // this group's 64 dQ columns
         uint32_t xr[32];
-        tmem_ld32(tDQ + lane_off + cc * 32, xr);
+        tmem_ld32(tDQ + lane_off + cb + cc * 32, xr);
         tmem_ld_wait();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(part_dq + slot * kD + cc * 32);
+          float4* dst = reinterpret_cast<float4*>(part_dq + slot * kD + cb + cc * 32);
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             dst[e / 4] = make_float4(__uint_as_float(xr[e]), __uint_as_float(xr[e + 1]),
@@ -388,7 +394,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     mbar_init(&bars->kv_full, 1);
     for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
     mbar_init(&bars->st_full, 1);
-    mbar_init(&bars->pd_full, 4);
+    mbar_init(&bars->pd_full, kSoftmaxWarps);
     mbar_init(&bars->acc_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -456,9 +462,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         // dV += P^T dO, dK += dS^T Q (queries are the reduction dim, MN-major B)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tV, tS + kk * 8, desc_sw128(ob + kk * 2048, kHalf, 1024), idAcc,
+          mma_ts(tV, tS + packed_col(kk), desc_sw128(ob + kk * 2048, kHalf, 1024), idAcc,
                  (g > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tK, tP + kk * 8, desc_sw128(qb + kk * 2048, kHalf, 1024), idAcc,
+          mma_ts(tK, tP + packed_col(kk), desc_sw128(qb + kk * 2048, kHalf, 1024), idAcc,
                  (g > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->qd_empty[b]);
@@ -466,8 +472,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (ok) mma_commit(&bars->acc_final);
     }
   } else if (warp >= 4) {
-    const int wq = warp - 4;
+    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
     const int c = wq * 32 + lane;                     // key row of this thread
+    const int cb = 64 * wg;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const bool kvalid = c < nkeys;
     bool ok = true;
@@ -479,33 +486,32 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, status, abort));
       if (!ok) break;
       tc_fence_after();
-      const float* L2 = sL + b * kTile;
-      const float* Dq = sD + b * kTile;
+      const float* L2 = sL + b * kTile + cb;
+      const float* Dq = sD + b * kTile + cb;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {                 // 64 query columns per wait
-        uint32_t xs[64], xp[64];
-        tmem_ld32(tS + lane_off + hh * 64, xs);
-        tmem_ld32(tS + lane_off + hh * 64 + 32, xs + 32);
-        tmem_ld32(tP + lane_off + hh * 64, xp);
-        tmem_ld32(tP + lane_off + hh * 64 + 32, xp + 32);
+      for (int hh = 0; hh < 2; ++hh) {                 // 32 query columns per wait
+        uint32_t xs[32], xp[32];
+        tmem_ld32(tS + lane_off + cb + hh * 32, xs);
+        tmem_ld32(tP + lane_off + cb + hh * 32, xp);
         tmem_ld_wait();
-        uint32_t pp[32], pd[32];
+        uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
+        for (int e = 0; e < 32; e += 2) {
           float pv2[2], dv2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qi = hh * 64 + e + u;
-            const float pr = kvalid ? exp2f(fmaf(__uint_as_float(xs[e + u]), sl2, -L2[qi])) : 0.f;
+            const int qi = hh * 32 + e + u;
+            const float pr =
+                kvalid ? fast_exp2(fmaf(__uint_as_float(xs[e + u]), sl2, -L2[qi])) : 0.f;
             pv2[u] = pr;
             dv2[u] = pr * (__uint_as_float(xp[e + u]) - Dq[qi]);
           }
           pp[e >> 1] = pack_bf16x2(pv2[0], pv2[1]);
           pd[e >> 1] = pack_bf16x2(dv2[0], dv2[1]);
         }
-        // P^T, dS^T columns [32 hh, 32 hh + 32): S^T / dP^T columns already read
-        tmem_st32(tS + lane_off + hh * 32, pp);
-        tmem_st32(tP + lane_off + hh * 32, pd);
+        // P^T, dS^T into the group's columns [cb + 16 hh, +16) (already read)
+        tmem_st16(tS + lane_off + cb + hh * 16, pp);
+        tmem_st16(tP + lane_off + cb + hh * 16, pd);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -519,8 +525,8 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (have) tc_fence_after();
       const int pk = key0 + c;
       const int n = kvalid ? perm_token(P, pk) : 0;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {            // half 0: dK, half 1: dV
+      {                                               // group 0: dV, group 1: dK
+        const int half = wg == 0 ? 1 : 0;
         const uint32_t base = half == 0 ? tK : tV;
         const float f = half == 0 ? scale : 1.0f;
         __nv_bfloat16* dst = (half == 0 ? dk : dv) + ((size_t)n * P.n_h + h) * kD;
