@@ -56,27 +56,6 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
   }
 }
 
-struct QItem {
-  int j, count;
-  const uint32_t* rows;
-};
-
-__device__ __forceinline__ QItem decode_qitem(const Prob& P, int n, const uint32_t* item_off,
-                                              const uint32_t* col_off, const uint32_t* col_rows) {
-  int lo = 0, hi = P.Nb;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
-  }
-  QItem it;
-  it.j = lo;
-  const int g = n - (int)__ldg(item_off + lo);
-  const int c0 = (int)__ldg(col_off + lo), c1 = (int)__ldg(col_off + lo + 1);
-  it.count = min(kTile, c1 - c0 - g * kTile);
-  it.rows = col_rows + c0 + g * kTile;
-  return it;
-}
-
 // =====================================================================
 // dQ pass.  TMEM: S [0,128), dP0 [128,256), dP1 [256,384), dQ [384,512).
 // Roles: warp 0 TMA (the item's Q and dO tiles from the item-ordered copies,
@@ -90,13 +69,15 @@ struct DqBars {
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kDqSmem = 1024 + 2 * kTileB /*Q,dO*/ + 4 * kTileB /*K,V x2*/ + sizeof(DqBars) + 64;
+constexpr uint32_t kStageB = 32 * 32 * 4;     // epilogue staging per softmax warp
+constexpr size_t kDqSmem = 1024 + 2 * kTileB /*Q,dO*/ + 4 * kTileB /*K,V x2*/ + 8 * kStageB +
+                           sizeof(DqBars) + 64;
+static_assert(kDqSmem <= 232448, "shared memory per CTA");
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-             Prob P, int h, const uint32_t* __restrict__ sel, PairsView pv,
-             const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
+             Prob P, int h, PairsView pv, const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
              float* __restrict__ part_dq, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -105,16 +86,15 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   uint8_t* sO = sQ + kTileB;              // dO tile
   uint8_t* sK = sO + kTileB;              // 2 stages
   uint8_t* sV = sK + 2 * kTileB;          // 2 stages
-  DqBars* bars = reinterpret_cast<DqBars*>(sV + 2 * kTileB);
+  uint8_t* sStage = sV + 2 * kTileB;      // 8 x kStageB
+  DqBars* bars = reinterpret_cast<DqBars*>(sStage + 8 * kStageB);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
-  const uint32_t* row_off = pv.row_off + (size_t)h * (P.s + 1);
-  const int n_items = (int)__ldg(pv.head_totals + 2 * h + 1);
+  const uint32_t* col_slot = pv.col_slot + (size_t)h * P.s * P.Nb;
+  const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int nch = (P.L + kTile - 1) / kTile;
+  const int kc_last = P.L - (nch - 1) * kTile;        // keys in the last chunk
   const int G = gridDim.x;
 
   if (threadIdx.x == 0) {
@@ -150,7 +130,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       int J = 0, it_local = 0;
       bool ok = true;
       for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-        const QItem it = decode_qitem(P, n, item_off, col_off, col_rows);
+        const WorkItem it = decode_item(pv, P, h, n);
         if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, status, abort);
         if (!ok) break;
         mbar_expect_tx(&bars->qd_full, 2 * kTileB);
@@ -177,7 +157,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idSS = idesc_bf16(128, 128, false, false);
+      const uint32_t idSS_last = idesc_bf16(128, (kc_last + 15) & ~15, false, false);
       const uint32_t idDQ = idesc_bf16(128, 128, false, true);
+      const int ks_last = (kc_last + 15) / 16;
       const uint32_t qb = smem_u32(sQ), ob = smem_u32(sO);
       int J = 0, it_local = 0, prev_c = -1, prev_it = -1;
       bool ok = true;
@@ -190,8 +172,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         tc_fence_after();
         const uint32_t kb = smem_u32(sK + b * kTileB);
         const uint32_t tdS = tmem + 128 + b * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        const int ks = cp == nch - 1 ? ks_last : 8;
+        for (int kk = 0; kk < ks; ++kk)
           mma_ts(tDQ, tdS + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
                  (cp > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty_k[b]);
@@ -207,10 +189,11 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, status, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kb = smem_u32(sK + st * kTileB);
+          const uint32_t idc = c == nch - 1 ? idSS_last : idSS;   // N = the chunk's keys
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tS, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idSS,
+            mma_ss(tS, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idc,
                    kk > 0 ? 1u : 0u);
           }
           if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, status, abort)) { ok = false; break; }
@@ -220,7 +203,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
             mma_ss(tmem + 128 + st * 128, desc_sw128(ob + off, 16, 1024),
-                   desc_sw128(vb + off, 16, 1024), idSS, kk > 0 ? 1u : 0u);
+                   desc_sw128(vb + off, 16, 1024), idc, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->empty_v[st]);
           mma_commit(&bars->s_full[st]);
@@ -237,15 +220,16 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const int r = wq * 32 + lane;
     const int cb = 64 * wg;                         // this group's key columns
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    float* stg = reinterpret_cast<float*>(sStage + (warp - 4) * kStageB);
     int J = 0, it_local = 0;
     bool ok = true;
     for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-      const QItem it = decode_qitem(P, n, item_off, col_off, col_rows);
+      const WorkItem it = decode_item(pv, P, h, n);
       const bool valid = r < it.count;
-      uint32_t i = 0;
       float l2 = 0.f, Di = 0.f;
+      uint32_t slot = 0xFFFFFFFFu;
       if (valid) {
-        i = __ldg(it.rows + r);
+        slot = __ldg(col_slot + it.first + r);
         l2 = __ldg(l2g + (size_t)n * kTile + r);
         Di = __ldg(dg + (size_t)n * kTile + r);
       }
@@ -254,7 +238,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, status, abort));
         if (!ok) break;
         tc_fence_after();
-        const int lim = P.L - c * kTile - cb;       // valid columns of this group
+        const int lim = (c == nch - 1 ? kc_last : kTile) - cb;   // valid columns of this group
+        if (lim <= 0) {
+          // no key of this chunk in the group's columns: the dQ MMA reads none of them
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(&bars->s_free); mbar_arrive(&bars->ds_full[b]); }
+          continue;
+        }
         const bool full = lim >= 64;
         uint32_t xr[64];
         tmem_ld32(tS + lane_off + cb, xr);
@@ -277,9 +267,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float d0 = __uint_as_float(xr[hh * 32 + e]) * (__uint_as_float(dp[e]) - Di);
+            // columns past the chunk's keys: dP is not written there, dS = 0
+            const bool on0 = full || hh * 32 + e < lim, on1 = full || hh * 32 + e + 1 < lim;
+            const float d0 =
+                on0 ? __uint_as_float(xr[hh * 32 + e]) * (__uint_as_float(dp[e]) - Di) : 0.f;
             const float d1 =
-                __uint_as_float(xr[hh * 32 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di);
+                on1 ? __uint_as_float(xr[hh * 32 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di)
+                    : 0.f;
             pk[e >> 1] = pack_bf16x2(d0, d1);
           }
           // dS into the group's columns [cb + 16 hh, +16): dP columns already read
@@ -294,21 +288,28 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, status, abort));
       if (!ok) break;
       tc_fence_after();
-      size_t slot = 0;
-      if (valid)
-        slot = pair_slot(row_off, sel + ((size_t)h * P.s + i) * P.Wb, P.Wb, (int)i, it.j);
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {               // this group's 64 dQ columns
         uint32_t xr[32];
         tmem_ld32(tDQ + lane_off + cb + cc * 32, xr);
         tmem_ld_wait();
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(part_dq + slot * kD + cb + cc * 32);
+        // row `lane` into the staging tile, 16-byte granules XOR-swizzled by row
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            dst[e / 4] = make_float4(__uint_as_float(xr[e]), __uint_as_float(xr[e + 1]),
-                                     __uint_as_float(xr[e + 2]), __uint_as_float(xr[e + 3]));
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<float4*>(stg + lane * 32 + ((g ^ (lane & 7)) << 2)) =
+              make_float4(__uint_as_float(xr[4 * g]), __uint_as_float(xr[4 * g + 1]),
+                          __uint_as_float(xr[4 * g + 2]), __uint_as_float(xr[4 * g + 3]));
+        __syncwarp();
+        // eight lanes per row: four whole 128-byte lines per store instruction
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), g = lane & 7;
+          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 32 + ((g ^ (rr & 7)) << 2));
+          const uint32_t sl = __shfl_sync(0xffffffffu, slot, rr);
+          if (sl != 0xFFFFFFFFu)
+            *reinterpret_cast<float4*>(part_dq + (size_t)sl * kD + cb + cc * 32 + g * 4) = v;
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
@@ -608,7 +609,7 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
-      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, sel, pv, ib.dg,
+      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, pv, ib.dg,
                                                         ib.l2g, sl2, part_dq, status);
     }
     {

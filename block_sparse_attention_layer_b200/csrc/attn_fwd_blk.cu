@@ -11,18 +11,27 @@
 // kernel then combines the partials of each query with log-sum-exp weights
 // into O, its fp32 copy and LSE.
 //
-// Persistent kernel, one head per launch: CTA b takes items b, b + G, ...
-// (all items of a layer cost the same, so a static round-robin balances).
-// Roles (256 threads):
-//   warp 0      TMA producer of the block's K / V chunks (2-stage rings);
-//   warp 1      TMEM owner (512 columns) and single-thread MMA issuer:
-//               S = Q K^T into two S buffers; O += P V with P read from TMEM;
-//   (warps 2-3 idle: the softmax warpgroup must start at a multiple of 4)
-// Query tiles come by TMA from the item-ordered copy of Q (gather.cu) into
-// two Q buffers, loaded by the producer ahead of the item.
-//   warps 4-7   softmax: one query row per thread, lazy 2^8 rescale of O,
-//               then the item's epilogue (partials out).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384).
+// Persistent kernel, one head per launch.  A CTA takes PAIRS of work items
+// (two consecutive 128-query tiles A, B of one block's list) so that every
+// K / V chunk it loads serves 256 queries; CTA b takes pairs b, b + G, ...
+// (static round-robin: all pairs of a layer cost about the same).
+// Roles (384 threads):
+//   warp 0      TMA producer: the pair's two query tiles (item-ordered copy
+//               of Q, gather.cu) and the block's K / V chunks (2-stage rings);
+//   warp 1      TMEM owner (512 columns) and single-thread MMA issuer;
+//   (warps 2-3 idle: a softmax warpgroup must start at a multiple of 4)
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query
+//               row per thread, lazy 2^8 rescale of O, then the tile's
+//               epilogue (partials out through a per-warp staging buffer so
+//               that the global stores are whole 128-byte lines).
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// The MMA issue order per chunk c is PV_A(c), S_A(c+1), PV_B(c), S_B(c+1):
+// while one warpgroup computes exponentials the tensor core serves the other.
+// P is written as bf16 pairs over the first half of its own S columns; the
+// next S of the same tile is issued after the PV that reads P, and MMAs of
+// one CTA execute in issue order.
+// The last chunk of a block whose size is not a multiple of 128 runs with
+// N = its key count rounded up to 16 (S) and that many 16-key steps (PV).
 #include "tc_prims.cuh"
 #include "pairs.cuh"
 
@@ -34,66 +43,97 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr uint32_t kHalf = 128 * 64 * 2;
 constexpr uint32_t kTileB = 2 * kHalf;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kStageB = 32 * 32 * 4;     // per softmax warp: 32 rows x 32 fp32
 
 struct Bars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
-  uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t o_final, o_free;
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], p_full[2], o_final[2], o_free[2];   // per tile of the pair
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + 2 * kTileB /*Q x2*/ + 2 * kTileB /*K*/ + 2 * kTileB /*V*/ +
-                              sizeof(Bars) + 64;
+constexpr size_t kSmemBytes = 1024 + 2 * kTileB /*Q pair*/ + 2 * kTileB /*K*/ + 2 * kTileB /*V*/ +
+                              8 * kStageB + sizeof(Bars) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-struct Item {
-  int j, count;           // block, queries in this tile (1..128)
-  const uint32_t* rows;   // the tile's query indices
-};
-
-__device__ __forceinline__ Item decode_item(const Prob& P, int n, const uint32_t* item_off,
-                                            const uint32_t* col_off, const uint32_t* col_rows) {
-  // largest j with item_off[j] <= n (item_off is non-decreasing, item_off[0] = 0)
-  int lo = 0, hi = P.Nb;   // invariant: item_off[lo] <= n < item_off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
+// One chunk of softmax for one row: P = 2^(S sl2 - m) over the chunk's kc
+// valid keys (NC columns loaded), written as bf16 pairs over S's first NC/2
+// columns; running max / sum updated, O rescaled when the max grew by more
+// than 2^8.
+template <int NC>
+__device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, float sl2,
+                                              float& m_run, float& l_run) {
+  uint32_t xr[NC];
+#pragma unroll
+  for (int g = 0; g < NC / 32; ++g) tmem_ld32(tS + g * 32, xr + g * 32);
+  tmem_ld_wait();
+  const bool full = kc >= NC;
+  float mt = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < NC; ++e)
+    mt = fmaxf(mt, (full || e < kc) ? __uint_as_float(xr[e]) : -INFINITY);
+  const float mt2 = mt * sl2;
+  const bool grows = m_run == -INFINITY || mt2 > m_run + kRescaleLog2;
+  const bool rescale = grows && m_run > -INFINITY;
+  const float m_new = grows ? fmaxf(mt2, m_run) : m_run;
+  float lsum = 0.f;
+#pragma unroll
+  for (int c4 = 0; c4 < NC / 32; ++c4) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int col = c4 * 32 + e;
+      const float a = (full || col < kc) ? fast_exp2(fmaf(__uint_as_float(xr[col]), sl2, -m_new))
+                                         : 0.f;
+      const float b = (full || col + 1 < kc)
+                          ? fast_exp2(fmaf(__uint_as_float(xr[col + 1]), sl2, -m_new)) : 0.f;
+      lsum += a + b;
+      pk[e >> 1] = pack_bf16x2(a, b);
+    }
+    tmem_st16(tS + c4 * 16, pk);
   }
-  Item it;
-  it.j = lo;
-  const int g = n - (int)__ldg(item_off + lo);
-  const int c0 = (int)__ldg(col_off + lo), c1 = (int)__ldg(col_off + lo + 1);
-  it.count = min(kTile, c1 - c0 - g * kTile);
-  it.rows = col_rows + c0 + g * kTile;
-  return it;
+  // O rescale after the S row is consumed (fewer live registers); O holds
+  // the previous chunks' PV, complete since this S was issued after it
+  float f = 1.0f;
+  if (__any_sync(0xffffffffu, rescale)) {
+    f = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t ob[32];
+      tmem_ld32(tO + cc * 32, ob);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * f);
+      tmem_st32(tO + cc * 32, ob);
+    }
+  }
+  m_run = m_new;
+  l_run = fmaf(l_run, f, lsum);
+  tmem_st_wait();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-          const __grid_constant__ CUtensorMap tm_q, Prob P, int h,
-          const uint32_t* __restrict__ sel,
-          PairsView pv, float sl2, float* __restrict__ part_o, float2* __restrict__ part_ml,
-          int* __restrict__ status) {
+          const __grid_constant__ CUtensorMap tm_q, Prob P, int h, PairsView pv, float sl2,
+          float* __restrict__ part_o, float2* __restrict__ part_ml, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                       // 2 buffers
-  uint8_t* sK = sQ + 2 * kTileB;
-  uint8_t* sV = sK + 2 * kTileB;
-  Bars* bars = reinterpret_cast<Bars*>(sV + 2 * kTileB);
+  uint8_t* sQ = smem;                       // tiles A, B
+  uint8_t* sK = sQ + 2 * kTileB;            // 2 stages
+  uint8_t* sV = sK + 2 * kTileB;            // 2 stages
+  uint8_t* sStage = sV + 2 * kTileB;        // 8 x kStageB
+  Bars* bars = reinterpret_cast<Bars*>(sStage + 8 * kStageB);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
-  const uint32_t* row_off = pv.row_off + (size_t)h * (P.s + 1);
-  const int n_items = (int)__ldg(pv.head_totals + 2 * h + 1);
+  const int n_pairs = (int)__ldg(pv.head_totals + 4 * h + 2);
   const int nch = (P.L + kTile - 1) / kTile;          // key chunks per block
+  const int kc_last = P.L - (nch - 1) * kTile;        // keys in the last chunk
   const int G = gridDim.x;
 
   if (threadIdx.x == 0) {
@@ -101,11 +141,10 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       mbar_init(&bars->full_k[i], 1); mbar_init(&bars->empty_k[i], 1);
       mbar_init(&bars->full_v[i], 1); mbar_init(&bars->empty_v[i], 1);
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 4);
-      mbar_init(&bars->o_done[i], 1);
-      mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 1);
+      mbar_init(&bars->o_final[i], 1); mbar_init(&bars->o_free[i], 4);
     }
-    mbar_init(&bars->o_final, 1);
-    mbar_init(&bars->o_free, 4);
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -117,7 +156,6 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tO = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -127,17 +165,21 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       tma_prefetch_desc(&tm_q);
       int J = 0, it_local = 0;
       bool ok = true;
-      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-        const Item it = decode_item(P, n, item_off, col_off, col_rows);
-        const int qb = it_local & 1;
-        if (it_local >= 2)
-          ok = mbar_wait(&bars->q_empty[qb], ((it_local >> 1) - 1) & 1, status, abort);
+      for (int p = blockIdx.x; p < n_pairs && ok; p += G, ++it_local) {
+        WorkItem b;
+        int n0;
+        const WorkItem a = decode_item_pair(pv, P, h, p, &b, &n0);
+        if (it_local >= 1) ok = mbar_wait(&bars->q_empty, (it_local - 1) & 1, status, abort);
         if (!ok) break;
-        mbar_expect_tx(&bars->q_full[qb], kTileB);
-        tma_load_2d(sQ + qb * kTileB, &tm_q, &bars->q_full[qb], 0, n * kTile);
-        tma_load_2d(sQ + qb * kTileB + kHalf, &tm_q, &bars->q_full[qb], 64, n * kTile);
+        mbar_expect_tx(&bars->q_full, b.count > 0 ? 2 * kTileB : kTileB);
+        tma_load_2d(sQ, &tm_q, &bars->q_full, 0, n0 * kTile);
+        tma_load_2d(sQ + kHalf, &tm_q, &bars->q_full, 64, n0 * kTile);
+        if (b.count > 0) {
+          tma_load_2d(sQ + kTileB, &tm_q, &bars->q_full, 0, (n0 + 1) * kTile);
+          tma_load_2d(sQ + kTileB + kHalf, &tm_q, &bars->q_full, 64, (n0 + 1) * kTile);
+        }
         for (int c = 0; c < nch && ok; ++c, ++J) {
-          const int row = h * P.s + it.j * P.L + c * kTile;
+          const int row = h * P.s + a.j * P.L + c * kTile;
           const int st = J & 1;
           if (J >= 2) ok = mbar_wait(&bars->empty_k[st], ((J >> 1) - 1) & 1, status, abort);
           if (!ok) break;
@@ -156,154 +198,143 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
+      const uint32_t idS_last = idesc_bf16(128, (kc_last + 15) & ~15, false, false);
       const uint32_t idPV = idesc_bf16(128, 128, false, true);
-      int J = 0, it_local = 0;
-      int prev_c = -1, prev_it = -1;   // chunk / item of the chunk whose PV is pending
+      const int ks_last = (kc_last + 15) / 16;
+      int Jk = 0;                 // chunks through the K / V rings
+      int Js[2] = {0, 0};         // S / P rounds per tile
+      int It[2] = {0, 0};         // items per tile
       bool ok = true;
-      auto issue_pv = [&](int Jp, int cp, int itp) -> bool {
-        const int sb = Jp & 1;
-        if (!mbar_wait(&bars->p_full[sb], (Jp >> 1) & 1, status, abort)) return false;
-        if (!mbar_wait(&bars->full_v[sb], (Jp >> 1) & 1, status, abort)) return false;
-        if (cp == 0 && itp > 0 && !mbar_wait(&bars->o_free, (itp - 1) & 1, status, abort))
-          return false;
-        tc_fence_after();
-        const uint32_t vb = smem_u32(sV + sb * kTileB);
-        const uint32_t tP = tmem + sb * 128;
+      auto issue_s = [&](int t, uint32_t kb, bool last) {
+        const uint32_t qbase = smem_u32(sQ + t * kTileB);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tO, tP + kk * 8, desc_sw128(vb + kk * 2048, kHalf, 1024), idPV,
-                 (cp > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->empty_v[sb]);
-        mma_commit(&bars->o_done[sb]);
-        if (cp == nch - 1) mma_commit(&bars->o_final);
-        return true;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, desc_sw128(qbase + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
+                 last ? idS_last : idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[t]);
       };
-      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-        const int qb = it_local & 1;
-        if (!mbar_wait(&bars->q_full[qb], (it_local >> 1) & 1, status, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qbase = smem_u32(sQ + qb * kTileB);
-        for (int c = 0; c < nch && ok; ++c, ++J) {
-          const int st = J & 1;
-          if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, status, abort)) { ok = false; break; }
+      auto issue_pv = [&](int t, uint32_t vb, int c) {
+        const int ks = c == nch - 1 ? ks_last : 8;
+        for (int kk = 0; kk < ks; ++kk)
+          mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                 desc_sw128(vb + kk * 2048, kHalf, 1024), idPV, (c > 0 || kk > 0) ? 1u : 0u);
+        if (c == nch - 1) mma_commit(&bars->o_final[t]);
+      };
+      for (int p = blockIdx.x, it_local = 0; p < n_pairs && ok; p += G, ++it_local) {
+        WorkItem b;
+        int n0;
+        decode_item_pair(pv, P, h, p, &b, &n0);
+        const int nt = b.count > 0 ? 2 : 1;
+        if (!mbar_wait(&bars->q_full, it_local & 1, status, abort)) { ok = false; break; }
+        {
+          const int st = Jk & 1;
+          if (!mbar_wait(&bars->full_k[st], (Jk >> 1) & 1, status, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kb = smem_u32(sK + st * kTileB);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tmem + st * 128, desc_sw128(qbase + off, 16, 1024),
-                   desc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-          }
+          for (int t = 0; t < nt; ++t) issue_s(t, kb, nch == 1);
           mma_commit(&bars->empty_k[st]);
-          mma_commit(&bars->s_full[st]);
-          if (c == nch - 1) mma_commit(&bars->q_empty[qb]);
-          if (J > 0) ok = issue_pv(J - 1, prev_c, prev_it);
-          prev_c = c;
-          prev_it = it_local;
+          if (nch == 1) mma_commit(&bars->q_empty);
         }
+        for (int c = 0; c < nch && ok; ++c) {
+          const int Jc = Jk + c, stc = Jc & 1, st1 = (Jc + 1) & 1;
+          const bool more = c + 1 < nch;
+          if (!mbar_wait(&bars->full_v[stc], (Jc >> 1) & 1, status, abort)) { ok = false; break; }
+          uint32_t kb1 = 0;
+          for (int t = 0; t < nt && ok; ++t) {
+            if (c == 0 && It[t] > 0 &&
+                !mbar_wait(&bars->o_free[t], (It[t] - 1) & 1, status, abort)) { ok = false; break; }
+            if (!mbar_wait(&bars->p_full[t], Js[t] & 1, status, abort)) { ok = false; break; }
+            ++Js[t];
+            tc_fence_after();
+            issue_pv(t, smem_u32(sV + stc * kTileB), c);
+            if (more) {
+              if (t == 0) {
+                if (!mbar_wait(&bars->full_k[st1], ((Jc + 1) >> 1) & 1, status, abort)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                kb1 = smem_u32(sK + st1 * kTileB);
+              }
+              issue_s(t, kb1, c + 1 == nch - 1);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars->empty_v[stc]);
+          if (more) {
+            mma_commit(&bars->empty_k[st1]);
+            if (c + 1 == nch - 1) mma_commit(&bars->q_empty);
+          }
+        }
+        Jk += nch;
+        for (int t = 0; t < nt; ++t) ++It[t];
       }
-      if (ok && J > 0) issue_pv(J - 1, prev_c, prev_it);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
-    const int wq = warp - 4;
+    const int t = (warp - 4) >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    int J = 0, it_local = 0;
+    const uint32_t tS = tmem + t * 128 + lane_off, tO = tmem + 256 + t * 128 + lane_off;
+    float* stg = reinterpret_cast<float*>(sStage + (warp - 4) * kStageB);
+    const uint32_t* col_slot = pv.col_slot + (size_t)h * P.s * P.Nb;
+    int Js = 0, It = 0;
     bool ok = true;
-    for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-      const Item it = decode_item(P, n, item_off, col_off, col_rows);
+    for (int p = blockIdx.x; p < n_pairs && ok; p += G) {
+      WorkItem b;
+      int n0;
+      const WorkItem a = decode_item_pair(pv, P, h, p, &b, &n0);
+      const WorkItem me = t == 0 ? a : b;
+      if (me.count == 0) continue;                 // no tile B in this pair
+      const bool valid = r < me.count;
+      const uint32_t slot = valid ? __ldg(col_slot + me.first + r) : 0xFFFFFFFFu;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int c = 0; c < nch; ++c, ++J) {
-        const int sb = J & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (J >> 1) & 1, status, abort));
+      for (int c = 0; c < nch; ++c, ++Js) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], Js & 1, status, abort));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = tmem + sb * 128 + lane_off;
-        const int lim = P.L - c * kTile;        // keys of this chunk inside block j
-        const bool full = lim >= kTile;         // uniform over the CTA
-        // the whole S row in registers: four loads, one wait
-        uint32_t xr[128];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, xr + c4 * 32);
-        tmem_ld_wait();
-        float mt = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          mt = fmaxf(mt, (full || e < lim) ? __uint_as_float(xr[e]) : -INFINITY);
-        const float mt2 = mt * sl2;
-        const bool grows = m_run == -INFINITY || mt2 > m_run + kRescaleLog2;
-        const bool rescale = grows && m_run > -INFINITY;
-        const float m_new = grows ? fmaxf(mt2, m_run) : m_run;
-        if (__any_sync(0xffffffffu, rescale)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[(J - 1) & 1], ((J - 1) >> 1) & 1,
-                                                 status, abort));
-          if (!ok) break;
-          tc_fence_after();
-          const float f = rescale ? exp2f(m_run - m_new) : 1.0f;
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t ob[32];
-            tmem_ld32(tO + cc * 32 + lane_off, ob);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * f);
-            tmem_st32(tO + cc * 32 + lane_off, ob);
-          }
-          tmem_st_wait();
-          l_run *= f;
-        }
-        m_run = m_new;
-        float lsum = 0.f;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int col = c4 * 32 + e;
-            const float a = (full || col < lim)
-                                ? exp2f(fmaf(__uint_as_float(xr[col]), sl2, -m_run)) : 0.f;
-            const float b = (full || col + 1 < lim)
-                                ? exp2f(fmaf(__uint_as_float(xr[col + 1]), sl2, -m_run)) : 0.f;
-            lsum += a + b;
-            pk[e >> 1] = pack_bf16x2(a, b);
-          }
-          tmem_st16(tS + c4 * 16, pk);
-        }
-        l_run += lsum;
-        tmem_st_wait();
+        const int kc = c == nch - 1 ? kc_last : kTile;
+        if (kc > 64) softmax_chunk<128>(tS, tO, kc, sl2, m_run, l_run);
+        else softmax_chunk<64>(tS, tO, kc, sl2, m_run, l_run);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
+        if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
       if (!ok) break;
       // epilogue: partial state of (query, block j) into the pair's slot
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, it_local & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[t], It & 1, status, abort));
+      ++It;
       if (!ok) break;
       tc_fence_after();
-      const bool valid = r < it.count;
-      size_t slot = 0;
-      if (valid) {
-        const uint32_t i = __ldg(it.rows + r);
-        slot = pair_slot(row_off, sel + ((size_t)h * P.s + i) * P.Wb, P.Wb, (int)i, it.j);
-        part_ml[slot] = make_float2(m_run, l_run);
-      }
-#pragma unroll
+      if (valid) part_ml[slot] = make_float2(m_run, l_run);
+#pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t ob[32];
-        tmem_ld32(tO + cc * 32 + lane_off, ob);
+        tmem_ld32(tO + cc * 32, ob);
         tmem_ld_wait();
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(part_o + slot * kD + cc * 32);
+        // row `lane` into the staging tile, 16-byte granules XOR-swizzled by row
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            dst[e / 4] = make_float4(__uint_as_float(ob[e]), __uint_as_float(ob[e + 1]),
-                                     __uint_as_float(ob[e + 2]), __uint_as_float(ob[e + 3]));
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<float4*>(stg + lane * 32 + ((g ^ (lane & 7)) << 2)) =
+              make_float4(__uint_as_float(ob[4 * g]), __uint_as_float(ob[4 * g + 1]),
+                          __uint_as_float(ob[4 * g + 2]), __uint_as_float(ob[4 * g + 3]));
+        __syncwarp();
+        // eight lanes per row: four whole 128-byte lines per store instruction
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), g = lane & 7;
+          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 32 + ((g ^ (rr & 7)) << 2));
+          const uint32_t sl = __shfl_sync(0xffffffffu, slot, rr);
+          if (sl != 0xFFFFFFFFu)
+            *reinterpret_cast<float4*>(part_o + (size_t)sl * kD + cc * 32 + g * 4) = v;
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->o_free);
+      if (lane == 0) mbar_arrive(&bars->o_free[t]);
     }
   }
   tc_fence_before();
@@ -379,8 +410,8 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_fwd_blk", st);
-      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, sel, pv, sl2, part_o,
-                                                        part_ml, status);
+      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, pv, sl2, part_o, part_ml,
+                                                        status);
     }
     {
       VMOBA_TRACE("k_fwd_merge", st);

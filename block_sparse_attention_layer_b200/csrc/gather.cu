@@ -19,22 +19,14 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
                __nv_bfloat16* __restrict__ bg, const float* __restrict__ fa,
                const float* __restrict__ fb, float* __restrict__ fag, float* __restrict__ fbg,
                float fa_pad) {
-  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
-  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
   const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
-  const int n_items = (int)__ldg(pv.head_totals + 2 * h + 1);
+  const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < n_items; n += warps) {
-    int lo = 0, hi = P.Nb;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
-    }
-    const int g = n - (int)__ldg(item_off + lo);
-    const int c0 = (int)__ldg(col_off + lo), c1 = (int)__ldg(col_off + lo + 1);
-    const int count = min(kTile, c1 - c0 - g * kTile);
-    const uint32_t* rows = col_rows + c0 + g * kTile;
+    const WorkItem it = decode_item(pv, P, h, n);
+    const int count = it.count;
+    const uint32_t* rows = col_rows + it.first;
     const size_t base = (size_t)n * kTile;
     for (int r0 = 0; r0 < kTile; r0 += kRowsInFlight) {
       uint2 va[kRowsInFlight], vb[kRowsInFlight];

@@ -8,8 +8,12 @@
 //                ("CSR"); partial results of the attention kernels live there;
 //   col_off[j]   start of block j's query list in col_rows ("CSC"), queries
 //                in ascending order (deterministic);
+//   col_slot     beside every col_rows entry, the pair slot of that
+//                (query, block) pair, so the attention kernels index the
+//                CSR partials directly;
 //   item_off[j]  first work item of block j: its query list cut into tiles of
-//                128 queries; item_off[N_b] = number of work items.
+//                128 queries; item_off[N_b] = number of work items;
+//   pitem_off[j] the same for pairs of consecutive tiles (256 queries).
 // Rows are processed in chunks of 256 (8 warps x 32 rows); per-chunk column
 // counts give each chunk's base inside every block list, and warp ballots
 // give each row's rank inside the chunk.
@@ -80,7 +84,8 @@ __device__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh, uint32_t* total) {
 __global__ void __launch_bounds__(1024)
 k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict__ chunk_cnt,
              int n_chunks, uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_off,
-             uint32_t* __restrict__ item_off, uint32_t* __restrict__ head_totals) {
+             uint32_t* __restrict__ item_off, uint32_t* __restrict__ pitem_off,
+             uint32_t* __restrict__ head_totals) {
   __shared__ uint32_t sh[32];
   const int h = blockIdx.x, t = threadIdx.x;
   uint32_t* cc = chunk_cnt + (size_t)h * n_chunks * P.Nb;
@@ -91,11 +96,13 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
   uint32_t all;
   const uint32_t off = block_excl_scan(t < P.Nb ? tot : 0u, sh, &all);
   const uint32_t tiles = t < P.Nb ? (tot + kTile - 1) / kTile : 0u;
-  uint32_t n_items;
+  uint32_t n_items, n_pitems;
   const uint32_t ioff = block_excl_scan(tiles, sh, &n_items);
+  const uint32_t poff = block_excl_scan((tiles + 1) / 2, sh, &n_pitems);
   if (t < P.Nb) {
     col_off[(size_t)h * (P.Nb + 1) + t] = off;
     item_off[(size_t)h * (P.Nb + 1) + t] = ioff;
+    pitem_off[(size_t)h * (P.Nb + 1) + t] = poff;
     // chunk bases in place: base of chunk c in block t's list
     uint32_t run = off;
     for (int c = 0; c < n_chunks; ++c) {
@@ -107,8 +114,11 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
   if (t == 0) {
     col_off[(size_t)h * (P.Nb + 1) + P.Nb] = all;
     item_off[(size_t)h * (P.Nb + 1) + P.Nb] = n_items;
-    head_totals[2 * h] = all;
-    head_totals[2 * h + 1] = n_items;
+    pitem_off[(size_t)h * (P.Nb + 1) + P.Nb] = n_pitems;
+    head_totals[4 * h] = all;
+    head_totals[4 * h + 1] = n_items;
+    head_totals[4 * h + 2] = n_pitems;
+    head_totals[4 * h + 3] = 0u;
   }
   // row offsets: exclusive scan of row_cnt over s rows, 1024 at a time
   uint32_t carry = 0;
@@ -124,16 +134,20 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
 }
 
 // Per (chunk, head): write every row of the chunk into the lists of the
-// blocks it selected, at chunk base + rank among the chunk's rows.
+// blocks it selected, at chunk base + rank among the chunk's rows, with the
+// row's pair slot (its CSR offset plus the blocks below j it selected).
 __global__ void __launch_bounds__(kChunkRows)
 k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restrict__ chunk_base,
-             int n_chunks, uint32_t* __restrict__ col_rows) {
+             int n_chunks, const uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_rows,
+             uint32_t* __restrict__ col_slot) {
   __shared__ uint32_t wcnt[kChunkRows / 32][32];
   const int c = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = c * kChunkRows + threadIdx.x;
   const uint32_t* cb = chunk_base + ((size_t)h * n_chunks + c) * P.Nb;
   uint32_t* rows = col_rows + (size_t)h * P.s * P.Nb;
+  uint32_t* slots = col_slot + (size_t)h * P.s * P.Nb;
+  uint32_t slot = (i < P.s) ? __ldg(row_off + (size_t)h * (P.s + 1) + i) : 0u;
   for (int w = 0; w < P.Wb; ++w) {
     const uint32_t bits = (i < P.s) ? __ldg(sel + ((size_t)h * P.s + i) * P.Wb + w) : 0u;
     const int jmax = min(32, P.Nb - w * 32);
@@ -158,6 +172,7 @@ k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restric
       if ((bits >> b) & 1u) {
         const uint32_t rank = __popc(m & ((1u << lane) - 1u));
         rows[wcnt[warp][b] + rank] = (uint32_t)i;
+        slots[wcnt[warp][b] + rank] = slot++;
       }
     }
     __syncthreads();
@@ -174,9 +189,11 @@ size_t pairs_ws_bytes(const Prob& P) {
   take(sizeof(uint32_t) * (size_t)P.n_h * (P.s + 1));           // row_off
   take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // col_off
   take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // item_off
-  take(sizeof(uint32_t) * 2 * P.n_h);                           // head totals
+  take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // pitem_off
+  take(sizeof(uint32_t) * 4 * P.n_h);                           // head totals
   take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);     // chunk counts / bases
   take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_rows (worst case)
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_slot (worst case)
   return b;
 }
 
@@ -189,9 +206,11 @@ PairsView pairs_view(const Prob& P, void* base) {
   v.row_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.s + 1));
   v.col_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
   v.item_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
-  v.head_totals = take(sizeof(uint32_t) * 2 * P.n_h);
+  v.pitem_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
+  v.head_totals = take(sizeof(uint32_t) * 4 * P.n_h);
   v.chunk = take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);
   v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
+  v.col_slot = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
   v.n_chunks = n_chunks;
   return v;
 }
@@ -205,11 +224,12 @@ cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v,
   {
     VMOBA_TRACE("k_pairs_scan", st);
     k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
-                                         v.item_off, v.head_totals);
+                                         v.item_off, v.pitem_off, v.head_totals);
   }
   {
     VMOBA_TRACE("k_pairs_fill", st);
-    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.col_rows);
+    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.row_off, v.col_rows,
+                                           v.col_slot);
   }
   count_launches(3);
   return cudaGetLastError();

@@ -10,11 +10,64 @@ struct PairsView {
   uint32_t* row_off;      // [n_h][s+1]   CSR offsets (pair slots of each query)
   uint32_t* col_off;      // [n_h][N_b+1] start of each block's query list
   uint32_t* item_off;     // [n_h][N_b+1] first 128-query work item of each block
-  uint32_t* head_totals;  // [n_h][2]     pairs, work items
+  uint32_t* pitem_off;    // [n_h][N_b+1] first pair of work items (256 queries) of each block
+  uint32_t* head_totals;  // [n_h][4]     pairs, work items, item pairs, 0
   uint32_t* chunk;        // [n_h][chunks][N_b] scratch (chunk bases)
   uint32_t* col_rows;     // [n_h][s*N_b] query lists, block by block
+  uint32_t* col_slot;     // [n_h][s*N_b] pair slot of each list entry
   int n_chunks;
 };
+
+// A work item: block j and one tile of up to 128 queries of its list.
+struct WorkItem {
+  int j;                  // block
+  int count;              // queries in the tile (0 when the tile does not exist)
+  uint32_t first;         // index of the tile's first entry in col_rows / col_slot
+};
+
+// Work item n of head h (n < head_totals[4h+1]).
+__device__ __forceinline__ WorkItem decode_item(const PairsView& pv, const Prob& P, int h, int n) {
+  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
+  int lo = 0, hi = P.Nb;   // invariant: item_off[lo] <= n < item_off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
+  }
+  WorkItem it;
+  it.j = lo;
+  const int g = n - (int)__ldg(item_off + lo);
+  const uint32_t c0 = __ldg(col_off + lo), c1 = __ldg(col_off + lo + 1);
+  it.first = c0 + (uint32_t)g * kTile;
+  it.count = min(kTile, (int)(c1 - it.first));
+  return it;
+}
+
+// Item pair p of head h: tiles 2q and 2q+1 of one block's list (the second
+// may be absent).  Returns the first tile; *second gets the other (count 0
+// when absent) and *n0 the first tile's work-item index.
+__device__ __forceinline__ WorkItem decode_item_pair(const PairsView& pv, const Prob& P, int h,
+                                                     int p, WorkItem* second, int* n0) {
+  const uint32_t* pitem_off = pv.pitem_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
+  int lo = 0, hi = P.Nb;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(pitem_off + mid) <= (uint32_t)p) lo = mid; else hi = mid;
+  }
+  const int q = p - (int)__ldg(pitem_off + lo);
+  const uint32_t c0 = __ldg(col_off + lo), c1 = __ldg(col_off + lo + 1);
+  WorkItem a, b;
+  a.j = b.j = lo;
+  a.first = c0 + (uint32_t)q * 2 * kTile;
+  b.first = a.first + kTile;
+  a.count = min(kTile, (int)(c1 - a.first));
+  b.count = c1 > b.first ? min(kTile, (int)(c1 - b.first)) : 0;
+  *n0 = (int)__ldg(item_off + lo) + 2 * q;
+  *second = b;
+  return a;
+}
 
 // Item-ordered copies (gather.cu): bf16 rows of Q and dO, fp32 LSE*log2e and D.
 struct ItemBufs {
@@ -47,18 +100,5 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
                                 const ItemBufs& ib, const float* o32, const float* lse,
                                 const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
                                 float scale, int* status, int num_sms, cudaStream_t st);
-
-// Pair slot of (query i, block j) for a selected pair: CSR offset of the row
-// plus the number of blocks below j the row selected.
-__device__ __forceinline__ uint32_t pair_slot(const uint32_t* __restrict__ row_off_h,
-                                              const uint32_t* __restrict__ sel_row, int Wb,
-                                              int i, int j) {
-  uint32_t r = 0;
-  const int wj = j >> 5;
-  for (int w = 0; w < wj; ++w) r += __popc(__ldg(sel_row + w));
-  r += __popc(__ldg(sel_row + wj) & ((1u << (j & 31)) - 1u));
-  (void)Wb;
-  return __ldg(row_off_h + i) + r;
-}
 
 }  // namespace vmoba
