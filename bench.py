@@ -192,8 +192,10 @@ def run_ours(args, rank, world, local):
     layers = [VMoBALayer(sh) for sh in shapes]
     stream = torch.cuda.current_stream()
 
-    def one_step(events=None):
+    def one_step(events=None, only=None):
         for li, L in enumerate(layers):
+            if only is not None and li != only:
+                continue
             ev = events[li] if events is not None else None
             if ev: ev[0].record(stream)
             V.partition(L.shape, k, v, L.k_perm, L.v_perm, L.blocks)
@@ -244,6 +246,16 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     elapsed_ms = start.elapsed_time(end)
+
+    # per-layer kernel times: one more (untimed) pass, layer by layer
+    kern_layer = {}
+    for li in range(len(layers)):
+        V.trace_enable(True)
+        one_step(only=li)
+        torch.cuda.synchronize()
+        V.trace_enable(False)
+        tr = V.trace_read()
+        kern_layer[f"l{li}"] = {n: round(ms, 4) for n, (_, ms) in tr.items() if ms >= 0.05}
 
     # per-call device times (ms, summed over layers, averaged over steps)
     call_ms = {c: 0.0 for c in CALLS}
@@ -319,6 +331,7 @@ def run_ours(args, rank, world, local):
             "clocks": clk.summary(),
             "detail": {
                 "call_ms_per_step": {c: round(call_ms[c], 4) for c in CALLS},
+                "kernel_ms_per_layer": kern_layer,
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
                                   for i, l in enumerate(LAYERS)},
                 "achieved": {c: [round(x[0], 3), x[1]] for c, x in achieved.items()},

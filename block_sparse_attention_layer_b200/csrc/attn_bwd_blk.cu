@@ -37,7 +37,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------- D_i, lse2
-// rowD[h][i] = dO_i . O_i (fp32 output copy); lse2[h][i] = LSE_i * log2(e).
+// rowD[h][i] = dO_i . O_i (fp32 output copy); nlse2[h][i] = -LSE_i * log2(e),
+// so that P = 2^(S scale log2(e) + nlse2) is one fused multiply-add and ex2.
 __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
                            const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                            float* __restrict__ rowD, float* __restrict__ lse2) {
@@ -52,7 +53,7 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   if (lane == 0) {
     rowD[(size_t)h * P.s + i] = acc;
-    lse2[(size_t)h * P.s + i] = lse[(size_t)h * P.s + i] * kLog2e;
+    lse2[(size_t)h * P.s + i] = -lse[(size_t)h * P.s + i] * kLog2e;
   }
 }
 
@@ -253,7 +254,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const bool on = valid && (full || e < lim);
-          xr[e] = __float_as_uint(on ? fast_exp2(fmaf(__uint_as_float(xr[e]), sl2, -l2)) : 0.f);
+          xr[e] = __float_as_uint(on ? fast_exp2(fmaf(__uint_as_float(xr[e]), sl2, l2)) : 0.f);
         }
         tc_fence_before();
         __syncwarp();
@@ -345,21 +346,27 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
 
 // =====================================================================
 // dK/dV pass.  Item = (key tile kt of block j, head h), one CTA each.
-// TMEM: S^T [0,128) (then P^T), dP^T [128,256) (then dS^T), dV [256,384),
-// dK [384,512).  Roles: warp 0 loads the K/V tile once, then each query
-// tile's Q and dO (TMA, item-ordered copies) and LSE*log2e, D (bulk copies)
-// into two buffers; warp 1 MMA; warps 4-7 softmax rows (one key per thread)
-// + epilogue (warps 2-3 idle).
+// Each query tile is taken in two halves of 64 queries, half h by softmax
+// warpgroup h, so that one half's exponentials overlap the other half's
+// MMAs.  TMEM: S^T_h [128h, 128h+64) (then P^T_h), dP^T_h [128h+64,
+// 128h+128) (then dS^T_h), dV [256,384), dK [384,512).  MMA issue order:
+// S/dP_0(g), S/dP_1(g), dVdK_0(g), S/dP_0(g+1), dVdK_1(g), S/dP_1(g+1), ...
+// (each S/dP_h overwrites only columns whose dVdK_h was issued before it).
+// Roles: warp 0 loads the K/V tile once, then each query tile's Q and dO
+// (TMA, item-ordered copies) and -LSE log2(e), D (bulk copies) into two
+// buffers; warp 1 MMA; warps 4-7 / 8-11 softmax of query half 0 / 1 (one
+// key row per thread) and the epilogue (dV / dK).
 // =====================================================================
 struct KvBars {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t st_full, pd_full, acc_final;
+  uint64_t st_full[2], pd_full[2];
+  uint64_t acc_final;
   uint32_t tmem_base;
   int abort;
 };
 constexpr size_t kKvSmem = 1024 + 2 * kTileB /*K,V*/ + 4 * kTileB /*Q,dO x2*/ +
-                           2 * 2 * kTile * sizeof(float) /*lse2, D x2*/ + sizeof(KvBars) + 64;
+                           2 * 2 * kTile * sizeof(float) /*nlse2, D x2*/ + sizeof(KvBars) + 64;
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -375,7 +382,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   uint8_t* sV = sK + kTileB;
   uint8_t* sQ = sV + kTileB;           // 2 buffers
   uint8_t* sO = sQ + 2 * kTileB;       // 2 buffers
-  float* sL = reinterpret_cast<float*>(sO + 2 * kTileB);   // [2][128] lse2
+  float* sL = reinterpret_cast<float*>(sO + 2 * kTileB);   // [2][128] -lse2
   float* sD = sL + 2 * kTile;                              // [2][128] D
   KvBars* bars = reinterpret_cast<KvBars*>(sD + 2 * kTile);
   volatile int* abort = &bars->abort;
@@ -393,9 +400,10 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
-    mbar_init(&bars->st_full, 1);
-    mbar_init(&bars->pd_full, kSoftmaxWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1);
+      mbar_init(&bars->st_full[i], 1); mbar_init(&bars->pd_full[i], 4);
+    }
     mbar_init(&bars->acc_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -408,7 +416,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
+  const uint32_t tV = tmem + 256, tK = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0 && ng > 0) {
@@ -435,16 +443,14 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else if (warp == 1) {
     if (lane == 0 && ng > 0) {
-      const uint32_t idSS = idesc_bf16(128, 128, false, false);
+      const uint32_t idSS = idesc_bf16(128, 64, false, false);    // keys x 64 queries
       const uint32_t idAcc = idesc_bf16(128, 128, false, true);
       const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
-      bool ok = mbar_wait(&bars->kv_full, 0, status, abort);
-      for (int g = 0; g < ng && ok; ++g) {
-        const int b = g & 1;
-        if (!mbar_wait(&bars->qd_full[b], (g >> 1) & 1, status, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qb = smem_u32(sQ + b * kTileB), ob = smem_u32(sO + b * kTileB);
-        // S^T = K Q^T and dP^T = V dO^T (keys x queries), K-major both sides
+      // S^T_h = K Q_h^T, dP^T_h = V dO_h^T (K-major both sides; Q_h = rows 64h..)
+      auto issue_sdp = [&](int hf, int b) {
+        const uint32_t qb = smem_u32(sQ + b * kTileB) + hf * 8192;
+        const uint32_t ob = smem_u32(sO + b * kTileB) + hf * 8192;
+        const uint32_t tS = tmem + 128 * hf, tP = tS + 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
@@ -457,67 +463,101 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           mma_ss(tP, desc_sw128(vb + off, 16, 1024), desc_sw128(ob + off, 16, 1024), idSS,
                  kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->st_full);
-        if (!mbar_wait(&bars->pd_full, g & 1, status, abort)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q (queries are the reduction dim, MN-major B)
+        mma_commit(&bars->st_full[hf]);
+      };
+      // dV += P^T_h dO_h, dK += dS^T_h Q_h (queries are the reduction dim, MN-major B)
+      auto issue_acc = [&](int hf, int b, int g) {
+        const uint32_t qb = smem_u32(sQ + b * kTileB), ob = smem_u32(sO + b * kTileB);
+        const uint32_t tS = tmem + 128 * hf, tP = tS + 64;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tV, tS + packed_col(kk), desc_sw128(ob + kk * 2048, kHalf, 1024), idAcc,
-                 (g > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tK, tP + packed_col(kk), desc_sw128(qb + kk * 2048, kHalf, 1024), idAcc,
-                 (g > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const int kq = 4 * hf + kk;                  // 16-query step within the tile
+          const uint32_t acc = (g > 0 || hf > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tV, tS + kk * 8, desc_sw128(ob + kq * 2048, kHalf, 1024), idAcc, acc);
+          mma_ts(tK, tP + kk * 8, desc_sw128(qb + kq * 2048, kHalf, 1024), idAcc, acc);
         }
-        mma_commit(&bars->qd_empty[b]);
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, status, abort) &&
+                mbar_wait(&bars->qd_full[0], 0, status, abort);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0, 0);
+        issue_sdp(1, 0);
+      }
+      for (int g = 0; g < ng && ok; ++g) {
+        const int b = g & 1;
+        const bool more = g + 1 < ng;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          if (!mbar_wait(&bars->pd_full[hf], g & 1, status, abort)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc(hf, b, g);
+          if (hf == 1) mma_commit(&bars->qd_empty[b]);
+          if (more) {
+            if (hf == 0) {
+              if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, status, abort)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            issue_sdp(hf, b ^ 1);
+          }
+        }
       }
       if (ok) mma_commit(&bars->acc_final);
     }
   } else if (warp >= 4) {
-    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
+    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query half
     const int c = wq * 32 + lane;                     // key row of this thread
-    const int cb = 64 * wg;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + 128 * wg + lane_off, tP = tS + 64;
     const bool kvalid = c < nkeys;
+    const uint64_t sl2x2 = f32x2(sl2, sl2);
     bool ok = true;
     for (int g = 0; g < ng && ok; ++g) {
       const int b = g & 1;
       // qd_full also covers sL / sD of this tile
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, status, abort));
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full[wg], g & 1, status, abort));
       if (!ok) break;
       tc_fence_after();
-      const float* L2 = sL + b * kTile + cb;
-      const float* Dq = sD + b * kTile + cb;
+      const float* NL = sL + b * kTile + 64 * wg;
+      const float* Dq = sD + b * kTile + 64 * wg;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {                 // 32 query columns per wait
         uint32_t xs[32], xp[32];
-        tmem_ld32(tS + lane_off + cb + hh * 32, xs);
-        tmem_ld32(tP + lane_off + cb + hh * 32, xp);
+        tmem_ld32(tS + hh * 32, xs);
+        tmem_ld32(tP + hh * 32, xp);
         tmem_ld_wait();
         uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv2[2], dv2[2];
+        for (int e = 0; e < 32; e += 4) {
+          // rows of keys past the tile's end are computed but never stored
+          const float4 nl = *reinterpret_cast<const float4*>(NL + hh * 32 + e);
+          const float4 dd = *reinterpret_cast<const float4*>(Dq + hh * 32 + e);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qi = hh * 32 + e + u;
-            const float pr =
-                kvalid ? fast_exp2(fmaf(__uint_as_float(xs[e + u]), sl2, -L2[qi])) : 0.f;
-            pv2[u] = pr;
-            dv2[u] = pr * (__uint_as_float(xp[e + u]) - Dq[qi]);
+            const int x = e + 2 * u;
+            const uint64_t t = fma_x2(f32x2(__uint_as_float(xs[x]), __uint_as_float(xs[x + 1])),
+                                      sl2x2, u ? f32x2(nl.z, nl.w) : f32x2(nl.x, nl.y));
+            const float2 tt = f32x2_split(t);
+            const float p0 = fast_exp2(tt.x), p1 = fast_exp2(tt.y);
+            const uint64_t dp = sub_x2(f32x2(__uint_as_float(xp[x]), __uint_as_float(xp[x + 1])),
+                                       u ? f32x2(dd.z, dd.w) : f32x2(dd.x, dd.y));
+            const float2 ds = f32x2_split(mul_x2(f32x2(p0, p1), dp));
+            pp[x >> 1] = pack_bf16x2(p0, p1);
+            pd[x >> 1] = pack_bf16x2(ds.x, ds.y);
           }
-          pp[e >> 1] = pack_bf16x2(pv2[0], pv2[1]);
-          pd[e >> 1] = pack_bf16x2(dv2[0], dv2[1]);
         }
-        // P^T, dS^T into the group's columns [cb + 16 hh, +16) (already read)
-        tmem_st16(tS + lane_off + cb + hh * 16, pp);
-        tmem_st16(tP + lane_off + cb + hh * 16, pd);
+        // P^T_h, dS^T_h into columns [16 hh, 16 hh + 16) of S^T_h, dP^T_h (already read)
+        tmem_st16(tS + hh * 16, pp);
+        tmem_st16(tP + hh * 16, pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pd_full);
+      if (lane == 0) mbar_arrive(&bars->pd_full[wg]);
     }
     // epilogue: dK (x scale) and dV of the tile's keys, original key order
     const bool have = ng > 0 && ok &&
@@ -602,10 +642,10 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
   float* part_dq = static_cast<float*>(part);
   const int nkt = (P.L + kTile - 1) / kTile;
   for (int h = 0; h < P.n_h; ++h) {
-    // padding rows get LSE = +inf, so their P is exactly 0
+    // padding rows get -LSE log2(e) = -inf, so their P is exactly 0
     e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q),
                             static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, lse2, rowD,
-                            ib.l2g, ib.dg, INFINITY, num_sms, st);
+                            ib.l2g, ib.dg, -INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
