@@ -58,14 +58,18 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
 }
 
 // =====================================================================
-// dQ pass.  TMEM: S [0,128), dP0 [128,256), dP1 [256,384), dQ [384,512).
-// Roles: warp 0 TMA (the item's Q and dO tiles from the item-ordered copies,
-// then the block's K, V chunks), warp 1 MMA, warps 4-7 softmax rows +
-// epilogue (warps 2-3 idle).
+// dQ pass.  TMEM: S0 [0,128), S1 [128,256), dP [256,384) (then dS), dQ
+// [384,512).  Roles: warp 0 TMA (the item's Q and dO tiles from the
+// item-ordered copies, then the block's K, V chunks), warp 1 MMA, warps
+// 4-7 / 8-11 softmax of key columns 0-63 / 64-127 + epilogue (warps 2-3
+// idle).  Per chunk J the softmax forms P(J) from S(J) and frees S, then
+// dS(J) = P (dP - D) once dP(J) is there; the MMA issue order S(J+1),
+// dQ(J) += dS(J) K, dP(J+1) lets S(J+1) run while dS(J) is formed and
+// dP(J+1) while P(J+1) is.
 // =====================================================================
 struct DqBars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
-  uint64_t s_full[2], s_free, ds_full[2];
+  uint64_t s_full[2], s_free[2], dp_full, ds_full;
   uint64_t qd_full, qd_empty, dq_final, dq_free;
   uint32_t tmem_base;
   int abort;
@@ -78,8 +82,9 @@ static_assert(kDqSmem <= 232448, "shared memory per CTA");
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-             Prob P, int h, PairsView pv, const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
-             float* __restrict__ part_dq, int* __restrict__ status) {
+             Prob P, int h, PairsView pv, const float* __restrict__ dg,
+             const float* __restrict__ l2g, float sl2, float* __restrict__ part_dq,
+             int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -102,9 +107,10 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->full_k[i], 1); mbar_init(&bars->empty_k[i], 1);
       mbar_init(&bars->full_v[i], 1); mbar_init(&bars->empty_v[i], 1);
-      mbar_init(&bars->s_full[i], 1); mbar_init(&bars->ds_full[i], kSoftmaxWarps);
+      mbar_init(&bars->s_full[i], 1); mbar_init(&bars->s_free[i], kSoftmaxWarps);
     }
-    mbar_init(&bars->s_free, kSoftmaxWarps);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->ds_full, kSoftmaxWarps);
     mbar_init(&bars->qd_full, 1);
     mbar_init(&bars->qd_empty, 1);
     mbar_init(&bars->dq_final, 1);
@@ -120,7 +126,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tS = tmem, tDQ = tmem + 384;
+  const uint32_t tdP = tmem + 256, tDQ = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -162,59 +168,74 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       const uint32_t idDQ = idesc_bf16(128, 128, false, true);
       const int ks_last = (kc_last + 15) / 16;
       const uint32_t qb = smem_u32(sQ), ob = smem_u32(sO);
-      int J = 0, it_local = 0, prev_c = -1, prev_it = -1;
+      const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / G + 1 : 0;
+      const int total = my_items * nch;                 // chunks of this CTA
       bool ok = true;
-      // dQ += dS_Jp K_Jp ; dS in dP[Jp & 1] columns [0, 64)
-      auto issue_dq = [&](int Jp, int cp, int itp) -> bool {
-        const int b = Jp & 1;
-        if (!mbar_wait(&bars->ds_full[b], (Jp >> 1) & 1, status, abort)) return false;
-        if (cp == 0 && itp > 0 && !mbar_wait(&bars->dq_free, (itp - 1) & 1, status, abort))
+      // S(J) = Q K^T into S[J & 1]; the chunk's first S of an item waits for its Q / dO
+      auto issue_s = [&](int J) -> bool {
+        const int st = J & 1, c = J % nch, itl = J / nch;
+        if (c == 0 && !mbar_wait(&bars->qd_full, itl & 1, status, abort)) return false;
+        if (J >= 2 && !mbar_wait(&bars->s_free[st], ((J >> 1) - 1) & 1, status, abort))
           return false;
+        if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, status, abort)) return false;
         tc_fence_after();
-        const uint32_t kb = smem_u32(sK + b * kTileB);
-        const uint32_t tdS = tmem + 128 + b * 128;
-        const int ks = cp == nch - 1 ? ks_last : 8;
-        for (int kk = 0; kk < ks; ++kk)
-          mma_ts(tDQ, tdS + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
-                 (cp > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->empty_k[b]);
-        if (cp == nch - 1) mma_commit(&bars->dq_final);
+        const uint32_t kb = smem_u32(sK + st * kTileB);
+        const uint32_t idc = c == nch - 1 ? idSS_last : idSS;   // N = the chunk's keys
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tmem + st * 128, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
+                 idc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[st]);
         return true;
       };
-      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-        if (!mbar_wait(&bars->qd_full, it_local & 1, status, abort)) { ok = false; break; }
+      // dP(J) = dO V^T; overwrites dS(J-1), whose dQ MMA was issued before
+      auto issue_dp = [&](int J) -> bool {
+        const int st = J & 1, c = J % nch;
+        if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, status, abort)) return false;
         tc_fence_after();
-        for (int c = 0; c < nch && ok; ++c, ++J) {
-          const int st = J & 1;
-          if (J > 0 && !mbar_wait(&bars->s_free, (J - 1) & 1, status, abort)) { ok = false; break; }
-          if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, status, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = smem_u32(sK + st * kTileB);
-          const uint32_t idc = c == nch - 1 ? idSS_last : idSS;   // N = the chunk's keys
+        const uint32_t vb = smem_u32(sV + st * kTileB);
+        const uint32_t idc = c == nch - 1 ? idSS_last : idSS;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tS, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idc,
-                   kk > 0 ? 1u : 0u);
-          }
-          if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, status, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t vb = smem_u32(sV + st * kTileB);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tmem + 128 + st * 128, desc_sw128(ob + off, 16, 1024),
-                   desc_sw128(vb + off, 16, 1024), idc, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->empty_v[st]);
-          mma_commit(&bars->s_full[st]);
-          if (c == nch - 1) mma_commit(&bars->qd_empty);
-          if (J > 0) ok = issue_dq(J - 1, prev_c, prev_it);
-          prev_c = c;
-          prev_it = it_local;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tdP, desc_sw128(ob + off, 16, 1024), desc_sw128(vb + off, 16, 1024), idc,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->empty_v[st]);
+        mma_commit(&bars->dp_full);
+        if (c == nch - 1) mma_commit(&bars->qd_empty);  // item's last reader of Q / dO
+        return true;
+      };
+      // dQ += dS(J) K(J); dS packed over the dP columns
+      auto issue_dq = [&](int J) -> bool {
+        const int st = J & 1, c = J % nch, itl = J / nch;
+        if (!mbar_wait(&bars->ds_full, J & 1, status, abort)) return false;
+        if (c == 0 && itl > 0 && !mbar_wait(&bars->dq_free, (itl - 1) & 1, status, abort))
+          return false;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(sK + st * kTileB);
+        const int ks = c == nch - 1 ? ks_last : 8;
+        for (int kk = 0; kk < ks; ++kk)
+          mma_ts(tDQ, tdP + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
+                 (c > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->empty_k[st]);
+        if (c == nch - 1) mma_commit(&bars->dq_final);
+        return true;
+      };
+      if (total > 0) ok = issue_s(0) && issue_dp(0);
+      for (int J = 0; J < total && ok; ++J) {
+        const bool more = J + 1 < total;
+        if (more && (J + 1) % nch == 0) {
+          // next item: its Q / dO arrive after this item's last dP, so issue dQ first
+          ok = issue_dq(J) && issue_s(J + 1) && issue_dp(J + 1);
+        } else if (more) {
+          ok = issue_s(J + 1) && issue_dq(J) && issue_dp(J + 1);
+        } else {
+          ok = issue_dq(J);
         }
       }
-      if (ok && J > 0) issue_dq(J - 1, prev_c, prev_it);
     }
   } else if (warp >= 4) {
     const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, column group
@@ -222,18 +243,20 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const int cb = 64 * wg;                         // this group's key columns
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     float* stg = reinterpret_cast<float*>(sStage + (warp - 4) * kStageB);
+    const uint64_t sl2x2 = f32x2(sl2, sl2);
     int J = 0, it_local = 0;
     bool ok = true;
     for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
       const WorkItem it = decode_item(pv, P, h, n);
       const bool valid = r < it.count;
-      float l2 = 0.f, Di = 0.f;
+      float nl2 = -INFINITY, Di = 0.f;
       uint32_t slot = 0xFFFFFFFFu;
       if (valid) {
         slot = __ldg(col_slot + it.first + r);
-        l2 = __ldg(l2g + (size_t)n * kTile + r);
+        nl2 = __ldg(l2g + (size_t)n * kTile + r);
         Di = __ldg(dg + (size_t)n * kTile + r);
       }
+      const uint64_t nl2x2 = f32x2(nl2, nl2), Dx2 = f32x2(Di, Di);
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, status, abort));
@@ -243,47 +266,57 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         if (lim <= 0) {
           // no key of this chunk in the group's columns: the dQ MMA reads none of them
           __syncwarp();
-          if (lane == 0) { mbar_arrive(&bars->s_free); mbar_arrive(&bars->ds_full[b]); }
+          if (lane == 0) mbar_arrive(&bars->s_free[b]);
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, status, abort));
+          if (!ok) break;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->ds_full);
           continue;
         }
         const bool full = lim >= 64;
-        uint32_t xr[64];
-        tmem_ld32(tS + lane_off + cb, xr);
-        tmem_ld32(tS + lane_off + cb + 32, xr + 32);
+        // P for the group's 64 key columns; rows past the tile's end give P = 0
+        uint32_t pr[64];
+        tmem_ld32(tmem + b * 128 + lane_off + cb, pr);
+        tmem_ld32(tmem + b * 128 + lane_off + cb + 32, pr + 32);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const bool on = valid && (full || e < lim);
-          xr[e] = __float_as_uint(on ? fast_exp2(fmaf(__uint_as_float(xr[e]), sl2, l2)) : 0.f);
+        for (int e = 0; e < 64; e += 2) {
+          const float2 t = f32x2_split(
+              fma_x2(f32x2(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1])), sl2x2, nl2x2));
+          // columns past the chunk's keys: S is not written there, P = 0
+          pr[e] = __float_as_uint((full || e < lim) ? fast_exp2(t.x) : 0.f);
+          pr[e + 1] = __float_as_uint((full || e + 1 < lim) ? fast_exp2(t.y) : 0.f);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free);       // S may be overwritten now
-        const uint32_t tdP = tmem + 128 + b * 128 + lane_off + cb;
+        if (lane == 0) mbar_arrive(&bars->s_free[b]);    // S[b] may be overwritten now
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, status, abort));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {                  // 32 dP columns per wait
           uint32_t dp[32];
-          tmem_ld32(tdP + hh * 32, dp);
+          tmem_ld32(tdP + lane_off + cb + hh * 32, dp);
           tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            // columns past the chunk's keys: dP is not written there, dS = 0
-            const bool on0 = full || hh * 32 + e < lim, on1 = full || hh * 32 + e + 1 < lim;
-            const float d0 =
-                on0 ? __uint_as_float(xr[hh * 32 + e]) * (__uint_as_float(dp[e]) - Di) : 0.f;
-            const float d1 =
-                on1 ? __uint_as_float(xr[hh * 32 + e + 1]) * (__uint_as_float(dp[e + 1]) - Di)
-                    : 0.f;
-            pk[e >> 1] = pack_bf16x2(d0, d1);
+            const int x = hh * 32 + e;
+            // dP past the chunk's keys is stale; P = 0 there must not meet it
+            const uint64_t dd = sub_x2(f32x2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                       Dx2);
+            const float2 ds = f32x2_split(
+                mul_x2(f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1])), dd));
+            pk[e >> 1] = pack_bf16x2((full || x < lim) ? ds.x : 0.f,
+                                     (full || x + 1 < lim) ? ds.y : 0.f);
           }
           // dS into the group's columns [cb + 16 hh, +16): dP columns already read
-          tmem_st16(tdP + hh * 16, pk);
+          tmem_st16(tdP + lane_off + cb + hh * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->ds_full[b]);
+        if (lane == 0) mbar_arrive(&bars->ds_full);
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, status, abort));
@@ -346,21 +379,23 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
 
 // =====================================================================
 // dK/dV pass.  Item = (key tile kt of block j, head h), one CTA each.
-// Each query tile is taken in two halves of 64 queries, half h by softmax
-// warpgroup h, so that one half's exponentials overlap the other half's
-// MMAs.  TMEM: S^T_h [128h, 128h+64) (then P^T_h), dP^T_h [128h+64,
-// 128h+128) (then dS^T_h), dV [256,384), dK [384,512).  MMA issue order:
-// S/dP_0(g), S/dP_1(g), dVdK_0(g), S/dP_0(g+1), dVdK_1(g), S/dP_1(g+1), ...
-// (each S/dP_h overwrites only columns whose dVdK_h was issued before it).
+// TMEM: S^T [0,128) (then P^T), dP^T [128,256) (then dS^T), dV [256,384),
+// dK [384,512).  Two softmax warpgroups split each query tile's columns
+// 64 / 64.  The tile's work is cut where its dependencies allow:
+//   S^T(g)  -> P^T(g) (exponentials)            -> dV(g) += P^T dO
+//   dP^T(g) -> dS^T(g) = P^T (dP^T - D)          -> dK(g) += dS^T Q
+// and the MMA issue order is dV(g), S^T(g+1), dK(g), dP^T(g+1): the next
+// S^T runs while dS^T(g) is formed, dP^T(g+1) while P^T(g+1) is.  Each MMA
+// overwrites only columns whose readers were issued before it.
 // Roles: warp 0 loads the K/V tile once, then each query tile's Q and dO
 // (TMA, item-ordered copies) and -LSE log2(e), D (bulk copies) into two
-// buffers; warp 1 MMA; warps 4-7 / 8-11 softmax of query half 0 / 1 (one
-// key row per thread) and the epilogue (dV / dK).
+// buffers; warp 1 MMA; warps 4-7 / 8-11 softmax of query columns 0-63 /
+// 64-127 (one key row per thread) and the epilogue (dV / dK).
 // =====================================================================
 struct KvBars {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t st_full[2], pd_full[2];
+  uint64_t st_full, dpt_full, p_full, ds_full;
   uint64_t acc_final;
   uint32_t tmem_base;
   int abort;
@@ -400,10 +435,11 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1);
-      mbar_init(&bars->st_full[i], 1); mbar_init(&bars->pd_full[i], 4);
-    }
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
+    mbar_init(&bars->st_full, 1);
+    mbar_init(&bars->dpt_full, 1);
+    mbar_init(&bars->p_full, kSoftmaxWarps);
+    mbar_init(&bars->ds_full, kSoftmaxWarps);
     mbar_init(&bars->acc_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -416,7 +452,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tV = tmem + 256, tK = tmem + 384;
+  const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0 && ng > 0) {
@@ -443,74 +479,66 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else if (warp == 1) {
     if (lane == 0 && ng > 0) {
-      const uint32_t idSS = idesc_bf16(128, 64, false, false);    // keys x 64 queries
+      const uint32_t idSS = idesc_bf16(128, 128, false, false);
       const uint32_t idAcc = idesc_bf16(128, 128, false, true);
       const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
-      // S^T_h = K Q_h^T, dP^T_h = V dO_h^T (K-major both sides; Q_h = rows 64h..)
-      auto issue_sdp = [&](int hf, int b) {
-        const uint32_t qb = smem_u32(sQ + b * kTileB) + hf * 8192;
-        const uint32_t ob = smem_u32(sO + b * kTileB) + hf * 8192;
-        const uint32_t tS = tmem + 128 * hf, tP = tS + 64;
+      // S^T = K Q^T (or dP^T = V dO^T): keys x queries, K-major both sides
+      auto issue_ss = [&](uint32_t tD, uint32_t ab, uint32_t bb) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tS, desc_sw128(kb + off, 16, 1024), desc_sw128(qb + off, 16, 1024), idSS,
+          mma_ss(tD, desc_sw128(ab + off, 16, 1024), desc_sw128(bb + off, 16, 1024), idSS,
                  kk > 0 ? 1u : 0u);
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tP, desc_sw128(vb + off, 16, 1024), desc_sw128(ob + off, 16, 1024), idSS,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->st_full[hf]);
       };
-      // dV += P^T_h dO_h, dK += dS^T_h Q_h (queries are the reduction dim, MN-major B)
-      auto issue_acc = [&](int hf, int b, int g) {
-        const uint32_t qb = smem_u32(sQ + b * kTileB), ob = smem_u32(sO + b * kTileB);
-        const uint32_t tS = tmem + 128 * hf, tP = tS + 64;
+      // acc += A^T B with A^T packed in TMEM, B = Q or dO (queries = reduction, MN-major)
+      auto issue_acc = [&](uint32_t tD, uint32_t tA, uint32_t bb, int g) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int kq = 4 * hf + kk;                  // 16-query step within the tile
-          const uint32_t acc = (g > 0 || hf > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(tV, tS + kk * 8, desc_sw128(ob + kq * 2048, kHalf, 1024), idAcc, acc);
-          mma_ts(tK, tP + kk * 8, desc_sw128(qb + kq * 2048, kHalf, 1024), idAcc, acc);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tD, tA + packed_col(kk), desc_sw128(bb + kk * 2048, kHalf, 1024), idAcc,
+                 (g > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&bars->kv_full, 0, status, abort) &&
                 mbar_wait(&bars->qd_full[0], 0, status, abort);
       if (ok) {
         tc_fence_after();
-        issue_sdp(0, 0);
-        issue_sdp(1, 0);
+        issue_ss(tS, kb, smem_u32(sQ));
+        mma_commit(&bars->st_full);
+        issue_ss(tP, vb, smem_u32(sO));
+        mma_commit(&bars->dpt_full);
       }
       for (int g = 0; g < ng && ok; ++g) {
         const int b = g & 1;
         const bool more = g + 1 < ng;
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          if (!mbar_wait(&bars->pd_full[hf], g & 1, status, abort)) { ok = false; break; }
-          tc_fence_after();
-          issue_acc(hf, b, g);
-          if (hf == 1) mma_commit(&bars->qd_empty[b]);
-          if (more) {
-            if (hf == 0) {
-              if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, status, abort)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            issue_sdp(hf, b ^ 1);
+        const uint32_t qb = smem_u32(sQ + b * kTileB), ob = smem_u32(sO + b * kTileB);
+        if (!mbar_wait(&bars->p_full, g & 1, status, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(tV, tS, ob, g);                       // dV += P^T dO
+        if (more) {
+          if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, status, abort)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          issue_ss(tS, kb, smem_u32(sQ + (b ^ 1) * kTileB));   // S^T(g+1)
+          mma_commit(&bars->st_full);
+        }
+        if (!mbar_wait(&bars->ds_full, g & 1, status, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(tK, tP, qb, g);                       // dK += dS^T Q
+        mma_commit(&bars->qd_empty[b]);
+        if (more) {
+          issue_ss(tP, vb, smem_u32(sO + (b ^ 1) * kTileB));   // dP^T(g+1)
+          mma_commit(&bars->dpt_full);
         }
       }
       if (ok) mma_commit(&bars->acc_final);
     }
   } else if (warp >= 4) {
-    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query half
+    const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
     const int c = wq * 32 + lane;                     // key row of this thread
+    const int cb = 64 * wg;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + 128 * wg + lane_off, tP = tS + 64;
     const bool kvalid = c < nkeys;
     const uint64_t sl2x2 = f32x2(sl2, sl2);
     bool ok = true;
@@ -519,45 +547,74 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       // qd_full also covers sL / sD of this tile
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, status, abort));
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full[wg], g & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, status, abort));
       if (!ok) break;
       tc_fence_after();
-      const float* NL = sL + b * kTile + 64 * wg;
-      const float* Dq = sD + b * kTile + 64 * wg;
+      const float* NL = sL + b * kTile + cb;
+      const float* Dq = sD + b * kTile + cb;
+      // P^T for the group's 64 query columns (kept in fp32 for dS^T);
+      // rows of keys past the tile's end are computed but never stored
+      uint32_t pr[64];
+      tmem_ld32(tS + lane_off + cb, pr);
+      tmem_ld32(tS + lane_off + cb + 32, pr + 32);
+      tmem_ld_wait();
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {                 // 32 query columns per wait
-        uint32_t xs[32], xp[32];
-        tmem_ld32(tS + hh * 32, xs);
-        tmem_ld32(tP + hh * 32, xp);
-        tmem_ld_wait();
-        uint32_t pp[16], pd[16];
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pp[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          // rows of keys past the tile's end are computed but never stored
-          const float4 nl = *reinterpret_cast<const float4*>(NL + hh * 32 + e);
-          const float4 dd = *reinterpret_cast<const float4*>(Dq + hh * 32 + e);
+          const int x = hh * 32 + e;
+          const float4 nl = *reinterpret_cast<const float4*>(NL + x);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int x = e + 2 * u;
-            const uint64_t t = fma_x2(f32x2(__uint_as_float(xs[x]), __uint_as_float(xs[x + 1])),
-                                      sl2x2, u ? f32x2(nl.z, nl.w) : f32x2(nl.x, nl.y));
-            const float2 tt = f32x2_split(t);
-            const float p0 = fast_exp2(tt.x), p1 = fast_exp2(tt.y);
-            const uint64_t dp = sub_x2(f32x2(__uint_as_float(xp[x]), __uint_as_float(xp[x + 1])),
-                                       u ? f32x2(dd.z, dd.w) : f32x2(dd.x, dd.y));
-            const float2 ds = f32x2_split(mul_x2(f32x2(p0, p1), dp));
-            pp[x >> 1] = pack_bf16x2(p0, p1);
-            pd[x >> 1] = pack_bf16x2(ds.x, ds.y);
+            const int y = x + 2 * u;
+            const float2 t = f32x2_split(
+                fma_x2(f32x2(__uint_as_float(pr[y]), __uint_as_float(pr[y + 1])), sl2x2,
+                       u ? f32x2(nl.z, nl.w) : f32x2(nl.x, nl.y)));
+            const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
+            pr[y] = __float_as_uint(p0);
+            pr[y + 1] = __float_as_uint(p1);
+            pp[(e >> 1) + u] = pack_bf16x2(p0, p1);
           }
         }
-        // P^T_h, dS^T_h into columns [16 hh, 16 hh + 16) of S^T_h, dP^T_h (already read)
-        tmem_st16(tS + hh * 16, pp);
-        tmem_st16(tP + hh * 16, pd);
+        // P^T into the group's columns [cb + 16 hh, +16) (S^T already read)
+        tmem_st16(tS + lane_off + cb + hh * 16, pp);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pd_full[wg]);
+      if (lane == 0) mbar_arrive(&bars->p_full);
+      // dS^T = P^T (dP^T - D)
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dpt_full, g & 1, status, abort));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t xp[32];
+        tmem_ld32(tP + lane_off + cb + hh * 32, xp);
+        tmem_ld_wait();
+        uint32_t pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int x = hh * 32 + e;
+          const float4 dd = *reinterpret_cast<const float4*>(Dq + x);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int y = e + 2 * u;
+            const uint64_t dp = sub_x2(f32x2(__uint_as_float(xp[y]), __uint_as_float(xp[y + 1])),
+                                       u ? f32x2(dd.z, dd.w) : f32x2(dd.x, dd.y));
+            const float2 ds = f32x2_split(mul_x2(
+                f32x2(__uint_as_float(pr[x + 2 * u]), __uint_as_float(pr[x + 2 * u + 1])), dp));
+            pd[(e >> 1) + u] = pack_bf16x2(ds.x, ds.y);
+          }
+        }
+        // dS^T into the group's columns [cb + 16 hh, +16) (dP^T already read)
+        tmem_st16(tP + lane_off + cb + hh * 16, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_full);
     }
     // epilogue: dK (x scale) and dV of the tile's keys, original key order
     const bool have = ng > 0 && ok &&
