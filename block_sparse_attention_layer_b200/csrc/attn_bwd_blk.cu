@@ -422,8 +422,10 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   KvBars* bars = reinterpret_cast<KvBars*>(sD + 2 * kTile);
   volatile int* abort = &bars->abort;
 
+  // longest query lists first (the hardware hands out CTAs in index order)
   const int nkt = (P.L + kTile - 1) / kTile;
-  const int j = blockIdx.x / nkt, kt = blockIdx.x - j * nkt;
+  const int rk = blockIdx.x / nkt, kt = blockIdx.x - rk * nkt;
+  const int j = (int)__ldg(pv.blk_order + (size_t)h * P.Nb + rk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
   const int item0 = (int)__ldg(pv.item_off + (size_t)h * (P.Nb + 1) + j);

@@ -13,7 +13,10 @@
 //                CSR partials directly;
 //   item_off[j]  first work item of block j: its query list cut into tiles of
 //                128 queries; item_off[N_b] = number of work items;
-//   pitem_off[j] the same for pairs of consecutive tiles (256 queries).
+//   pitem_off[j] the same for pairs of consecutive tiles (256 queries);
+//   blk_order    the blocks by list length, longest first (ties: lower j
+//                first), so that kernels launching one CTA per block start
+//                the longest ones first.
 // Rows are processed in chunks of 256 (8 warps x 32 rows); per-chunk column
 // counts give each chunk's base inside every block list, and warp ballots
 // give each row's rank inside the chunk.
@@ -85,8 +88,9 @@ __global__ void __launch_bounds__(1024)
 k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict__ chunk_cnt,
              int n_chunks, uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_off,
              uint32_t* __restrict__ item_off, uint32_t* __restrict__ pitem_off,
-             uint32_t* __restrict__ head_totals) {
+             uint32_t* __restrict__ head_totals, uint32_t* __restrict__ blk_order) {
   __shared__ uint32_t sh[32];
+  __shared__ uint32_t len[kMaxBlocks];
   const int h = blockIdx.x, t = threadIdx.x;
   uint32_t* cc = chunk_cnt + (size_t)h * n_chunks * P.Nb;
   // column totals (one thread per block)
@@ -99,6 +103,13 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
   uint32_t n_items, n_pitems;
   const uint32_t ioff = block_excl_scan(tiles, sh, &n_items);
   const uint32_t poff = block_excl_scan((tiles + 1) / 2, sh, &n_pitems);
+  if (t < P.Nb) len[t] = tot;
+  __syncthreads();
+  if (t < P.Nb) {
+    uint32_t rank = 0;
+    for (int u = 0; u < P.Nb; ++u) rank += (len[u] > tot || (len[u] == tot && u < t)) ? 1u : 0u;
+    blk_order[(size_t)h * P.Nb + rank] = (uint32_t)t;
+  }
   if (t < P.Nb) {
     col_off[(size_t)h * (P.Nb + 1) + t] = off;
     item_off[(size_t)h * (P.Nb + 1) + t] = ioff;
@@ -194,6 +205,7 @@ size_t pairs_ws_bytes(const Prob& P) {
   take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);     // chunk counts / bases
   take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_rows (worst case)
   take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_slot (worst case)
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);                // blk_order
   return b;
 }
 
@@ -211,6 +223,7 @@ PairsView pairs_view(const Prob& P, void* base) {
   v.chunk = take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);
   v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
   v.col_slot = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
+  v.blk_order = take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);
   v.n_chunks = n_chunks;
   return v;
 }
@@ -224,7 +237,7 @@ cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v,
   {
     VMOBA_TRACE("k_pairs_scan", st);
     k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
-                                         v.item_off, v.pitem_off, v.head_totals);
+                                         v.item_off, v.pitem_off, v.head_totals, v.blk_order);
   }
   {
     VMOBA_TRACE("k_pairs_fill", st);

@@ -15,6 +15,7 @@ struct PairsView {
   uint32_t* chunk;        // [n_h][chunks][N_b] scratch (chunk bases)
   uint32_t* col_rows;     // [n_h][s*N_b] query lists, block by block
   uint32_t* col_slot;     // [n_h][s*N_b] pair slot of each list entry
+  uint32_t* blk_order;    // [n_h][N_b]   blocks by query-list length, longest first
   int n_chunks;
 };
 
