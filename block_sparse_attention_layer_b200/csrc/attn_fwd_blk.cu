@@ -6,10 +6,12 @@
 // from block j's query list); every query of the tile selected block j, so
 // the tile attends all keys of the block with no per-row masking and no
 // wasted pairs.  The item computes, for each of its queries, the partial
-// softmax state of block j (running max m, sum l, unnormalised O) over the
-// block's keys in chunks of 128 and stores it in the pair's slot.  A merge
-// kernel then combines the partials of each query with log-sum-exp weights
-// into O, its fp32 copy and LSE.
+// softmax state of block j (running max m, sum l, and O / l) over the
+// block's keys in chunks of 128 and stores it in the pair's slot: (m, l) in
+// fp32, O / l in fp16 -- a convex combination of V rows, so |O / l| <= max
+// |V| and fp16 keeps it to 2^-12 relative, below the bf16 output's rounding.
+// A merge kernel then combines the partials of each query with log-sum-exp
+// weights into O, its fp32 copy and LSE.
 //
 // Persistent kernel, one head per launch.  A CTA takes PAIRS of work items
 // (two consecutive 128-query tiles A, B of one block's list) so that every
@@ -119,7 +121,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, 
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const __grid_constant__ CUtensorMap tm_q, Prob P, int h, PairsView pv, float sl2,
-          float* __restrict__ part_o, float2* __restrict__ part_ml, int* __restrict__ status) {
+          __half* __restrict__ part_o, float2* __restrict__ part_ml, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -309,26 +311,36 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       if (!ok) break;
       tc_fence_after();
       if (valid) part_ml[slot] = make_float2(m_run, l_run);
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint32_t* stw = reinterpret_cast<uint32_t*>(stg);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t ob[32];
-        tmem_ld32(tO + cc * 32, ob);
+      for (int cc = 0; cc < 2; ++cc) {               // 64 columns: 128 fp16 bytes per row
+        uint32_t ob[64];
+        tmem_ld32(tO + cc * 64, ob);
+        tmem_ld32(tO + cc * 64 + 32, ob + 32);
         tmem_ld_wait();
         // row `lane` into the staging tile, 16-byte granules XOR-swizzled by row
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          *reinterpret_cast<float4*>(stg + lane * 32 + ((g ^ (lane & 7)) << 2)) =
-              make_float4(__uint_as_float(ob[4 * g]), __uint_as_float(ob[4 * g + 1]),
-                          __uint_as_float(ob[4 * g + 2]), __uint_as_float(ob[4 * g + 3]));
+        for (int g = 0; g < 8; ++g) {
+          uint4 u;
+          u.x = pack_f16x2(__uint_as_float(ob[8 * g]) * inv_l, __uint_as_float(ob[8 * g + 1]) * inv_l);
+          u.y = pack_f16x2(__uint_as_float(ob[8 * g + 2]) * inv_l,
+                           __uint_as_float(ob[8 * g + 3]) * inv_l);
+          u.z = pack_f16x2(__uint_as_float(ob[8 * g + 4]) * inv_l,
+                           __uint_as_float(ob[8 * g + 5]) * inv_l);
+          u.w = pack_f16x2(__uint_as_float(ob[8 * g + 6]) * inv_l,
+                           __uint_as_float(ob[8 * g + 7]) * inv_l);
+          *reinterpret_cast<uint4*>(stw + lane * 32 + ((g ^ (lane & 7)) << 2)) = u;
+        }
         __syncwarp();
         // eight lanes per row: four whole 128-byte lines per store instruction
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int rr = 4 * k + (lane >> 3), g = lane & 7;
-          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 32 + ((g ^ (rr & 7)) << 2));
+          const uint4 v = *reinterpret_cast<const uint4*>(stw + rr * 32 + ((g ^ (rr & 7)) << 2));
           const uint32_t sl = __shfl_sync(0xffffffffu, slot, rr);
           if (sl != 0xFFFFFFFFu)
-            *reinterpret_cast<float4*>(part_o + (size_t)sl * kD + cc * 32 + g * 4) = v;
+            *reinterpret_cast<uint4*>(part_o + (size_t)sl * kD + cc * 64 + g * 8) = v;
         }
         __syncwarp();
       }
@@ -345,11 +357,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   }
 }
 
-// Combine the partial (m, l, O) of every query's selected blocks:
-// O_i = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j, LSE_i = (M + log2 L) ln 2.
+// Combine the partial (m, l, O / l) of every query's selected blocks:
+// O_i = sum_j 2^(m_j - M) l_j (O / l)_j / sum_j 2^(m_j - M) l_j,
+// LSE_i = (M + log2 sum_j 2^(m_j - M) l_j) ln 2.
 // One warp per query row, four dims per lane, blocks in ascending order.
 __global__ void __launch_bounds__(256)
-k_fwd_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_o,
+k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
             const float2* __restrict__ part_ml, __nv_bfloat16* __restrict__ out,
             float* __restrict__ o32, float* __restrict__ lse) {
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -362,11 +375,12 @@ k_fwd_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_o,
   float Lsum = 0.f;
   for (uint32_t k = 0; k < cnt; ++k) {
     const float2 ml = part_ml[off + k];
-    const float w = exp2f(ml.x - M);
-    Lsum = fmaf(w, ml.y, Lsum);
-    const float4 o = reinterpret_cast<const float4*>(part_o + (size_t)(off + k) * 128)[lane];
-    acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
-    acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
+    const float wl = exp2f(ml.x - M) * ml.y;
+    Lsum += wl;
+    const uint2 u = reinterpret_cast<const uint2*>(part_o + (size_t)(off + k) * 128)[lane];
+    const float2 a = unpack_f16x2(u.x), b = unpack_f16x2(u.y);
+    acc.x = fmaf(wl, a.x, acc.x); acc.y = fmaf(wl, a.y, acc.y);
+    acc.z = fmaf(wl, b.x, acc.z); acc.w = fmaf(wl, b.y, acc.w);
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
@@ -400,7 +414,7 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
   cudaError_t e = cudaFuncSetAttribute(k_fwd_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  float* part_o = static_cast<float*>(part);
+  __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
   float2* part_ml = reinterpret_cast<float2*>(
       static_cast<char*>(part) + align_up((size_t)P.s * P.Nb * 128 * sizeof(float), 256));
   const float sl2 = scale * 1.4426950408889634f;

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include <cuda_fp16.h>
 
 namespace vmoba {
 namespace tc {
@@ -248,6 +249,15 @@ __device__ __forceinline__ uint64_t sub_x2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
