@@ -47,6 +47,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile-layer", type=int, default=None,
+                    help="profiling case for ncu: run layer L of the workload (its partition "
+                         "mode) twice with --heads heads, print per-call times, no timed bench")
+    ap.add_argument("--heads", type=int, default=2)
     return ap.parse_args()
 
 
@@ -504,8 +508,51 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """One layer of the bench workload with few heads (same per-head sizes), run
+    twice: a small case for ncu captures, whose launches are per head like the
+    bench's."""
+    import numpy as np
+    import torch
+
+    import synth
+    from synth.video_latents import round_to
+    from block_sparse_attention_layer_b200 import LayerShape, metrics
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    mode = args.profile_layer % 3
+    nh = args.heads
+    q, k, v = synth.make_qkv(w.wid, 0, w.T, w.H, w.W, nh, w.head_dim, kind=w.kind)
+    do = synth.make_dout(w.wid, 0, w.s, nh, w.head_dim)
+    q, k, v, do = (torch.from_numpy(round_to(x, "bf16").astype(np.float32))
+                   .to(torch.bfloat16).cuda() for x in (q, k, v, do))
+    sh = LayerShape(w.T, w.H, w.W, nh, w.head_dim, mode, *w.boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    times = []
+    for _ in range(2):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record()
+        L.select(q, k, v, TAU)
+        ev[1].record()
+        L.forward(q)
+        ev[2].record()
+        L.backward(q, do)
+        ev[3].record()
+        torch.cuda.synchronize()
+        times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(3)])
+    st = L.head_stats()
+    pairs = metrics.token_pairs_from_stats(st["n_selected"], L.block_len)
+    print(json.dumps({"case": f"layer {args.profile_layer} (mode {mode}), {nh} heads",
+                      "select_ms": round(times[-1][0], 4), "fwd_ms": round(times[-1][1], 4),
+                      "bwd_ms": round(times[-1][2], 4),
+                      "density": round(pairs / (sh.s * sh.s * nh), 5)}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.profile_layer is not None:
+        run_profile_case(args)
+        return
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
