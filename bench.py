@@ -261,6 +261,10 @@ def run_ours(args, rank, world, local):
         tr = V.trace_read()
         kern_layer[f"l{li}"] = {n: round(ms, 4) for n, (_, ms) in tr.items() if ms >= 0.05}
 
+    # the paper's own block counts (8 / 48 / 72) on the same inputs, untimed by
+    # the headline: density and ms per layer beside the main workload's
+    second = paper_block_counts(V, w, (q, k, v, dout), stream)
+
     # per-call device times (ms, summed over layers, averaged over steps)
     call_ms = {c: 0.0 for c in CALLS}
     layer_call_ms = [[0.0] * len(CALLS) for _ in layers]
@@ -336,6 +340,7 @@ def run_ours(args, rank, world, local):
             "detail": {
                 "call_ms_per_step": {c: round(call_ms[c], 4) for c in CALLS},
                 "kernel_ms_per_layer": kern_layer,
+                "blocks_8_48_72": second,
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
                                   for i, l in enumerate(LAYERS)},
                 "achieved": {c: [round(x[0], 3), x[1]] for c, x in achieved.items()},
@@ -349,6 +354,50 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def paper_block_counts(V, w, tensors, stream, warm=2, reps=3):
+    """Each partition mode with the paper's 8-48-72 block counts (same q, k, v,
+    dO): selected density and device ms of one layer (partition, select, plan,
+    forward, backward), averaged over ``reps`` after ``warm`` runs."""
+    import torch
+
+    import synth
+    from block_sparse_attention_layer_b200 import LayerShape, metrics
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+    q, k, v, dout = tensors
+    res = {"boxes": [list(b) for b in synth.BOXES_8_48_72], "n_blocks": [], "density": [],
+           "ms_per_layer": [], "tflops": []}
+    for mode, box in enumerate(synth.BOXES_8_48_72):
+        sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *box, "bf16")
+        L = VMoBALayer(sh)
+
+        def layer():
+            V.partition(L.shape, k, v, L.k_perm, L.v_perm, L.blocks)
+            V.score_select(L.shape, q, L.blocks, TAU, 0.0, L.sel, L.stats, L.ws)
+            V.build_plan(L.shape, L.sel, L.ws)
+            L.forward(q)
+            L.backward(q, dout)
+
+        for _ in range(warm):
+            layer()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            layer()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        st = L.head_stats()
+        pairs = metrics.token_pairs_from_stats(st["n_selected"], L.block_len)
+        fl = metrics.attention_flops(pairs, w.head_dim, True, True)
+        res["n_blocks"].append(int(V.num_blocks(sh)))
+        res["density"].append(round(pairs / (sh.s * sh.s * sh.n_heads), 5))
+        res["ms_per_layer"].append(round(ms, 4))
+        res["tflops"].append(round(fl / (ms * 1e-3) / 1e12, 2))
+        del L
+    return res
 
 
 def kernel_traffic(name, w):

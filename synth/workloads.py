@@ -52,3 +52,10 @@ WORKLOADS = {
                 ((1, 45, 80), (21, 9, 8), (3, 9, 8)), (0.1, 0.25, 0.5), True,
                 head_gain=True, layers=30, notes="30-layer sweep, mode = layer mod 3"),
 }
+
+# The paper's own block counts on the 55296-token latent: 8 / 48 / 72 blocks
+# for 1D / 2D / 3D (VMoBA notes, training strategy).  The pages give counts,
+# not boxes: 1D is 3 frames per block; 2D is the 6x8 spatial box of workload
+# 4; 3D is workload 4's 4x6x8 box doubled in height and width (4x12x16).
+BOXES_8_48_72 = ((3, 36, 64), (24, 6, 8), (4, 12, 16))
+

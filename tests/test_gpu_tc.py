@@ -204,3 +204,58 @@ def test_tc_backward_full_size(mode):
             keys = np.flatnonzero(blk == j)
             assert out_err(gk[keys, h], dk_ref[keys], "bf16") <= TOL["bf16"]
             assert out_err(gv[keys, h], dv_ref[keys], "bf16") <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("mode", [0, 2])
+def test_paper_block_counts_fwd_bwd(mode):
+    """The paper's 8-48-72 block counts on the 55296-token latent (1D: 3-frame
+    blocks of 6912 keys; 3D: 4x12x16 boxes of 768 keys; 2D is workload 4's):
+    full pair sets of two heads, then forward rows and dQ rows on the oracle's
+    pairs, and every key of the least-selected block."""
+    w = synth.WORKLOADS[4]
+    box_cfg = synth.BOXES_8_48_72[mode]
+    nh = 2
+    tau = 0.25
+    scale = 1 / math.sqrt(128)
+    q, k, v = synth.make_qkv(w.wid, 20 + mode, w.T, w.H, w.W, nh, w.head_dim)
+    dout = synth.make_dout(w.wid, 20 + mode, w.s, nh, w.head_dim)
+    q, k, v, dout = (round_to(x, "bf16") for x in (q, k, v, dout))
+    sh = LayerShape(w.T, w.H, w.W, nh, w.head_dim, mode, *box_cfg, "bf16")
+    L = VMoBALayer(sh)
+    qd = to_device(q, "bf16")
+    L.select(qd, to_device(k, "bf16"), to_device(v, "bf16"), tau)
+    torch.cuda.synchronize()
+    box = O.mode_box(mode, w.T, w.H, w.W, *box_cfg)
+    B = O.pool_blocks(k, w.T, w.H, w.W, box)
+    blk = O.block_of_token(w.T, w.H, w.W, box)
+    bits = L.sel.cpu().numpy().copy()
+    g = unpack_bits(bits, L.n_blocks)
+    for h in range(nh):
+        S_h = O.block_scores(q[:, h:h + 1], B[h:h + 1], scale)[0]
+        m, st = O.threshold_select(S_h, tau)
+        assert pair_set_mismatch(g[h], S_h, m, st["cut_score"]) == 0
+        bits[h] = pack_bits(m)
+        g[h] = m
+    L.use_selection(torch.from_numpy(bits).cuda())
+    out, _ = L.forward(qd)
+    dq, dk, dv = L.backward(qd, to_device(dout, "bf16"))
+    torch.cuda.synchronize()
+    go, gq, gk, gv = from_device(out), from_device(dq), from_device(dk), from_device(dv)
+    for h in range(nh):
+        empty = np.flatnonzero(~g[h].any(axis=1))[:8]
+        rows = sample_rows(w.s, 96, seed=300 + h, must=empty)
+        o_ref, _ = O.attention_fwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows)
+        assert out_err(go[rows, h], o_ref, "bf16") <= TOL["bf16"]
+        dq_ref, _, _ = O.attention_bwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows,
+                                            dout[rows, h])
+        assert out_err(gq[rows, h], dq_ref, "bf16") <= TOL["bf16"]
+        counts = g[h].sum(axis=0)
+        order = [j for j in np.argsort(counts, kind="stable") if counts[j] > 0]
+        j = order[0]
+        if counts[j] <= 1024:
+            qrows = np.flatnonzero(g[h][:, j])
+            _, dk_ref, dv_ref = O.attention_bwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale,
+                                                     qrows, dout[qrows, h])
+            keys = np.flatnonzero(blk == j)
+            assert out_err(gk[keys, h], dk_ref[keys], "bf16") <= TOL["bf16"]
+            assert out_err(gv[keys, h], dv_ref[keys], "bf16") <= TOL["bf16"]
