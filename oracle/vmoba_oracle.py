@@ -34,6 +34,14 @@ step open, the reading taken is stated in the function's docstring:
    the result: 0.03 at |x| = 9 in bf16) is not an error of the computation,
    so tolerances apply to |stored - exact| - half_ulp(exact) (io_excess_error);
    round_io gives the rounded exact value itself.
+10. The ablation's selection variants (notes, ablation table rows "topk +
+    global", "threshold + local", "topk + local (about MoBA's selection)";
+    digest App. A, training-free runs: 3D blocks with MoBA's local top-k):
+    "local" normalises each query row's own N_b scores with a softmax at the
+    same temperature and selects per row; "top-k" keeps a fixed count -- k
+    pairs of the head's pool (global) or k blocks per query row (local) --
+    ranked like the method, ties by index.  The pages give no k; it is a
+    parameter here.
 
 Pins (what ties each function to something other than itself) are in
 ``tests/test_oracle_pins.py``; each function's docstring lists them.
@@ -191,6 +199,95 @@ def select_all_heads(S: np.ndarray, tau: float):
         masks.append(m)
         stats.append(st)
     return np.stack(masks), stats
+
+
+# --------------------------------------------------------------------------
+# Selection variants of the ablation (notes, ablation table: the method is
+# "threshold + global"; the other rows replace the threshold by a fixed
+# count, the global pool by per-query selection, or both; digest App. A)
+# --------------------------------------------------------------------------
+
+def topk_global_select(S_h: np.ndarray, k: int):
+    """"topk + global": the k pairs of the head's whole pool ranked first by
+    (S desc, query asc, block asc) -- the method's ranking with a fixed count
+    in place of the mass threshold (reading 10).
+
+    Returns (mask [s][N_b] bool, stats) with stats = dict(k, cut_score, mass),
+    mass under the head's pool normalisation (reading 1).
+    Pinned: equals threshold_select when k is that selection's k*; the kept
+    set has the largest score sum of all k-subsets (brute force on tiny
+    pools); nested in k; a constant pool keeps the first k flat indices.
+    """
+    if not (k >= 1) or int(k) != k:
+        raise ValueError("k must be a positive integer")
+    flat = S_h.reshape(-1)
+    k = min(int(k), flat.size)
+    order = np.argsort(-flat, kind="stable")
+    mask = np.zeros(flat.size, dtype=bool)
+    mask[order[:k]] = True
+    p = normalised_pool(S_h).reshape(-1)
+    stats = dict(k=k, cut_score=float(flat[order[k - 1]]), mass=float(p[order[:k]].sum()))
+    return mask.reshape(S_h.shape), stats
+
+
+def _row_softmax(row: np.ndarray) -> np.ndarray:
+    e = np.exp(row - row.max())
+    return e / e.sum()
+
+
+def threshold_local_select(S_h: np.ndarray, tau: float):
+    """"threshold + local": per query row, p = softmax of the row's own N_b
+    scores; rank the row's blocks (S desc, block asc) and keep the shortest
+    prefix whose mass reaches tau (every block if rounding leaves the total
+    short) -- key design 3's rule applied to one row (reading 10).
+
+    Returns (mask, stats) with stats = dict(k (pairs), cut_scores [s] (score
+    of each row's last kept block), mass (mean kept mass per row)).
+    Pinned: one query row equals threshold_select; per-row minimality
+    (kept mass >= tau > mass without the last block); the kept set has the
+    fewest blocks reaching tau and the largest mass among such sets (brute
+    force on tiny rows); every row keeps >= 1 block.
+    """
+    if not (tau > 0.0) or math.isnan(tau):
+        raise ValueError("tau must be > 0")
+    s, nb = S_h.shape
+    mask = np.zeros((s, nb), dtype=bool)
+    cuts = np.empty(s)
+    kept = np.empty(s)
+    for i in range(s):
+        p = _row_softmax(S_h[i])
+        order = np.argsort(-S_h[i], kind="stable")
+        c = np.cumsum(p[order])
+        reached = np.flatnonzero(c >= tau)
+        k = int(reached[0]) + 1 if reached.size else nb
+        mask[i, order[:k]] = True
+        cuts[i] = S_h[i, order[k - 1]]
+        kept[i] = c[k - 1]
+    return mask, dict(k=int(mask.sum()), cut_scores=cuts, mass=float(kept.mean()))
+
+
+def topk_local_select(S_h: np.ndarray, k: int):
+    """"topk + local" (about MoBA's selection): each query row keeps its
+    min(k, N_b) blocks ranked first by (S desc, block asc) (reading 10).
+
+    Returns (mask, stats) as threshold_local_select, mass under the row
+    softmax.  Pinned: every row keeps exactly min(k, N_b); one query row
+    equals topk_global_select; the kept blocks have the largest score sum of
+    all k-subsets of the row (brute force on tiny rows).
+    """
+    if not (k >= 1) or int(k) != k:
+        raise ValueError("k must be a positive integer")
+    s, nb = S_h.shape
+    k = min(int(k), nb)
+    mask = np.zeros((s, nb), dtype=bool)
+    cuts = np.empty(s)
+    kept = np.empty(s)
+    for i in range(s):
+        order = np.argsort(-S_h[i], kind="stable")
+        mask[i, order[:k]] = True
+        cuts[i] = S_h[i, order[k - 1]]
+        kept[i] = _row_softmax(S_h[i])[order[:k]].sum()
+    return mask, dict(k=int(mask.sum()), cut_scores=cuts, mass=float(kept.mean()))
 
 
 # --------------------------------------------------------------------------

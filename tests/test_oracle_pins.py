@@ -204,6 +204,105 @@ def test_selection_tie_break_and_full_threshold():
         O.threshold_select(S, float("nan"))
 
 
+# -------------------------------------------- selection variants (ablation)
+
+def _brute_best_k_subset(x, k):
+    """Largest sum of any k-subset of x (enumeration)."""
+    return max(sum(x[list(c)]) for c in itertools.combinations(range(x.size), k))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_global_brute_force_and_nesting(seed):
+    rng = np.random.default_rng(300 + seed)
+    S = rng.standard_normal((3, 4)) * (1 + seed)
+    flat = S.reshape(-1)
+    prev = None
+    for k in range(1, flat.size + 1):
+        mask, st = O.topk_global_select(S, k)
+        m = mask.reshape(-1)
+        assert m.sum() == k == st["k"]
+        assert math.isclose(flat[m].sum(), _brute_best_k_subset(flat, k), rel_tol=1e-12)
+        e = np.exp(S - S.max())
+        assert math.isclose(st["mass"], (e / e.sum()).reshape(-1)[m].sum(), rel_tol=1e-12)
+        if prev is not None:
+            assert np.all(m[prev])
+        prev = m
+    assert O.topk_global_select(S, 10 ** 6)[0].all()
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("tau", [0.1, 0.25, 0.6])
+def test_topk_global_at_k_star_is_the_threshold_rule(seed, tau):
+    # the method's rule is a prefix of the same ranking: its k* pairs are the top-k*
+    rng = np.random.default_rng(400 + seed)
+    S = rng.standard_normal((40, 9)) * 2.0
+    m_thr, st = O.threshold_select(S, tau)
+    m_top, st2 = O.topk_global_select(S, st["k"])
+    assert np.array_equal(m_thr, m_top)
+    assert math.isclose(st["mass"], st2["mass"], rel_tol=1e-12)
+
+
+def test_topk_global_ties_and_arguments():
+    mask, st = O.topk_global_select(np.zeros((3, 2)), 4)     # constant pool
+    assert mask.reshape(-1).tolist() == [True] * 4 + [False] * 2
+    for bad in (0, -1, 1.5):
+        with pytest.raises(ValueError):
+            O.topk_global_select(np.zeros((2, 2)), bad)
+
+
+def _brute_min_card_row(p, tau):
+    for k in range(1, p.size + 1):
+        best = _brute_best_k_subset(p, k)
+        if best >= tau:
+            return k, best
+    return p.size, p.sum()
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("tau", [0.2, 0.5, 0.9])
+def test_threshold_local_brute_force_per_row(seed, tau):
+    rng = np.random.default_rng(500 + seed)
+    S = rng.standard_normal((5, 6)) * (0.5 + seed)
+    mask, st = O.threshold_local_select(S, tau)
+    masses = []
+    for i in range(S.shape[0]):
+        e = np.exp(S[i] - S[i].max())
+        p = e / e.sum()
+        k_bf, best = _brute_min_card_row(p, tau)
+        assert mask[i].sum() == k_bf >= 1
+        assert math.isclose(p[mask[i]].sum(), best, rel_tol=1e-12)
+        # minimality: without its lowest kept block the row falls short of tau
+        lowest = np.flatnonzero(mask[i])[np.argmin(S[i][mask[i]])]
+        assert p[mask[i]].sum() - p[lowest] < tau
+        masses.append(best)
+    assert st["k"] == mask.sum()
+    assert math.isclose(st["mass"], float(np.mean(masses)), rel_tol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.37, 0.8])
+def test_local_rules_on_one_query_equal_global_ones(tau):
+    # with a single query row the head's pool is that row: local == global
+    S = np.random.default_rng(7).standard_normal((1, 11)) * 2.0
+    assert np.array_equal(O.threshold_local_select(S, tau)[0], O.threshold_select(S, tau)[0])
+    for k in (1, 4, 11):
+        assert np.array_equal(O.topk_local_select(S, k)[0], O.topk_global_select(S, k)[0])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_local_brute_force_and_counts(seed):
+    rng = np.random.default_rng(600 + seed)
+    S = rng.standard_normal((6, 5)) * (1 + seed)
+    for k in (1, 2, 4, 5, 9):
+        mask, st = O.topk_local_select(S, k)
+        kk = min(k, S.shape[1])
+        assert np.all(mask.sum(axis=1) == kk) and st["k"] == kk * S.shape[0]
+        for i in range(S.shape[0]):
+            assert math.isclose(S[i][mask[i]].sum(), _brute_best_k_subset(S[i], kk),
+                                rel_tol=1e-12)
+    mask, _ = O.topk_local_select(np.zeros((2, 4)), 2)        # ties: lower block first
+    assert mask.tolist() == [[True, True, False, False]] * 2
+
+
 # ---------------------------------------------------------------- attention
 
 def _sdpa(Qh, Kh, Vh, allow, scale):
