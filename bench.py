@@ -264,6 +264,7 @@ def run_ours(args, rank, world, local):
     # the paper's own block counts (8 / 48 / 72) on the same inputs, untimed by
     # the headline: density and ms per layer beside the main workload's
     second = paper_block_counts(V, w, (q, k, v, dout), stream)
+    variants = selection_variants(V, w, layers, q, density, stream)
 
     # per-call device times (ms, summed over layers, averaged over steps)
     call_ms = {c: 0.0 for c in CALLS}
@@ -341,6 +342,7 @@ def run_ours(args, rank, world, local):
                 "call_ms_per_step": {c: round(call_ms[c], 4) for c in CALLS},
                 "kernel_ms_per_layer": kern_layer,
                 "blocks_8_48_72": second,
+                "selection_variants": variants,
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
                                   for i, l in enumerate(LAYERS)},
                 "achieved": {c: [round(x[0], 3), x[1]] for c, x in achieved.items()},
@@ -354,6 +356,47 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def selection_variants(V, w, layers, q, density, stream, warm=1, reps=3):
+    """The ablation's selection rules on each layer's pool (partition already
+    done by the timed steps): device ms of one score + select call and the
+    selected density, with k set to the method's density at tau (top-k
+    global: its pair count; top-k local: that share of N_b per row)."""
+    import torch
+
+    from block_sparse_attention_layer_b200 import metrics
+    res = {}
+    for name in ("threshold_global", "topk_global", "threshold_local", "topk_local"):
+        ms_l, dens_l, gbs_l = [], [], []
+        for li, L in enumerate(layers):
+            sh, nb = L.shape, L.n_blocks
+            if name in ("threshold_global", "threshold_local"):
+                param = TAU
+            elif name == "topk_global":
+                param = max(1, round(density[li] * sh.s * nb))
+            else:
+                param = max(1, round(density[li] * nb))
+
+            def call():
+                V.score_select_variant(sh, q, L.blocks, name, param, 0.0, L.sel, L.stats, L.ws)
+
+            for _ in range(warm):
+                call()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(reps):
+                call()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / reps
+            st = L.head_stats()
+            ms_l.append(round(ms, 4))
+            dens_l.append(round(float(st["n_selected"].sum()) / (sh.s * nb * sh.n_heads), 5))
+            gbs_l.append(round(metrics.select_bytes(sh.s, sh.n_heads, nb) / (ms * 1e-3) / 1e9, 1))
+        res[name] = {"ms_per_layer": ms_l, "pair_density": dens_l, "select_GBps": gbs_l}
+    return res
 
 
 def paper_block_counts(V, w, tensors, stream, warm=2, reps=3):

@@ -10,12 +10,12 @@ from ._lib import (  # noqa: F401
     LayerShape, VmobaError, lib, mode_for_layer, num_blocks, workspace_size,
     bwd_workspace_size, partition, score_select, build_plan, attn_fwd, attn_bwd, get_status,
     decode_stats, default_scale, kernel_launches, trace_enable, trace_read, score_select_static,
-    HEAD_STATS_DTYPE,
+    score_select_variant, SELECT_VARIANTS, HEAD_STATS_DTYPE,
 )
 
 __all__ = [
     "LayerShape", "VmobaError", "lib", "mode_for_layer", "num_blocks", "workspace_size",
     "bwd_workspace_size", "partition", "score_select", "build_plan", "attn_fwd", "attn_bwd",
     "get_status", "decode_stats", "default_scale", "kernel_launches", "trace_enable", "trace_read",
-    "score_select_static", "HEAD_STATS_DTYPE",
+    "score_select_static", "score_select_variant", "SELECT_VARIANTS", "HEAD_STATS_DTYPE",
 ]

@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_bwd_workspace_size": (Z, [S]),
         "vmoba_partition": (I, [S, P, P, P, P, P, P]),
         "vmoba_score_select": (I, [S, P, P, F, F, P, P, P, Z, P]),
+        "vmoba_score_select_variant": (I, [S, P, P, I, ctypes.c_double, F, P, P, P, Z, P]),
         "vmoba_build_plan": (I, [S, P, P, Z, P]),
         "vmoba_attn_fwd": (I, [S, P, P, P, P, P, Z, F, P, P, P]),
         "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, Z, P]),
@@ -211,6 +212,28 @@ def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None)
         raise ValueError("stats buffer too small")
     _check("vmoba_score_select", lib().vmoba_score_select(
         ctypes.byref(shape.c()), _ptr(q), _ptr(blocks), float(tau), float(scale),
+        _ptr(sel_bits), _ptr(stats), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+# selection variants of the ablation (include/vmoba.h: vmoba_score_select_variant)
+SELECT_THRESHOLD_GLOBAL, SELECT_TOPK_GLOBAL, SELECT_THRESHOLD_LOCAL, SELECT_TOPK_LOCAL = 0, 1, 2, 3
+SELECT_VARIANTS = {"threshold_global": 0, "topk_global": 1, "threshold_local": 2, "topk_local": 3}
+
+
+def score_select_variant(shape, q, blocks, variant, param, scale, sel_bits, stats, ws,
+                         stream=None):
+    """Steps 2-3 with one of the ablation's selection rules: variant is a
+    SELECT_* code or a SELECT_VARIANTS name; param is tau or k."""
+    import torch
+    if isinstance(variant, str):
+        variant = SELECT_VARIANTS[variant]
+    _check_common(shape, q=q, sel_bits=sel_bits, ws=ws)
+    _expect(blocks, (shape.n_heads, num_blocks(shape), shape.head_dim), torch.float32, "blocks")
+    if stats.numel() * stats.element_size() < shape.n_heads * HEAD_STATS_DTYPE.itemsize:
+        raise ValueError("stats buffer too small")
+    _check("vmoba_score_select_variant", lib().vmoba_score_select_variant(
+        ctypes.byref(shape.c()), _ptr(q), _ptr(blocks), int(variant), float(param), float(scale),
         _ptr(sel_bits), _ptr(stats), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
 

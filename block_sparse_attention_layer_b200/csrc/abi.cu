@@ -139,6 +139,43 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
       launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
 }
 
+int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const float* blocks,
+                               int variant, double param, float scale, uint32_t* sel_bits,
+                               vmoba_head_stats* stats, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  Prob P;
+  int rc = make_prob(shape, &P);
+  if (rc != VMOBA_OK) return rc;
+  if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (std::isnan(param) || std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
+  const bool topk = variant == VMOBA_SELECT_TOPK_GLOBAL || variant == VMOBA_SELECT_TOPK_LOCAL;
+  if (variant < VMOBA_SELECT_THRESHOLD_GLOBAL || variant > VMOBA_SELECT_TOPK_LOCAL)
+    return VMOBA_ERR_ARG;
+  if (topk ? !(param >= 1.0 && param == std::floor(param) && param < 9.0e15) : !(param > 0.0))
+    return VMOBA_ERR_ARG;
+  WsLayout L;
+  if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  const double pool = (double)P.s * (double)P.Nb;
+  switch (variant) {
+    case VMOBA_SELECT_THRESHOLD_GLOBAL: {
+      const float tau_dev = param >= 1.0 ? 2.0f : (float)param;
+      return cuda_status(
+          launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
+    }
+    case VMOBA_SELECT_TOPK_GLOBAL:
+      // k at or above the pool keeps every pair (the walk can never reach pool + 1)
+      return cuda_status(launch_score_select(P, q, blocks, 0.0f, scale, sel_bits, stats, ws, L,
+                                             stream, 1, param >= pool ? pool + 1.0 : param));
+    default: {
+      cudaError_t e = launch_score_pool(P, q, blocks, scale, ws, L, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      const double p = topk ? param : (param >= 1.0 ? 2.0 : param);
+      return cuda_status(launch_select_local(P, topk ? 1 : 0, p, sel_bits, stats, ws, L, stream));
+    }
+  }
+}
+
 int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits, void* ws,
                      size_t ws_bytes, cudaStream_t stream) {
   Prob P;

@@ -151,9 +151,20 @@ void count_launches(int n);
 // ---- launch wrappers (one per kernel family; defined in the .cu files) ----
 cudaError_t launch_partition(const Prob& P, const void* k, const void* v, void* kp, void* vp,
                              float* blocks, cudaStream_t st);
+// by_count = 0: the method's mass threshold tau; by_count = 1: the kcount
+// highest pairs of each head's pool (top-k global), same ranking and ties.
 cudaError_t launch_score_select(const Prob& P, const void* q, const float* blocks, float tau,
                                 float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
-                                const WsLayout& L, cudaStream_t st);
+                                const WsLayout& L, cudaStream_t st, int by_count = 0,
+                                double kcount = 0.0);
+// The score pool S = scale q b^T of every head into the workspace.
+cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks, float scale,
+                              void* ws, const WsLayout& L, cudaStream_t st);
+// Per-query-row selection (threshold local / top-k local); scores in the
+// workspace pool, per-row scratch in the forward-output copy.
+cudaError_t launch_select_local(const Prob& P, int topk, double param, uint32_t* sel,
+                                vmoba_head_stats* stats, void* ws, const WsLayout& L,
+                                cudaStream_t st);
 cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLayout& L,
                         cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(const Prob& P, const void* q, const void* kp, const void* vp,

@@ -16,6 +16,12 @@
 //
 // Kernels, in stream order: init -> score -> {hist, scan} x 3 ->
 // {tie_hist, tie_scan} x 3 -> emit (bitmap) -> stats.
+//
+// The ablation's "topk + global" variant (VMoBA notes, ablation table) runs
+// the same passes with the digit walk counting pairs instead of mass: the
+// cut is then the k-th pair of the same ranking; the masses still ride
+// along for the stats (a last-pass bucket holds one score value, so its
+// share of the mass is exact).
 #include "common.cuh"
 
 namespace vmoba {
@@ -159,7 +165,7 @@ k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t*
 template <int PASS>
 __global__ void __launch_bounds__(32)
 k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __restrict__ hm,
-       float tau) {
+       float tau, int by_count, double kcount) {
   const int h = blockIdx.x, lane = threadIdx.x;
   SelState& S = st[h];
   if (S.state != kSel_Search) return;
@@ -183,9 +189,13 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
     above = 0.0;
     cabove = 0;
-    target = (double)tau * tot;
+    target = by_count ? kcount : (double)tau * tot;
     if (lane == 0) { S.Z = tot; S.target = target; }
   }
+  // the walk stops where the running mass (or pair count) reaches the target
+  auto reach = [&](double m, unsigned long long cnt) {
+    return by_count ? (double)cnt >= target : m >= target;
+  };
   double incl = lm;
   unsigned long long cincl = lc;
 #pragma unroll
@@ -194,7 +204,7 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     unsigned long long yc = __shfl_up_sync(0xffffffffu, cincl, o);
     if (lane >= o) { incl += y; cincl += yc; }
   }
-  const unsigned ball = __ballot_sync(0xffffffffu, above + incl >= target);
+  const unsigned ball = __ballot_sync(0xffffffffu, reach(above + incl, cabove + cincl));
   const unsigned nz = __ballot_sync(0xffffffffu, lc > 0);
   if (nz == 0u || (ball == 0u && PASS == 0)) {
     // tau reaches the whole pool: every pair is selected
@@ -223,7 +233,7 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     for (int k = 0; k < per; ++k) {
       int d = nb - 1 - lane * per - k;
       if (c[d]) {
-        if (acc + mm[d] >= target) { chosen = d; break; }
+        if (reach(acc + mm[d], cacc + c[d])) { chosen = d; break; }
         last = d;
         acc_last = acc;
         cacc_last = cacc;
@@ -244,9 +254,9 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     S.count_above = cacc;
     if (PASS == 2) {
       const uint32_t nt = c[chosen];
-      const double e = mm[chosen] / (double)nt;
-      const double need = target - acc;
-      const double rr = (need > 0.0 && e > 0.0) ? ceil(need / e) : 1.0;
+      const double e = mm[chosen] / (double)nt;   // one score value: equal shares
+      const double need = by_count ? target - (double)cacc : target - acc;
+      const double rr = by_count ? need : ((need > 0.0 && e > 0.0) ? ceil(need / e) : 1.0);
       const uint32_t r = (rr < 1.0) ? 1u : (rr >= (double)nt ? nt : (uint32_t)rr);
       S.cut_key = pre;
       S.tie_count = nt;
@@ -399,9 +409,31 @@ cudaError_t launch_score(const Prob& P, const void* q, const float* B, float sca
 
 }  // namespace
 
+cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks, float scale,
+                              void* ws, const WsLayout& L, cudaStream_t stream) {
+  SelState* st = ws_ptr<SelState>(ws, L.sel_state);
+  {
+    VMOBA_TRACE("k_init", stream);
+    k_init<<<64, 256, 0, stream>>>(st, ws_ptr<uint32_t>(ws, L.hist_count),
+                                   ws_ptr<double>(ws, L.hist_mass), P.n_h);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  float* S = ws_ptr<float>(ws, L.scores);
+  if (P.dtype == VMOBA_BF16)
+    e = (P.d == 128) ? launch_score<__nv_bfloat16, 128>(P, q, blocks, scale, S, st, stream)
+                     : launch_score<__nv_bfloat16, 64>(P, q, blocks, scale, S, st, stream);
+  else
+    e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
+                     : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
+  count_launches(2);
+  return e;
+}
+
 cudaError_t launch_score_select(const Prob& P, const void* q, const float* blocks, float tau,
                                 float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
-                                const WsLayout& L, cudaStream_t stream) {
+                                const WsLayout& L, cudaStream_t stream, int by_count,
+                                double kcount) {
   SelState* st = ws_ptr<SelState>(ws, L.sel_state);
   uint32_t* hc = ws_ptr<uint32_t>(ws, L.hist_count);
   double* hm = ws_ptr<double>(ws, L.hist_mass);
@@ -429,7 +461,7 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   }
   {
     VMOBA_TRACE("k_scan", stream);
-    k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+    k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
   }
   {
     VMOBA_TRACE("k_hist", stream);
@@ -437,7 +469,7 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   }
   {
     VMOBA_TRACE("k_scan", stream);
-    k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+    k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
   }
   {
     VMOBA_TRACE("k_hist", stream);
@@ -445,7 +477,7 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   }
   {
     VMOBA_TRACE("k_scan", stream);
-    k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau);
+    k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
   }
   {
     VMOBA_TRACE("k_tie_hist", stream);

@@ -46,6 +46,16 @@ class VMoBALayer:
         _lib.score_select(sh, q, self.blocks, tau, scale, self.sel, self.stats, self.ws)
         _lib.build_plan(sh, self.sel, self.ws)
 
+    def select_variant(self, q, k, v, variant, param, scale=0.0):
+        """As select, with one of the ablation's selection rules (see
+        _lib.score_select_variant): "threshold_global" (the method),
+        "topk_global", "threshold_local", "topk_local"."""
+        sh = self.shape
+        _lib.partition(sh, k, v, self.k_perm, self.v_perm, self.blocks)
+        _lib.score_select_variant(sh, q, self.blocks, variant, param, scale, self.sel,
+                                  self.stats, self.ws)
+        _lib.build_plan(sh, self.sel, self.ws)
+
     def use_selection(self, sel_bits):
         """Adopt a caller-built bitmap (e.g. a reference selection) and plan for it."""
         self.sel.copy_(sel_bits)

@@ -126,6 +126,40 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
                        vmoba_head_stats* stats, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* The ablation's selection variants (notes, ablation table; digest App. A),
+ * the research alternatives to step 3 -- no counterpart is needed on the
+ * method's own path.  variant:
+ *   VMOBA_SELECT_THRESHOLD_GLOBAL  the method itself (= vmoba_score_select),
+ *                                  param = tau;
+ *   VMOBA_SELECT_TOPK_GLOBAL       "topk + global": the param = k highest
+ *                                  pairs of each head's pool, ranked (score
+ *                                  desc, index asc) like the method;
+ *   VMOBA_SELECT_THRESHOLD_LOCAL   "threshold + local": per query row, the
+ *                                  shortest prefix of its own blocks (score
+ *                                  desc, block asc) whose mass under the
+ *                                  row's own softmax reaches param = tau;
+ *   VMOBA_SELECT_TOPK_LOCAL        "topk + local" (about MoBA's selection;
+ *                                  the training-free runs use it on 3D
+ *                                  blocks): per query row its first
+ *                                  min(param = k, N_b) blocks.
+ * tau must be > 0 (>= 1 keeps everything); k a whole number >= 1 (at or
+ * above the pool / N_b keeps everything); anything else, or an unknown
+ * variant, -> VMOBA_ERR_ARG.  Same buffers and outputs as
+ * vmoba_score_select.  stats of the local variants: n_selected = pairs,
+ * mass = mean kept mass per row under the row softmax, cut_score = NaN
+ * (each row has its own cut); the per-row bookkeeping uses workspace that
+ * vmoba_attn_fwd overwrites later. */
+enum {
+  VMOBA_SELECT_THRESHOLD_GLOBAL = 0,
+  VMOBA_SELECT_TOPK_GLOBAL = 1,
+  VMOBA_SELECT_THRESHOLD_LOCAL = 2,
+  VMOBA_SELECT_TOPK_LOCAL = 3
+};
+int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const float* blocks,
+                               int variant, double param, float scale, uint32_t* sel_bits,
+                               vmoba_head_stats* stats, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+
 /* Step 4a: from any selection bitmap (vmoba_score_select's, or one the
  * caller built), build the tile work lists the attention kernels walk:
  * per 128-query tile (queries in partition order) the key tiles its rows
