@@ -100,6 +100,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, Z, P]),
         "vmoba_get_status": (I, [P, ctypes.POINTER(I), P]),
         "vmoba_status_string": (ctypes.c_char_p, [I]),
+        "vmoba_last_cuda_error": (ctypes.c_char_p, []),
         "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
         "vmoba_score_select_static": (I, [S, P, P, F, F, P, P, P]),
         "vmoba_trace_enable": (I, [I]),
@@ -115,7 +116,10 @@ def lib() -> ctypes.CDLL:
 
 def _check(fn: str, rc: int) -> None:
     if rc != 0:
-        raise VmobaError(fn, rc)
+        err = VmobaError(fn, rc)
+        if rc == -5:        # VMOBA_ERR_CUDA: name the CUDA error behind it
+            err.args = (f"{err.args[0]} ({lib().vmoba_last_cuda_error().decode()})",)
+        raise err
 
 
 def _stream(stream):

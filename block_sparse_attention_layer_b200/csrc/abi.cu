@@ -54,7 +54,20 @@ int check_ws(const Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
   return VMOBA_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? VMOBA_OK : VMOBA_ERR_CUDA; }
+// The CUDA error behind the calling thread's last VMOBA_ERR_CUDA.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return VMOBA_OK;
+  g_last_cuda_error = e;
+  return VMOBA_ERR_CUDA;
+}
+
+// The runtime's last-error slot is per host thread and the launchers read it
+// after their launches; drop whatever another caller on this thread left
+// there so it is not reported as ours (errors that break the context
+// persist and still surface on our own launches).
+void drop_stale_error() { (void)cudaGetLastError(); }
 
 ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
   ItemBufs b{};
@@ -118,6 +131,7 @@ int vmoba_partition(const vmoba_shape* shape, const void* k, const void* v, void
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_perm) || !aligned16(v_perm) ||
       !aligned16(blocks))
     return VMOBA_ERR_ARG;
+  drop_stale_error();
   return cuda_status(launch_partition(P, k, v, k_perm, v_perm, blocks, stream));
 }
 
@@ -135,6 +149,7 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   // tau at or above the whole pool keeps every pair; 2 can never be reached
   const float tau_dev = tau >= 1.0f ? 2.0f : tau;
+  drop_stale_error();
   return cuda_status(
       launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
 }
@@ -157,6 +172,7 @@ int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const fl
   if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   const double pool = (double)P.s * (double)P.Nb;
+  drop_stale_error();
   switch (variant) {
     case VMOBA_SELECT_THRESHOLD_GLOBAL: {
       const float tau_dev = param >= 1.0 ? 2.0f : (float)param;
@@ -184,6 +200,7 @@ int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits, void* w
   if (!sel_bits) return VMOBA_ERR_ARG;
   WsLayout L;
   if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
+  drop_stale_error();
   return cuda_status(launch_plan(P, sel_bits, ws, L, stream));
 }
 
@@ -202,6 +219,7 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   // bf16 with head_dim 128 runs on the tensor cores; fp32 I/O (whose 1e-4
   // bar rules out TF32) and head_dim 64 run on the CUDA cores
+  drop_stale_error();
   if (uses_blk_path(P))
     return cuda_status(launch_attn_fwd_blk(
         P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
@@ -229,6 +247,7 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   if (!ws_bwd || ws_bwd_bytes < vmoba_bwd_workspace_size(shape) || !aligned16(ws_bwd))
     return VMOBA_ERR_WORKSPACE;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
+  drop_stale_error();
   if (uses_blk_path(P))
     return cuda_status(launch_attn_bwd_blk(
         P, q, k_perm, v_perm, sel_bits, pairs_view(P, ws_ptr<char>(ws, L.pairs)),
@@ -252,6 +271,8 @@ int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream) {
   *device_status = v;
   return VMOBA_OK;
 }
+
+const char* vmoba_last_cuda_error(void) { return cudaGetErrorName(g_last_cuda_error); }
 
 const char* vmoba_status_string(int status) {
   switch (status) {
@@ -346,6 +367,7 @@ int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const flo
   const float tau_dev = tau >= 1.0f ? 2.0f : tau;
   // the first kernel of the selection clears the histograms and the search
   // state; the score pool is fully overwritten before it is read
+  drop_stale_error();
   return cuda_status(
       launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, scratch, L, stream));
 }

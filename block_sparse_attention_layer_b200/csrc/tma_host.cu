@@ -17,6 +17,9 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (cols * 2) % 16 != 0) return false;
+  // a driver call: make sure this host thread has the device's context bound
+  // (a thread whose first CUDA work is this call would have none)
+  if (cudaFree(nullptr) != cudaSuccess) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
   const cuuint32_t box[2] = {64, box_rows};

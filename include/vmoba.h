@@ -248,6 +248,12 @@ int vmoba_trace_read(vmoba_trace_entry* out, int max_entries);
 /* Static text of a vmoba_status code. */
 const char* vmoba_status_string(int status);
 
+/* Name of the CUDA error (e.g. "cudaErrorInvalidValue") behind the calling
+ * host thread's most recent VMOBA_ERR_CUDA, or "cudaSuccess" if none.  Each
+ * compute call first drops any error another caller left in the thread's
+ * runtime error slot, so a returned VMOBA_ERR_CUDA is the library's own. */
+const char* vmoba_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

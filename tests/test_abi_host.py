@@ -143,3 +143,9 @@ def test_binding_rejects_wrong_tensors_before_the_call():
     k = torch.zeros((sh.s, 2, 64), dtype=torch.float32)
     with pytest.raises(ValueError):
         _lib.partition(sh, k, k, k, k, k)   # wrong shapes for k_perm / blocks
+
+
+def test_full_attention_steps_of_the_training_strategy():
+    from block_sparse_attention_layer_b200.attention import full_attention_steps
+    assert full_attention_steps(50) == 13 and full_attention_steps(40) == 10
+    assert full_attention_steps(1) == 1 and full_attention_steps(8, 0.0) == 0
