@@ -469,30 +469,67 @@ def kernel_traffic(name, w):
 
 def run_e2e(args, layers, host, flops_step, world):
     """Same metric through the public API with host buffers: per layer, H2D of
-    q, k, v, dO from pinned memory, the ABI calls, D2H of O, dQ, dK, dV."""
+    q, k, v, dO from pinned memory, the ABI calls, D2H of O, dQ, dK, dV.
+
+    The copies run on two copy streams (host-to-device, device-to-host) so
+    that layer l+1's inputs arrive and layer l-1's outputs leave while layer l
+    computes: two device input sets alternate between layers, each layer
+    object's outputs go to their own pinned host buffers, and events order
+    every reuse of a buffer after its last reader."""
     import torch
     hq, hk, hv, hdo = host
-    stream = torch.cuda.current_stream()
-    outs = [torch.empty_like(hq).pin_memory() for _ in range(4)]
-    dq_in, dk_in, dv_in, ddo_in = (torch.empty_like(x, device="cuda") for x in host)
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = [[torch.empty_like(hq).pin_memory() for _ in range(4)] for _ in layers]
+    sets = [[torch.empty_like(x, device="cuda") for x in host] for _ in range(2)]
+    ev = lambda: torch.cuda.Event()  # noqa: E731
 
-    def step():
-        for L in layers:
-            for dst, src in ((dq_in, hq), (dk_in, hk), (dv_in, hv), (ddo_in, hdo)):
-                dst.copy_(src, non_blocking=True)
-            L.step(dq_in, dk_in, dv_in, TAU, dout=ddo_in)
-            for dst, src in zip(outs, (L.out, L.dq, L.dk, L.dv)):
-                dst.copy_(src, non_blocking=True)
+    def run(n_steps):
+        seq = [L for _ in range(n_steps) for L in layers]
+        done = [None] * len(seq)      # compute of use u finished
+        out_done = [None] * len(seq)  # outputs of use u copied to the host
+        arrived = [None] * len(seq)
+        start = ev()
+        start.record(comp)
 
-    for _ in range(max(1, min(args.warmup, 2))):
-        step()
+        def load(u):
+            h2d.wait_event(start)
+            if u >= 2:
+                h2d.wait_event(done[u - 2])   # set u % 2 was last read by use u - 2
+            with torch.cuda.stream(h2d):
+                for dst, src in zip(sets[u % 2], (hq, hk, hv, hdo)):
+                    dst.copy_(src, non_blocking=True)
+            arrived[u] = ev()
+            arrived[u].record(h2d)
+
+        load(0)
+        for u, L in enumerate(seq):
+            if u + 1 < len(seq):
+                load(u + 1)
+            comp.wait_event(arrived[u])
+            if u >= len(layers):
+                comp.wait_event(out_done[u - len(layers)])   # L's outputs left the GPU
+            q, k, v, do = sets[u % 2]
+            L.step(q, k, v, TAU, dout=do)
+            done[u] = ev()
+            done[u].record(comp)
+            d2h.wait_event(done[u])
+            with torch.cuda.stream(d2h):
+                for dst, src in zip(outs[u % len(layers)], (L.out, L.dq, L.dk, L.dv)):
+                    dst.copy_(src, non_blocking=True)
+            out_done[u] = ev()
+            out_done[u].record(d2h)
+        comp.wait_event(out_done[-1])
+        return start
+
+    run(max(1, min(args.warmup, 2)))
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     K = max(1, args.steps)
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    run(K)
+    b.record(comp)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     ms, _ = reduce_over_ranks(ms, 0.0, "cuda")
@@ -500,7 +537,8 @@ def run_e2e(args, layers, host, flops_step, world):
     return {"value": round(flops_step * K * world / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
             "h2d_bytes_per_step": 4 * nbytes * len(layers),
             "d2h_bytes_per_step": 4 * nbytes * len(layers),
-            "ms_per_step": round(ms / K, 3)}
+            "ms_per_step": round(ms / K, 3),
+            "copies": "H2D and D2H on their own streams, overlapped with the layers"}
 
 
 # ------------------------------------------------------------- CPU oracle
