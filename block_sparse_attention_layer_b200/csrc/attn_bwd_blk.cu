@@ -159,6 +159,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
           tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
+        if (ok && n + G < n_items) {
+          // the next item's Q / dO into L2 behind this item's loads (one buffer in smem)
+          tma_prefetch_l2_2d(&tm_q, 0, (n + G) * kTile);
+          tma_prefetch_l2_2d(&tm_q, 64, (n + G) * kTile);
+          tma_prefetch_l2_2d(&tm_o, 0, (n + G) * kTile);
+          tma_prefetch_l2_2d(&tm_o, 64, (n + G) * kTile);
+        }
       }
     }
   } else if (warp == 1) {
@@ -246,17 +253,25 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const uint64_t sl2x2 = f32x2(sl2, sl2);
     int J = 0, it_local = 0;
     bool ok = true;
-    for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-      const WorkItem it = decode_item(pv, P, h, n);
-      const bool valid = r < it.count;
-      float nl2 = -INFINITY, Di = 0.f;
-      uint32_t slot = 0xFFFFFFFFu;
-      if (valid) {
-        slot = __ldg(col_slot + it.first + r);
-        nl2 = __ldg(l2g + (size_t)n * kTile + r);
-        Di = __ldg(dg + (size_t)n * kTile + r);
+    // the row's slot, -LSE log2(e) and D of item nn; fetched one item ahead,
+    // before the epilogue, so the decode and the loads are off the critical path
+    auto fetch = [&](int nn, uint32_t& sl, float& l2, float& d) {
+      const WorkItem w = decode_item(pv, P, h, nn);
+      sl = 0xFFFFFFFFu;
+      l2 = -INFINITY;
+      d = 0.f;
+      if (r < w.count) {
+        sl = __ldg(col_slot + w.first + r);
+        l2 = __ldg(l2g + (size_t)nn * kTile + r);
+        d = __ldg(dg + (size_t)nn * kTile + r);
       }
-      const uint64_t nl2x2 = f32x2(nl2, nl2), Dx2 = f32x2(Di, Di);
+    };
+    uint32_t nx_slot = 0xFFFFFFFFu;
+    float nx_l2 = -INFINITY, nx_d = 0.f;
+    if (blockIdx.x < n_items) fetch(blockIdx.x, nx_slot, nx_l2, nx_d);
+    for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
+      const uint32_t slot = nx_slot;
+      const uint64_t nl2x2 = f32x2(nx_l2, nx_l2), Dx2 = f32x2(nx_d, nx_d);
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, status, abort));
@@ -319,6 +334,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         if (lane == 0) mbar_arrive(&bars->ds_full);
       }
       if (!ok) break;
+      if (n + G < n_items) fetch(n + G, nx_slot, nx_l2, nx_d);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, status, abort));
       if (!ok) break;
       tc_fence_after();

@@ -194,6 +194,16 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
           tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
+        if (ok && p + G < n_pairs) {
+          // the next pair's Q tiles into L2 behind this pair's loads
+          WorkItem b1;
+          int n1;
+          decode_item_pair(pv, P, h, p + G, &b1, &n1);
+          for (int t = 0; t < (b1.count > 0 ? 2 : 1); ++t) {
+            tma_prefetch_l2_2d(&tm_q, 0, (n1 + t) * kTile);
+            tma_prefetch_l2_2d(&tm_q, 64, (n1 + t) * kTile);
+          }
+        }
       }
     }
   } else if (warp == 1) {
@@ -284,14 +294,26 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     const uint32_t* col_slot = pv.col_slot + (size_t)h * P.s * P.Nb;
     int Js = 0, It = 0;
     bool ok = true;
+    // this tile of pair pp and the row's slot; fetched one pair ahead, before
+    // the epilogue, so the decode and the slot load are off the critical path
+    auto fetch = [&](int pp, WorkItem& m, uint32_t& sl) {
+      WorkItem bb;
+      int nn;
+      const WorkItem aa = decode_item_pair(pv, P, h, pp, &bb, &nn);
+      m = t == 0 ? aa : bb;
+      sl = r < m.count ? __ldg(col_slot + m.first + r) : 0xFFFFFFFFu;
+    };
+    WorkItem nx_me;
+    uint32_t nx_slot = 0xFFFFFFFFu;
+    if (blockIdx.x < n_pairs) fetch(blockIdx.x, nx_me, nx_slot);
     for (int p = blockIdx.x; p < n_pairs && ok; p += G) {
-      WorkItem b;
-      int n0;
-      const WorkItem a = decode_item_pair(pv, P, h, p, &b, &n0);
-      const WorkItem me = t == 0 ? a : b;
-      if (me.count == 0) continue;                 // no tile B in this pair
+      const WorkItem me = nx_me;
+      const uint32_t slot = nx_slot;
+      if (me.count == 0) {                         // no tile B in this pair
+        if (p + G < n_pairs) fetch(p + G, nx_me, nx_slot);
+        continue;
+      }
       const bool valid = r < me.count;
-      const uint32_t slot = valid ? __ldg(col_slot + me.first + r) : 0xFFFFFFFFu;
       float m_run = -INFINITY, l_run = 0.f;
       for (int c = 0; c < nch; ++c, ++Js) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], Js & 1, status, abort));
@@ -305,6 +327,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
       if (!ok) break;
+      if (p + G < n_pairs) fetch(p + G, nx_me, nx_slot);
       // epilogue: partial state of (query, block j) into the pair's slot
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[t], It & 1, status, abort));
       ++It;
