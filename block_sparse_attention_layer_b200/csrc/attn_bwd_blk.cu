@@ -134,10 +134,10 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_o);
-      int J = 0, it_local = 0;
+      int J = 0, it_local = 0, hint = 0;
       bool ok = true;
       for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-        const WorkItem it = decode_item(pv, P, h, n);
+        const WorkItem it = decode_item<false>(pv, P, h, n, hint);
         if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, status, abort);
         if (!ok) break;
         mbar_expect_tx(&bars->qd_full, 2 * kTileB);
@@ -255,8 +255,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     bool ok = true;
     // the row's slot, -LSE log2(e) and D of item nn; fetched one item ahead,
     // before the epilogue, so the decode and the loads are off the critical path
+    int hint = 0;
     auto fetch = [&](int nn, uint32_t& sl, float& l2, float& d) {
-      const WorkItem w = decode_item(pv, P, h, nn);
+      const WorkItem w = decode_item<true>(pv, P, h, nn, hint);
       sl = 0xFFFFFFFFu;
       l2 = -INFINITY;
       d = 0.f;

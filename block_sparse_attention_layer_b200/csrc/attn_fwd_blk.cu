@@ -165,12 +165,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_q);
-      int J = 0, it_local = 0;
+      int J = 0, it_local = 0, hint = 0, hint_pf = 0;
       bool ok = true;
       for (int p = blockIdx.x; p < n_pairs && ok; p += G, ++it_local) {
         WorkItem b;
         int n0;
-        const WorkItem a = decode_item_pair(pv, P, h, p, &b, &n0);
+        const WorkItem a = decode_item_pair<false>(pv, P, h, p, &b, &n0, hint);
         if (it_local >= 1) ok = mbar_wait(&bars->q_empty, (it_local - 1) & 1, status, abort);
         if (!ok) break;
         mbar_expect_tx(&bars->q_full, b.count > 0 ? 2 * kTileB : kTileB);
@@ -198,7 +198,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           // the next pair's Q tiles into L2 behind this pair's loads
           WorkItem b1;
           int n1;
-          decode_item_pair(pv, P, h, p + G, &b1, &n1);
+          decode_item_pair<false>(pv, P, h, p + G, &b1, &n1, hint_pf);
           for (int t = 0; t < (b1.count > 0 ? 2 : 1); ++t) {
             tma_prefetch_l2_2d(&tm_q, 0, (n1 + t) * kTile);
             tma_prefetch_l2_2d(&tm_q, 64, (n1 + t) * kTile);
@@ -234,10 +234,11 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                  desc_sw128(vb + kk * 2048, kHalf, 1024), idPV, (c > 0 || kk > 0) ? 1u : 0u);
         if (c == nch - 1) mma_commit(&bars->o_final[t]);
       };
+      int hint = 0;
       for (int p = blockIdx.x, it_local = 0; p < n_pairs && ok; p += G, ++it_local) {
         WorkItem b;
         int n0;
-        decode_item_pair(pv, P, h, p, &b, &n0);
+        decode_item_pair<false>(pv, P, h, p, &b, &n0, hint);
         const int nt = b.count > 0 ? 2 : 1;
         if (!mbar_wait(&bars->q_full, it_local & 1, status, abort)) { ok = false; break; }
         {
@@ -296,10 +297,11 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     bool ok = true;
     // this tile of pair pp and the row's slot; fetched one pair ahead, before
     // the epilogue, so the decode and the slot load are off the critical path
+    int hint = 0;
     auto fetch = [&](int pp, WorkItem& m, uint32_t& sl) {
       WorkItem bb;
       int nn;
-      const WorkItem aa = decode_item_pair(pv, P, h, pp, &bb, &nn);
+      const WorkItem aa = decode_item_pair<true>(pv, P, h, pp, &bb, &nn, hint);
       m = t == 0 ? aa : bb;
       sl = r < m.count ? __ldg(col_slot + m.first + r) : 0xFFFFFFFFu;
     };

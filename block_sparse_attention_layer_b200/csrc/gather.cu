@@ -23,8 +23,9 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
   const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
+  int hint = 0;
   for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < n_items; n += warps) {
-    const WorkItem it = decode_item(pv, P, h, n);
+    const WorkItem it = decode_item<true>(pv, P, h, n, hint);
     const int count = it.count;
     const uint32_t* rows = col_rows + it.first;
     const size_t base = (size_t)n * kTile;

@@ -26,19 +26,46 @@ struct WorkItem {
   uint32_t first;         // index of the tile's first entry in col_rows / col_slot
 };
 
-// Work item n of head h (n < head_totals[4h+1]).
-__device__ __forceinline__ WorkItem decode_item(const PairsView& pv, const Prob& P, int h, int n) {
+// Block j with off[j] <= n < off[j+1], for a non-decreasing offset array
+// (off[N_b] > n), scanned forward from `hint` (off[hint] <= n); `hint`
+// becomes j.  Every role of a CTA visits its work in increasing order, so the
+// scan passes only the blocks finished since its last item.  kWarp: the
+// whole warp takes 32 entries per coalesced step (n warp-uniform, all lanes
+// present); otherwise one thread steps one entry at a time.
+template <bool kWarp>
+__device__ __forceinline__ int find_block(const uint32_t* off, int Nb, uint32_t n, int& hint) {
+  int j = hint;
+  if (kWarp) {
+    const int lane = threadIdx.x & 31;
+    for (;;) {
+      const int jj = j + 1 + lane;
+      // entries <= n form a prefix of the window (off is non-decreasing)
+      const uint32_t m = __ballot_sync(0xffffffffu, jj <= Nb && __ldg(off + jj) <= n);
+      if (m != 0xffffffffu) {
+        j += __popc(m);
+        break;
+      }
+      j += 32;
+    }
+  } else {
+    while (__ldg(off + j + 1) <= n) ++j;
+  }
+  hint = j;
+  return j;
+}
+
+// Work item n of head h (n < head_totals[4h+1]); `hint` as in find_block
+// (0 before a role's first item).
+template <bool kWarp>
+__device__ __forceinline__ WorkItem decode_item(const PairsView& pv, const Prob& P, int h, int n,
+                                                int& hint) {
   const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
   const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
-  int lo = 0, hi = P.Nb;   // invariant: item_off[lo] <= n < item_off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(item_off + mid) <= (uint32_t)n) lo = mid; else hi = mid;
-  }
+  const int j = find_block<kWarp>(item_off, P.Nb, (uint32_t)n, hint);
   WorkItem it;
-  it.j = lo;
-  const int g = n - (int)__ldg(item_off + lo);
-  const uint32_t c0 = __ldg(col_off + lo), c1 = __ldg(col_off + lo + 1);
+  it.j = j;
+  const int g = n - (int)__ldg(item_off + j);
+  const uint32_t c0 = __ldg(col_off + j), c1 = __ldg(col_off + j + 1);
   it.first = c0 + (uint32_t)g * kTile;
   it.count = min(kTile, (int)(c1 - it.first));
   return it;
@@ -46,26 +73,25 @@ __device__ __forceinline__ WorkItem decode_item(const PairsView& pv, const Prob&
 
 // Item pair p of head h: tiles 2q and 2q+1 of one block's list (the second
 // may be absent).  Returns the first tile; *second gets the other (count 0
-// when absent) and *n0 the first tile's work-item index.
+// when absent) and *n0 the first tile's work-item index.  `hint` as in
+// find_block, over the pair offsets.
+template <bool kWarp>
 __device__ __forceinline__ WorkItem decode_item_pair(const PairsView& pv, const Prob& P, int h,
-                                                     int p, WorkItem* second, int* n0) {
+                                                     int p, WorkItem* second, int* n0,
+                                                     int& hint) {
   const uint32_t* pitem_off = pv.pitem_off + (size_t)h * (P.Nb + 1);
   const uint32_t* item_off = pv.item_off + (size_t)h * (P.Nb + 1);
   const uint32_t* col_off = pv.col_off + (size_t)h * (P.Nb + 1);
-  int lo = 0, hi = P.Nb;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(pitem_off + mid) <= (uint32_t)p) lo = mid; else hi = mid;
-  }
-  const int q = p - (int)__ldg(pitem_off + lo);
-  const uint32_t c0 = __ldg(col_off + lo), c1 = __ldg(col_off + lo + 1);
+  const int j = find_block<kWarp>(pitem_off, P.Nb, (uint32_t)p, hint);
+  const int q = p - (int)__ldg(pitem_off + j);
+  const uint32_t c0 = __ldg(col_off + j), c1 = __ldg(col_off + j + 1);
   WorkItem a, b;
-  a.j = b.j = lo;
+  a.j = b.j = j;
   a.first = c0 + (uint32_t)q * 2 * kTile;
   b.first = a.first + kTile;
   a.count = min(kTile, (int)(c1 - a.first));
   b.count = c1 > b.first ? min(kTile, (int)(c1 - b.first)) : 0;
-  *n0 = (int)__ldg(item_off + lo) + 2 * q;
+  *n0 = (int)__ldg(item_off + j) + 2 * q;
   *second = b;
   return a;
 }
