@@ -7,8 +7,10 @@
 // Two passes over the pair lists (pairs.cu), no atomics, deterministic:
 //  * dQ pass: a work item is (block j, 128 queries of block j's list); it
 //    walks the block's keys in chunks of 128: S = Q K^T, dP = dO V^T, then
-//    dS in TMEM and dQ += dS K.  The per-pair partial dQ goes to the pair's
-//    slot; a merge sums each query's partials (blocks in ascending order).
+//    dS in TMEM and dQ += dS K.  The per-pair partial dQ goes to the item's
+//    rows (128 n + r) by asynchronous TMA stores of each warp's staging
+//    tile; a merge sums each query's partials, found through the pair lists'
+//    slot -> item row map, in ascending block order.
 //  * dK/dV pass: a work item is (block j, 128-key tile of block j); it walks
 //    all query tiles of block j's list: S^T = K Q^T, dP^T = V dO^T,
 //    P^T and dS^T in TMEM, dV += P^T dO, dK += dS^T Q; dK, dV of the tile's
@@ -82,8 +84,8 @@ static_assert(kDqSmem <= 232448, "shared memory per CTA");
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-             Prob P, int h, PairsView pv, const float* __restrict__ dg,
-             const float* __restrict__ l2g, float sl2, float* __restrict__ part_dq,
+             const __grid_constant__ CUtensorMap tm_pd, Prob P, int h, PairsView pv,
+             const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
              int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -97,7 +99,6 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t* col_slot = pv.col_slot + (size_t)h * P.s * P.Nb;
   const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int nch = (P.L + kTile - 1) / kTile;
   const int kc_last = P.L - (nch - 1) * kTile;        // keys in the last chunk
@@ -253,25 +254,16 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const uint64_t sl2x2 = f32x2(sl2, sl2);
     int J = 0, it_local = 0;
     bool ok = true;
-    // the row's slot, -LSE log2(e) and D of item nn; fetched one item ahead,
-    // before the epilogue, so the decode and the loads are off the critical path
-    int hint = 0;
-    auto fetch = [&](int nn, uint32_t& sl, float& l2, float& d) {
-      const WorkItem w = decode_item<true>(pv, P, h, nn, hint);
-      sl = 0xFFFFFFFFu;
-      l2 = -INFINITY;
-      d = 0.f;
-      if (r < w.count) {
-        sl = __ldg(col_slot + w.first + r);
-        l2 = __ldg(l2g + (size_t)nn * kTile + r);
-        d = __ldg(dg + (size_t)nn * kTile + r);
-      }
+    // -LSE log2(e) and D of the row in item nn (the item-ordered copies hold
+    // -inf and 0 past the tile's queries); loaded one item ahead, before the
+    // epilogue, so their latency is off the critical path
+    auto fetch = [&](int nn, float& l2, float& d) {
+      l2 = __ldg(l2g + (size_t)nn * kTile + r);
+      d = __ldg(dg + (size_t)nn * kTile + r);
     };
-    uint32_t nx_slot = 0xFFFFFFFFu;
     float nx_l2 = -INFINITY, nx_d = 0.f;
-    if (blockIdx.x < n_items) fetch(blockIdx.x, nx_slot, nx_l2, nx_d);
+    if (blockIdx.x < n_items) fetch(blockIdx.x, nx_l2, nx_d);
     for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
-      const uint32_t slot = nx_slot;
       const uint64_t nl2x2 = f32x2(nx_l2, nx_l2), Dx2 = f32x2(nx_d, nx_d);
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
@@ -335,7 +327,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         if (lane == 0) mbar_arrive(&bars->ds_full);
       }
       if (!ok) break;
-      if (n + G < n_items) fetch(n + G, nx_slot, nx_l2, nx_d);
+      if (n + G < n_items) fetch(n + G, nx_l2, nx_d);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, status, abort));
       if (!ok) break;
       tc_fence_after();
@@ -344,28 +336,29 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         uint32_t xr[32];
         tmem_ld32(tDQ + lane_off + cb + cc * 32, xr);
         tmem_ld_wait();
-        // row `lane` into the staging tile, 16-byte granules XOR-swizzled by row
+        // the staging tile is free once the previous store has read it
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        // row `lane` into the staging tile in the 128-byte swizzle of the
+        // store's tensor map: 16-byte granule g at g ^ (row & 7)
 #pragma unroll
         for (int g = 0; g < 8; ++g)
           *reinterpret_cast<float4*>(stg + lane * 32 + ((g ^ (lane & 7)) << 2)) =
               make_float4(__uint_as_float(xr[4 * g]), __uint_as_float(xr[4 * g + 1]),
                           __uint_as_float(xr[4 * g + 2]), __uint_as_float(xr[4 * g + 3]));
+        fence_proxy_async();
         __syncwarp();
-        // eight lanes per row: four whole 128-byte lines per store instruction
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = 4 * k + (lane >> 3), g = lane & 7;
-          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 32 + ((g ^ (rr & 7)) << 2));
-          const uint32_t sl = __shfl_sync(0xffffffffu, slot, rr);
-          if (sl != 0xFFFFFFFFu)
-            *reinterpret_cast<float4*>(part_dq + (size_t)sl * kD + cb + cc * 32 + g * 4) = v;
+        // the warp's 32 item rows, 32 columns, in one asynchronous store
+        if (lane == 0) {
+          tma_store_2d(&tm_pd, stg, cb + cc * 32, n * kTile + wq * 32);
+          bulk_commit();
         }
-        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free);
     }
+    if (lane == 0) bulk_wait_all();      // partials in global memory before the CTA retires
   }
   tc_fence_before();
   __syncthreads();
@@ -376,6 +369,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 }
 
 // dQ_i = scale * sum_j partial_ij, blocks in ascending order; one warp per row.
+// The partials sit at the pairs' item rows (slot_row).
 __global__ void __launch_bounds__(256)
 k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, float scale,
                __nv_bfloat16* __restrict__ dq) {
@@ -383,15 +377,18 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
   if (i >= P.s) return;
   const uint32_t off = __ldg(pv.row_off + (size_t)h * (P.s + 1) + i);
   const uint32_t cnt = __ldg(pv.row_cnt + (size_t)h * P.s + i);
+  const uint32_t* srow = pv.slot_row + (size_t)h * P.s * P.Nb + off;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (uint32_t k = 0; k < cnt; ++k) {
-    const float4 o = reinterpret_cast<const float4*>(part_dq + (size_t)(off + k) * kD)[lane];
+    const uint32_t row = __ldg(srow + k);
+    const float4 o = reinterpret_cast<const float4*>(part_dq + (size_t)row * kD)[lane];
     acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
   }
-  uint2 b;
-  b.x = pack_bf16x2(acc.x * scale, acc.y * scale);
-  b.y = pack_bf16x2(acc.z * scale, acc.w * scale);
-  reinterpret_cast<uint2*>(dq + ((size_t)i * P.n_h + h) * kD)[lane] = b;
+  uint2 ob;
+  ob.x = pack_bf16x2(acc.x * scale, acc.y * scale);
+  ob.y = pack_bf16x2(acc.z * scale, acc.w * scale);
+  reinterpret_cast<uint2*>(dq + ((size_t)i * P.n_h + h) * kD)[lane] = ob;
 }
 
 // =====================================================================
@@ -693,11 +690,14 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
                                 const ItemBufs& ib, const float* o32, const float* lse,
                                 const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
                                 float scale, int* status, int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv, tq, to;
+  CUtensorMap tk, tv, tq, to, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
+  float* part_dq = static_cast<float*>(part);
   if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
       !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128) ||
-      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, kD, 128))
+      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, kD, 128) ||
+      !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), kD,
+                    32, 32))
     return cudaErrorInvalidValue;
   float* rowD = static_cast<float*>(ws_bwd);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws_bwd) +
@@ -715,7 +715,6 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
                            (int)kKvSmem);
   if (e != cudaSuccess) return e;
   const float sl2 = scale * kLog2e;
-  float* part_dq = static_cast<float*>(part);
   const int nkt = (P.L + kTile - 1) / kTile;
   for (int h = 0; h < P.n_h; ++h) {
     // padding rows get -LSE log2(e) = -inf, so their P is exactly 0
@@ -725,8 +724,8 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
-      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, P, h, pv, ib.dg,
-                                                        ib.l2g, sl2, part_dq, status);
+      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, tpd, P, h, pv, ib.dg,
+                                                        ib.l2g, sl2, status);
     }
     {
       VMOBA_TRACE("k_bwd_dq_merge", st);

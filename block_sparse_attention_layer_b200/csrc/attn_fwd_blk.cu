@@ -7,11 +7,14 @@
 // the tile attends all keys of the block with no per-row masking and no
 // wasted pairs.  The item computes, for each of its queries, the partial
 // softmax state of block j (running max m, sum l, and O / l) over the
-// block's keys in chunks of 128 and stores it in the pair's slot: (m, l) in
-// fp32, O / l in fp16 -- a convex combination of V rows, so |O / l| <= max
-// |V| and fp16 keeps it to 2^-12 relative, below the bf16 output's rounding.
-// A merge kernel then combines the partials of each query with log-sum-exp
-// weights into O, its fp32 copy and LSE.
+// block's keys in chunks of 128 and stores it at the item's rows (row
+// 128 n + r for row r of item n): (m, l) in fp32, O / l in fp16 -- a convex
+// combination of V rows, so |O / l| <= max |V| and fp16 keeps it to 2^-12
+// relative, below the bf16 output's rounding.  O / l leaves through the
+// staging tiles as asynchronous TMA stores of 32 rows x 64 columns.  A merge
+// kernel then combines the partials of each query (found through the pair
+// lists' slot -> item row map) with log-sum-exp weights into O, its fp32
+// copy and LSE.
 //
 // Persistent kernel, one head per launch.  A CTA takes PAIRS of work items
 // (two consecutive 128-query tiles A, B of one block's list) so that every
@@ -24,8 +27,8 @@
 //   (warps 2-3 idle: a softmax warpgroup must start at a multiple of 4)
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query
 //               row per thread, lazy 2^8 rescale of O, then the tile's
-//               epilogue (partials out through a per-warp staging buffer so
-//               that the global stores are whole 128-byte lines).
+//               epilogue (partials out through a per-warp staging tile and
+//               an asynchronous TMA store).
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // The MMA issue order per chunk c is PV_A(c), S_A(c+1), PV_B(c), S_B(c+1):
 // while one warpgroup computes exponentials the tensor core serves the other.
@@ -120,8 +123,9 @@ __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, 
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-          const __grid_constant__ CUtensorMap tm_q, Prob P, int h, PairsView pv, float sl2,
-          __half* __restrict__ part_o, float2* __restrict__ part_ml, int* __restrict__ status) {
+          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_po,
+          Prob P, int h, PairsView pv, float sl2, float2* __restrict__ part_ml,
+          int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -292,30 +296,27 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + t * 128 + lane_off, tO = tmem + 256 + t * 128 + lane_off;
     float* stg = reinterpret_cast<float*>(sStage + (warp - 4) * kStageB);
-    const uint32_t* col_slot = pv.col_slot + (size_t)h * P.s * P.Nb;
     int Js = 0, It = 0;
     bool ok = true;
-    // this tile of pair pp and the row's slot; fetched one pair ahead, before
-    // the epilogue, so the decode and the slot load are off the critical path
+    // this tile of pair pp: its work item and query count; decoded one pair
+    // ahead, before the epilogue, so the decode is off the critical path
     int hint = 0;
-    auto fetch = [&](int pp, WorkItem& m, uint32_t& sl) {
+    auto fetch = [&](int pp, int& n, int& cnt) {
       WorkItem bb;
       int nn;
       const WorkItem aa = decode_item_pair<true>(pv, P, h, pp, &bb, &nn, hint);
-      m = t == 0 ? aa : bb;
-      sl = r < m.count ? __ldg(col_slot + m.first + r) : 0xFFFFFFFFu;
+      n = nn + t;
+      cnt = t == 0 ? aa.count : bb.count;
     };
-    WorkItem nx_me;
-    uint32_t nx_slot = 0xFFFFFFFFu;
-    if (blockIdx.x < n_pairs) fetch(blockIdx.x, nx_me, nx_slot);
+    int nx_n = 0, nx_cnt = 0;
+    if (blockIdx.x < n_pairs) fetch(blockIdx.x, nx_n, nx_cnt);
     for (int p = blockIdx.x; p < n_pairs && ok; p += G) {
-      const WorkItem me = nx_me;
-      const uint32_t slot = nx_slot;
-      if (me.count == 0) {                         // no tile B in this pair
-        if (p + G < n_pairs) fetch(p + G, nx_me, nx_slot);
+      const int n = nx_n, cnt = nx_cnt;
+      if (cnt == 0) {                              // no tile B in this pair
+        if (p + G < n_pairs) fetch(p + G, nx_n, nx_cnt);
         continue;
       }
-      const bool valid = r < me.count;
+      const bool valid = r < cnt;
       float m_run = -INFINITY, l_run = 0.f;
       for (int c = 0; c < nch; ++c, ++Js) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], Js & 1, status, abort));
@@ -329,13 +330,13 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
       if (!ok) break;
-      if (p + G < n_pairs) fetch(p + G, nx_me, nx_slot);
-      // epilogue: partial state of (query, block j) into the pair's slot
+      if (p + G < n_pairs) fetch(p + G, nx_n, nx_cnt);
+      // epilogue: partial state of (query, block j) into the item's rows
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[t], It & 1, status, abort));
       ++It;
       if (!ok) break;
       tc_fence_after();
-      if (valid) part_ml[slot] = make_float2(m_run, l_run);
+      if (valid) part_ml[(size_t)n * kTile + r] = make_float2(m_run, l_run);
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       uint32_t* stw = reinterpret_cast<uint32_t*>(stg);
 #pragma unroll 1
@@ -344,7 +345,11 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         tmem_ld32(tO + cc * 64, ob);
         tmem_ld32(tO + cc * 64 + 32, ob + 32);
         tmem_ld_wait();
-        // row `lane` into the staging tile, 16-byte granules XOR-swizzled by row
+        // the staging tile is free once the previous store has read it
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        // row `lane` into the staging tile in the 128-byte swizzle of the
+        // store's tensor map: 16-byte granule g at g ^ (row & 7)
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           uint4 u;
@@ -357,22 +362,19 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                            __uint_as_float(ob[8 * g + 7]) * inv_l);
           *reinterpret_cast<uint4*>(stw + lane * 32 + ((g ^ (lane & 7)) << 2)) = u;
         }
+        fence_proxy_async();
         __syncwarp();
-        // eight lanes per row: four whole 128-byte lines per store instruction
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = 4 * k + (lane >> 3), g = lane & 7;
-          const uint4 v = *reinterpret_cast<const uint4*>(stw + rr * 32 + ((g ^ (rr & 7)) << 2));
-          const uint32_t sl = __shfl_sync(0xffffffffu, slot, rr);
-          if (sl != 0xFFFFFFFFu)
-            *reinterpret_cast<uint4*>(part_o + (size_t)sl * kD + cc * 64 + g * 8) = v;
+        // the warp's 32 item rows, 64 columns, in one asynchronous store
+        if (lane == 0) {
+          tma_store_2d(&tm_po, stw, cc * 64, n * kTile + wq * 32);
+          bulk_commit();
         }
-        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->o_free[t]);
     }
+    if (lane == 0) bulk_wait_all();      // partials in global memory before the CTA retires
   }
   tc_fence_before();
   __syncthreads();
@@ -385,7 +387,8 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 // Combine the partial (m, l, O / l) of every query's selected blocks:
 // O_i = sum_j 2^(m_j - M) l_j (O / l)_j / sum_j 2^(m_j - M) l_j,
 // LSE_i = (M + log2 sum_j 2^(m_j - M) l_j) ln 2.
-// One warp per query row, four dims per lane, blocks in ascending order.
+// One warp per query row, four dims per lane, blocks in ascending order; the
+// partials sit at the pairs' item rows (slot_row).
 __global__ void __launch_bounds__(256)
 k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
             const float2* __restrict__ part_ml, __nv_bfloat16* __restrict__ out,
@@ -394,27 +397,53 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
   if (i >= P.s) return;
   const uint32_t off = __ldg(pv.row_off + (size_t)h * (P.s + 1) + i);
   const uint32_t cnt = __ldg(pv.row_cnt + (size_t)h * P.s + i);
-  float M = -INFINITY;
-  for (uint32_t k = 0; k < cnt; ++k) M = fmaxf(M, part_ml[off + k].x);
+  const uint32_t* srow = pv.slot_row + (size_t)h * P.s * P.Nb + off;
+  // lane k takes pairs k, k + 32, ...: item rows and (m, l) are loaded
+  // lane-parallel and broadcast to the warp by shuffles
+  uint32_t row0 = 0u;
+  float2 ml0 = make_float2(-INFINITY, 0.f);
+  if ((uint32_t)lane < cnt) {
+    row0 = __ldg(srow + lane);
+    ml0 = part_ml[row0];
+  }
+  float M = ml0.x;
+  for (uint32_t b = 32 + lane; b < cnt; b += 32) M = fmaxf(M, part_ml[__ldg(srow + b)].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float Lsum = 0.f;
-  for (uint32_t k = 0; k < cnt; ++k) {
-    const float2 ml = part_ml[off + k];
-    const float wl = exp2f(ml.x - M) * ml.y;
-    Lsum += wl;
-    const uint2 u = reinterpret_cast<const uint2*>(part_o + (size_t)(off + k) * 128)[lane];
-    const float2 a = unpack_f16x2(u.x), b = unpack_f16x2(u.y);
-    acc.x = fmaf(wl, a.x, acc.x); acc.y = fmaf(wl, a.y, acc.y);
-    acc.z = fmaf(wl, b.x, acc.z); acc.w = fmaf(wl, b.y, acc.w);
+  for (uint32_t b = 0; b < cnt; b += 32) {
+    uint32_t my_row = row0;
+    float2 ml = ml0;
+    if (b > 0) {
+      my_row = 0u;
+      ml = make_float2(-INFINITY, 0.f);
+      if (b + lane < cnt) {
+        my_row = __ldg(srow + b + lane);
+        ml = part_ml[my_row];
+      }
+    }
+    const float my_w = b + lane < cnt ? exp2f(ml.x - M) * ml.y : 0.f;
+    const int kn = (int)min(32u, cnt - b);
+#pragma unroll 4
+    for (int k = 0; k < kn; ++k) {
+      const uint32_t row = __shfl_sync(0xffffffffu, my_row, k);
+      const float wl = __shfl_sync(0xffffffffu, my_w, k);
+      Lsum += wl;
+      const uint2 u = reinterpret_cast<const uint2*>(part_o + (size_t)row * 128)[lane];
+      const float2 a = unpack_f16x2(u.x), c = unpack_f16x2(u.y);
+      acc.x = fmaf(wl, a.x, acc.x); acc.y = fmaf(wl, a.y, acc.y);
+      acc.z = fmaf(wl, c.x, acc.z); acc.w = fmaf(wl, c.y, acc.w);
+    }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
   const size_t row = ((size_t)i * P.n_h + h) * 128;
   reinterpret_cast<float4*>(o32 + row)[lane] = acc;
-  uint2 b;
-  b.x = pack_bf16x2(acc.x, acc.y);
-  b.y = pack_bf16x2(acc.z, acc.w);
-  reinterpret_cast<uint2*>(out + row)[lane] = b;
+  uint2 ob;
+  ob.x = pack_bf16x2(acc.x, acc.y);
+  ob.y = pack_bf16x2(acc.z, acc.w);
+  reinterpret_cast<uint2*>(out + row)[lane] = ob;
   if (lane == 0)
     lse[(size_t)h * P.s + i] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY;
 }
@@ -422,26 +451,29 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
 }  // namespace
 
 size_t blk_partial_bytes(const Prob& P) {
-  // one head's worst case: every (query, block) pair selected
-  return align_up((size_t)P.s * P.Nb * 128 * sizeof(float), 256) +
-         align_up((size_t)P.s * P.Nb * sizeof(float2), 256);
+  // one head's partials, one row per work-item row (item_rows_capacity rows):
+  // 128 fp32 (dQ pass) or 128 fp16 (forward O / l), then the forward's (m, l)
+  const size_t rows = item_rows_capacity(P);
+  return align_up(rows * 128 * sizeof(float), 256) + align_up(rows * sizeof(float2), 256);
 }
 
 cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
                                 const ItemBufs& ib, float scale, void* out, float* o32,
                                 float* lse, int* status, int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv, tq;
+  CUtensorMap tk, tv, tq, tpo;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
+  const size_t prows = item_rows_capacity(P);
+  __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
+  float2* part_ml = reinterpret_cast<float2*>(
+      static_cast<char*>(part) + align_up(prows * 128 * sizeof(float), 256));
   if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
-      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128))
+      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128) ||
+      !make_tmap_2d(&tpo, part_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, prows, kD, 64, 32))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_fwd_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
-  float2* part_ml = reinterpret_cast<float2*>(
-      static_cast<char*>(part) + align_up((size_t)P.s * P.Nb * 128 * sizeof(float), 256));
   const float sl2 = scale * 1.4426950408889634f;
   for (int h = 0; h < P.n_h; ++h) {
     e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q), nullptr, ib.qg,
@@ -449,7 +481,7 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_fwd_blk", st);
-      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, P, h, pv, sl2, part_o, part_ml,
+      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, tpo, P, h, pv, sl2, part_ml,
                                                         status);
     }
     {

@@ -5,14 +5,16 @@
 //   row_cnt[i]   number of blocks query i selected;
 //   row_off[i]   exclusive prefix of row_cnt: the pairs of query i occupy
 //                slots row_off[i] .. row_off[i]+row_cnt[i]-1, in block order
-//                ("CSR"); partial results of the attention kernels live there;
+//                ("CSR");
 //   col_off[j]   start of block j's query list in col_rows ("CSC"), queries
 //                in ascending order (deterministic);
-//   col_slot     beside every col_rows entry, the pair slot of that
-//                (query, block) pair, so the attention kernels index the
-//                CSR partials directly;
 //   item_off[j]  first work item of block j: its query list cut into tiles of
 //                128 queries; item_off[N_b] = number of work items;
+//   slot_row     for every CSR slot, the item row of that (query, block) pair:
+//                128 item_off[j] + its position in block j's list.  The
+//                attention kernels write partial results item by item (whole
+//                128-row tiles) and the merges read them through slot_row in
+//                each query's block order;
 //   pitem_off[j] the same for pairs of consecutive tiles (256 queries);
 //   blk_order    the blocks by list length, longest first (ties: lower j
 //                first), so that kernels launching one CTA per block start
@@ -145,19 +147,23 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
 }
 
 // Per (chunk, head): write every row of the chunk into the lists of the
-// blocks it selected, at chunk base + rank among the chunk's rows, with the
-// row's pair slot (its CSR offset plus the blocks below j it selected).
+// blocks it selected, at chunk base + rank among the chunk's rows, and the
+// item row of that entry at the row's pair slot (its CSR offset plus the
+// blocks below j it selected).
 __global__ void __launch_bounds__(kChunkRows)
 k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restrict__ chunk_base,
-             int n_chunks, const uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_rows,
-             uint32_t* __restrict__ col_slot) {
+             int n_chunks, const uint32_t* __restrict__ row_off,
+             const uint32_t* __restrict__ col_off, const uint32_t* __restrict__ item_off,
+             uint32_t* __restrict__ col_rows, uint32_t* __restrict__ slot_row) {
   __shared__ uint32_t wcnt[kChunkRows / 32][32];
   const int c = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = c * kChunkRows + threadIdx.x;
   const uint32_t* cb = chunk_base + ((size_t)h * n_chunks + c) * P.Nb;
   uint32_t* rows = col_rows + (size_t)h * P.s * P.Nb;
-  uint32_t* slots = col_slot + (size_t)h * P.s * P.Nb;
+  uint32_t* srow = slot_row + (size_t)h * P.s * P.Nb;
+  const uint32_t* coff = col_off + (size_t)h * (P.Nb + 1);
+  const uint32_t* ioff = item_off + (size_t)h * (P.Nb + 1);
   uint32_t slot = (i < P.s) ? __ldg(row_off + (size_t)h * (P.s + 1) + i) : 0u;
   for (int w = 0; w < P.Wb; ++w) {
     const uint32_t bits = (i < P.s) ? __ldg(sel + ((size_t)h * P.s + i) * P.Wb + w) : 0u;
@@ -182,8 +188,10 @@ k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restric
       const unsigned m = __ballot_sync(0xffffffffu, (bits >> b) & 1u);
       if ((bits >> b) & 1u) {
         const uint32_t rank = __popc(m & ((1u << lane) - 1u));
-        rows[wcnt[warp][b] + rank] = (uint32_t)i;
-        slots[wcnt[warp][b] + rank] = slot++;
+        const uint32_t e = wcnt[warp][b] + rank;    // entry of block j's list
+        const int j = w * 32 + b;
+        rows[e] = (uint32_t)i;
+        srow[slot++] = kTile * __ldg(ioff + j) + (e - __ldg(coff + j));
       }
     }
     __syncthreads();
@@ -204,7 +212,7 @@ size_t pairs_ws_bytes(const Prob& P) {
   take(sizeof(uint32_t) * 4 * P.n_h);                           // head totals
   take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);     // chunk counts / bases
   take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_rows (worst case)
-  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_slot (worst case)
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // slot_row (worst case)
   take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);                // blk_order
   return b;
 }
@@ -222,7 +230,7 @@ PairsView pairs_view(const Prob& P, void* base) {
   v.head_totals = take(sizeof(uint32_t) * 4 * P.n_h);
   v.chunk = take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);
   v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
-  v.col_slot = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
+  v.slot_row = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
   v.blk_order = take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);
   v.n_chunks = n_chunks;
   return v;
@@ -241,8 +249,8 @@ cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v,
   }
   {
     VMOBA_TRACE("k_pairs_fill", st);
-    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.row_off, v.col_rows,
-                                           v.col_slot);
+    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.row_off, v.col_off,
+                                           v.item_off, v.col_rows, v.slot_row);
   }
   count_launches(3);
   return cudaGetLastError();

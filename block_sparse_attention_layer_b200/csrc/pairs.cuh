@@ -14,7 +14,7 @@ struct PairsView {
   uint32_t* head_totals;  // [n_h][4]     pairs, work items, item pairs, 0
   uint32_t* chunk;        // [n_h][chunks][N_b] scratch (chunk bases)
   uint32_t* col_rows;     // [n_h][s*N_b] query lists, block by block
-  uint32_t* col_slot;     // [n_h][s*N_b] pair slot of each list entry
+  uint32_t* slot_row;     // [n_h][s*N_b] item row of each CSR pair slot
   uint32_t* blk_order;    // [n_h][N_b]   blocks by query-list length, longest first
   int n_chunks;
 };
@@ -23,7 +23,7 @@ struct PairsView {
 struct WorkItem {
   int j;                  // block
   int count;              // queries in the tile (0 when the tile does not exist)
-  uint32_t first;         // index of the tile's first entry in col_rows / col_slot
+  uint32_t first;         // index of the tile's first entry in col_rows
 };
 
 // Block j with off[j] <= n < off[j+1], for a non-decreasing offset array

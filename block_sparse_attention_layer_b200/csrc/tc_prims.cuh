@@ -93,6 +93,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// 2-D tiled store of the box at (x, y) from shared memory (x, y >= 0; x *
+// elem a multiple of 16 bytes), tracked by the issuing thread's bulk groups.
+// The shared source must have been written before a fence_proxy_async().
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x,
+                                             int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// All committed bulk stores of this thread have read their shared source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// All committed bulk stores of this thread are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 // Bring the box at (x, y) into L2 ahead of its load (no shared memory, no
 // barrier; same x alignment rule as the load).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
@@ -275,9 +295,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 }  // namespace tc
 
-// Host: a 2-D bf16 tensor map over `rows` x `cols` (row pitch cols*2 bytes)
-// with a 64-column x box_rows box and 128-byte swizzle.  Returns false if the
-// driver entry point is missing or rejects the map.
+// Host: a 2-D tensor map over `rows` x `cols` elements of `elem_bytes` each
+// (row pitch cols * elem_bytes) with a box_cols x box_rows box whose inner
+// extent is one 128-byte swizzled row (box_cols * elem_bytes == 128).
+// Returns false if the arguments break that, or if the driver entry point is
+// missing or rejects the map.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  uint32_t elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                  uint32_t box_rows);
+// The bf16 case: 64-column x box_rows box.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows);
 
