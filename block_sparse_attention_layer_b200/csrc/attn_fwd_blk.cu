@@ -52,6 +52,7 @@ constexpr int kThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageB = 32 * 32 * 4;     // per softmax warp: 32 rows x 32 fp32
+constexpr uint32_t kGatherThreads = 64;       // warps 2-3 gather the query tiles
 
 struct Bars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
@@ -123,7 +124,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, 
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_po,
+          const __grid_constant__ CUtensorMap tm_po, const __nv_bfloat16* __restrict__ q,
           Prob P, int h, PairsView pv, float sl2, float2* __restrict__ part_ml,
           int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
@@ -149,7 +150,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 4);
       mbar_init(&bars->o_final[i], 1); mbar_init(&bars->o_free[i], 4);
     }
-    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_full, kGatherThreads);
     mbar_init(&bars->q_empty, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -168,22 +169,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_q);
-      int J = 0, it_local = 0, hint = 0, hint_pf = 0;
+      int J = 0, hint = 0;
       bool ok = true;
-      for (int p = blockIdx.x; p < n_pairs && ok; p += G, ++it_local) {
+      for (int p = blockIdx.x; p < n_pairs && ok; p += G) {
         WorkItem b;
         int n0;
         const WorkItem a = decode_item_pair<false>(pv, P, h, p, &b, &n0, hint);
-        if (it_local >= 1) ok = mbar_wait(&bars->q_empty, (it_local - 1) & 1, status, abort);
-        if (!ok) break;
-        mbar_expect_tx(&bars->q_full, b.count > 0 ? 2 * kTileB : kTileB);
-        tma_load_2d(sQ, &tm_q, &bars->q_full, 0, n0 * kTile);
-        tma_load_2d(sQ + kHalf, &tm_q, &bars->q_full, 64, n0 * kTile);
-        if (b.count > 0) {
-          tma_load_2d(sQ + kTileB, &tm_q, &bars->q_full, 0, (n0 + 1) * kTile);
-          tma_load_2d(sQ + kTileB + kHalf, &tm_q, &bars->q_full, 64, (n0 + 1) * kTile);
-        }
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + a.j * P.L + c * kTile;
           const int st = J & 1;
@@ -198,17 +189,55 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
           tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
-        if (ok && p + G < n_pairs) {
-          // the next pair's Q tiles into L2 behind this pair's loads
-          WorkItem b1;
-          int n1;
-          decode_item_pair<false>(pv, P, h, p + G, &b1, &n1, hint_pf);
-          for (int t = 0; t < (b1.count > 0 ? 2 : 1); ++t) {
-            tma_prefetch_l2_2d(&tm_q, 0, (n1 + t) * kTile);
-            tma_prefetch_l2_2d(&tm_q, 64, (n1 + t) * kTile);
-          }
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // -------------------------------------------------------- query gather
+    // The pair's query rows straight from Q (one head's rows stay in L2):
+    // warp w copies rows [64 w, 64 w + 64) of each tile, two rows per step
+    // (16 lanes x 16 bytes per 256-byte row), into the 128-byte-swizzled
+    // layout the MMA descriptors read (16-byte granule g of row r at
+    // g ^ (r & 7)); rows past the tile's queries are zero-filled.
+    const int w = warp - 2, c = lane & 15, hr = lane >> 4;
+    const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
+    const uint32_t qbase = smem_u32(sQ);
+    int it_local = 0, hint = 0;
+    bool ok = true;
+    for (int p = blockIdx.x; p < n_pairs && ok; p += G, ++it_local) {
+      WorkItem tb;
+      int n0;
+      const WorkItem ta = decode_item_pair<true>(pv, P, h, p, &tb, &n0, hint);
+      if (it_local >= 1)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars->q_empty, (it_local - 1) & 1, status, abort));
+      if (!ok) break;
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const WorkItem m = t == 0 ? ta : tb;
+        if (m.count == 0) continue;                // no tile B in this pair
+        const int base = 64 * w;
+        // query indices of the warp's 64 rows, one per lane and half
+        const uint32_t idx0 =
+            base + lane < m.count ? __ldg(col_rows + m.first + base + lane) : 0u;
+        const uint32_t idx1 =
+            base + 32 + lane < m.count ? __ldg(col_rows + m.first + base + 32 + lane) : 0u;
+        const uint32_t tbase = qbase + t * kTileB + (c >> 3) * kHalf;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const int rr = 2 * k + hr;                // row within the warp's 64
+          const uint32_t i0 = __shfl_sync(0xffffffffu, idx0, rr & 31);
+          const uint32_t i1 = __shfl_sync(0xffffffffu, idx1, rr & 31);
+          const int r = base + rr;
+          const bool in = r < m.count;
+          const uint32_t i = in ? (rr < 32 ? i0 : i1) : 0u;
+          cp_async16(tbase + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                     q + ((size_t)i * P.n_h + h) * kD + c * 8, in ? 16u : 0u);
         }
       }
+      // copies landed, made visible to the tensor core's (async) proxy
+      cp_async_wait_all();
+      fence_proxy_async();
+      mbar_arrive(&bars->q_full);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -461,14 +490,13 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
                                 const uint32_t* sel, const PairsView& pv, void* part,
                                 const ItemBufs& ib, float scale, void* out, float* o32,
                                 float* lse, int* status, int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv, tq, tpo;
+  CUtensorMap tk, tv, tpo;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   const size_t prows = item_rows_capacity(P);
   __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
   float2* part_ml = reinterpret_cast<float2*>(
       static_cast<char*>(part) + align_up(prows * 128 * sizeof(float), 256));
   if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
-      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128) ||
       !make_tmap_2d(&tpo, part_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, prows, kD, 64, 32))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_fwd_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -476,13 +504,10 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
   if (e != cudaSuccess) return e;
   const float sl2 = scale * 1.4426950408889634f;
   for (int h = 0; h < P.n_h; ++h) {
-    e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q), nullptr, ib.qg,
-                            nullptr, nullptr, nullptr, nullptr, nullptr, 0.f, num_sms, st);
-    if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_fwd_blk", st);
-      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(tk, tv, tq, tpo, P, h, pv, sl2, part_ml,
-                                                        status);
+      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(
+          tk, tv, tpo, static_cast<const __nv_bfloat16*>(q), P, h, pv, sl2, part_ml, status);
     }
     {
       VMOBA_TRACE("k_fwd_merge", st);

@@ -93,6 +93,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// 16-byte asynchronous copy global -> shared through L2 (cp.async.cg); with
+// src_bytes = 0 the 16 bytes are zero-filled and nothing is read.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// This thread's cp.async copies have landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
 // 2-D tiled store of the box at (x, y) from shared memory (x, y >= 0; x *
 // elem a multiple of 16 bytes), tracked by the issuing thread's bulk groups.
 // The shared source must have been written before a fence_proxy_async().
