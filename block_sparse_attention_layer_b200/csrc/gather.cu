@@ -4,14 +4,14 @@
 // [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
 // rows past the list end are zero.  The attention kernels then fetch query
 // tiles with plain 2-D TMA instead of scattered loads.  One warp per item;
-// each lane moves 8 bytes of a 256-byte row, eight rows in flight.
+// 16 lanes x 16 bytes move a 256-byte row, sixteen rows in flight.
 #include "common.cuh"
 #include "pairs.cuh"
 
 namespace vmoba {
 namespace {
 
-constexpr int kRowsInFlight = 8;
+constexpr int kPairsInFlight = 8;        // two rows per warp instruction
 
 __global__ void __launch_bounds__(256)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
@@ -22,6 +22,7 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
   const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
   const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int lane = threadIdx.x & 31;
+  const int half = lane >> 4, c = lane & 15;     // row of the instruction's two, 16-byte chunk
   const int warps = (gridDim.x * blockDim.x) >> 5;
   int hint = 0;
   for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < n_items; n += warps) {
@@ -29,24 +30,24 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
     const int count = it.count;
     const uint32_t* rows = col_rows + it.first;
     const size_t base = (size_t)n * kTile;
-    for (int r0 = 0; r0 < kTile; r0 += kRowsInFlight) {
-      uint2 va[kRowsInFlight], vb[kRowsInFlight];
+    for (int r0 = 0; r0 < kTile; r0 += 2 * kPairsInFlight) {
+      uint4 va[kPairsInFlight], vb[kPairsInFlight];
 #pragma unroll
-      for (int u = 0; u < kRowsInFlight; ++u) {
-        const int r = r0 + u;
-        va[u] = make_uint2(0u, 0u);
-        vb[u] = make_uint2(0u, 0u);
+      for (int u = 0; u < kPairsInFlight; ++u) {
+        const int r = r0 + 2 * u + half;
+        va[u] = make_uint4(0u, 0u, 0u, 0u);
+        vb[u] = make_uint4(0u, 0u, 0u, 0u);
         if (r < count) {
           const size_t src = ((size_t)__ldg(rows + r) * P.n_h + h) * 128;
-          va[u] = __ldg(reinterpret_cast<const uint2*>(a + src) + lane);
-          if (b) vb[u] = __ldg(reinterpret_cast<const uint2*>(b + src) + lane);
+          va[u] = __ldg(reinterpret_cast<const uint4*>(a + src) + c);
+          if (b) vb[u] = __ldg(reinterpret_cast<const uint4*>(b + src) + c);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kRowsInFlight; ++u) {
-        const size_t dst = (base + r0 + u) * 128;
-        reinterpret_cast<uint2*>(ag + dst)[lane] = va[u];
-        if (b) reinterpret_cast<uint2*>(bg + dst)[lane] = vb[u];
+      for (int u = 0; u < kPairsInFlight; ++u) {
+        const size_t dst = (base + r0 + 2 * u + half) * 128;
+        reinterpret_cast<uint4*>(ag + dst)[c] = va[u];
+        if (b) reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
       }
     }
     if (fa) {
