@@ -56,7 +56,7 @@ constexpr uint32_t kGatherThreads = 64;       // warps 2-3 gather the query tile
 
 struct Bars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];                          // per query tile of the pair
   uint64_t s_full[2], p_full[2], o_final[2], o_free[2];   // per tile of the pair
   uint32_t tmem_base;
   int abort;
@@ -150,8 +150,10 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 4);
       mbar_init(&bars->o_final[i], 1); mbar_init(&bars->o_free[i], 4);
     }
-    mbar_init(&bars->q_full, kGatherThreads);
-    mbar_init(&bars->q_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->q_full[t], kGatherThreads);
+      mbar_init(&bars->q_empty[t], 1);
+    }
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -207,14 +209,19 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       WorkItem tb;
       int n0;
       const WorkItem ta = decode_item_pair<true>(pv, P, h, p, &tb, &n0, hint);
-      if (it_local >= 1)
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars->q_empty, (it_local - 1) & 1, status, abort));
-      if (!ok) break;
+      // tile by tile: the next pair's tile A is copied while this pair's
+      // tile B is still being read
 #pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
+      for (int t = 0; t < 2 && ok; ++t) {
         const WorkItem m = t == 0 ? ta : tb;
-        if (m.count == 0) continue;                // no tile B in this pair
+        if (it_local >= 1)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&bars->q_empty[t], (it_local - 1) & 1, status, abort));
+        if (!ok) break;
+        if (m.count == 0) {                        // no tile B in this pair
+          mbar_arrive(&bars->q_full[t]);
+          continue;
+        }
         const int base = 64 * w;
         // query indices of the warp's 64 rows, one per lane and half
         const uint32_t idx0 =
@@ -233,11 +240,11 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           cp_async16(tbase + r * 128 + (((c & 7) ^ (r & 7)) << 4),
                      q + ((size_t)i * P.n_h + h) * kD + c * 8, in ? 16u : 0u);
         }
+        // copies landed, made visible to the tensor core's (async) proxy
+        cp_async_wait_all();
+        fence_proxy_async();
+        mbar_arrive(&bars->q_full[t]);
       }
-      // copies landed, made visible to the tensor core's (async) proxy
-      cp_async_wait_all();
-      fence_proxy_async();
-      mbar_arrive(&bars->q_full);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -273,15 +280,20 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         int n0;
         decode_item_pair<false>(pv, P, h, p, &b, &n0, hint);
         const int nt = b.count > 0 ? 2 : 1;
-        if (!mbar_wait(&bars->q_full, it_local & 1, status, abort)) { ok = false; break; }
         {
           const int st = Jk & 1;
           if (!mbar_wait(&bars->full_k[st], (Jk >> 1) & 1, status, abort)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t kb = smem_u32(sK + st * kTileB);
-          for (int t = 0; t < nt; ++t) issue_s(t, kb, nch == 1);
+          for (int t = 0; t < 2 && ok; ++t) {
+            // every pair passes both tiles' barriers; an absent tile B is
+            // released at once
+            if (!mbar_wait(&bars->q_full[t], it_local & 1, status, abort)) { ok = false; break; }
+            tc_fence_after();
+            if (t < nt) issue_s(t, kb, nch == 1);
+            if (t >= nt || nch == 1) mma_commit(&bars->q_empty[t]);
+          }
+          if (!ok) break;
           mma_commit(&bars->empty_k[st]);
-          if (nch == 1) mma_commit(&bars->q_empty);
         }
         for (int c = 0; c < nch && ok; ++c) {
           const int Jc = Jk + c, stc = Jc & 1, st1 = (Jc + 1) & 1;
@@ -305,14 +317,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
                 kb1 = smem_u32(sK + st1 * kTileB);
               }
               issue_s(t, kb1, c + 1 == nch - 1);
+              if (c + 1 == nch - 1) mma_commit(&bars->q_empty[t]);   // tile t's last S
             }
           }
           if (!ok) break;
           mma_commit(&bars->empty_v[stc]);
-          if (more) {
-            mma_commit(&bars->empty_k[st1]);
-            if (c + 1 == nch - 1) mma_commit(&bars->q_empty);
-          }
+          if (more) mma_commit(&bars->empty_k[st1]);
         }
         Jk += nch;
         for (int t = 0; t < nt; ++t) ++It[t];
