@@ -23,14 +23,26 @@
 // along for the stats (a last-pass bucket holds one score value, so its
 // share of the mass is exact).
 #include "common.cuh"
+#include "tc_prims.cuh"
 
 namespace vmoba {
 namespace {
 
 constexpr int kSel_Search = 0, kSel_Resolved = 1, kSel_All = 2, kSel_Ties = 3;
 
-__device__ __forceinline__ float ld_f(const float* p) { return __ldg(p); }
-__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+// Element k of a 16-byte vector held as four 32-bit words.
+template <typename E>
+__device__ __forceinline__ float word_elem(const uint32_t* w, int k);
+template <>
+__device__ __forceinline__ float word_elem<float>(const uint32_t* w, int k) {
+  return __uint_as_float(w[k]);
+}
+template <>
+__device__ __forceinline__ float word_elem<__nv_bfloat16>(const uint32_t* w, int k) {
+  // bf16 is the top half of an fp32: element 2m in the low 16 bits of word m
+  const uint32_t x = w[k >> 1];
+  return __uint_as_float((k & 1) ? (x & 0xFFFF0000u) : (x << 16));
+}
 
 __global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_h * kHistBins;
@@ -49,7 +61,10 @@ __global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
 
 // ---------------------------------------------------------------- scores
 // 64 queries x 64 blocks per CTA step, 256 threads, 4x4 outputs per thread,
-// fp32 FMA over d.  Q tile and B chunk staged transposed in shared memory.
+// fp32 FMA over d in pairs (fma.rn.f32x2: two round-to-nearest FMAs, the same
+// results as scalar ones in the same order).  Q tile and B chunk are staged
+// transposed in shared memory: 16-byte global loads, one row per lane, so the
+// transposed stores hit 32 distinct banks (row pitch 68 floats).
 constexpr int kSQ = 64, kSB = 64, kSPad = 68;
 
 template <typename E, int D>
@@ -62,47 +77,65 @@ k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scal
   const int i0 = blockIdx.x * kSQ, h = blockIdx.y;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 
-  for (int idx = threadIdx.x; idx < kSQ * D; idx += 256) {
-    int r = idx / D, c = idx - r * D;
-    int i = i0 + r;
-    Qs[c * kSPad + r] = (i < P.s) ? ld_f(q + ((size_t)i * P.n_h + h) * D + c) : 0.f;
+  // Q: 16-byte vectors of V elements; item = (vector g, query r), r fastest
+  constexpr int V = 16 / (int)sizeof(E);
+  for (int id = threadIdx.x; id < kSQ * (D / V); id += 256) {
+    const int r = id % kSQ, g = id / kSQ, i = i0 + r;
+    float x[V];
+    if (i < P.s) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)i * P.n_h + h) * D) + g);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < V; ++k) x[k] = word_elem<E>(w, k);
+    } else {
+#pragma unroll
+      for (int k = 0; k < V; ++k) x[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < V; ++k) Qs[(g * V + k) * kSPad + r] = x[k];
   }
   float vmax = -INFINITY;
   const float* Bh = B + (size_t)h * P.Nb * D;
   for (int j0 = 0; j0 < P.Nb; j0 += kSB) {
     __syncthreads();
-    for (int idx = threadIdx.x; idx < kSB * D; idx += 256) {
-      int r = idx / D, c = idx - r * D;
-      int j = j0 + r;
-      Bs[c * kSPad + r] = (j < P.Nb) ? __ldg(Bh + (size_t)j * D + c) : 0.f;
+    for (int id = threadIdx.x; id < kSB * (D / 4); id += 256) {
+      const int r = id % kSB, g = id / kSB, j = j0 + r;
+      const float4 v = j < P.Nb ? __ldg(reinterpret_cast<const float4*>(Bh + (size_t)j * D) + g)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      Bs[(4 * g + 0) * kSPad + r] = v.x;
+      Bs[(4 * g + 1) * kSPad + r] = v.y;
+      Bs[(4 * g + 2) * kSPad + r] = v.z;
+      Bs[(4 * g + 3) * kSPad + r] = v.w;
     }
     __syncthreads();
-    float acc[4][4];
+    uint64_t acc[4][2];            // [query a][block pair (0,1) / (2,3)]
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0ull;
 #pragma unroll 8
     for (int c = 0; c < D; ++c) {
-      float4 qa = *reinterpret_cast<const float4*>(Qs + c * kSPad + 4 * ty);
-      float4 bb = *reinterpret_cast<const float4*>(Bs + c * kSPad + 4 * tx);
+      const float4 qa = *reinterpret_cast<const float4*>(Qs + c * kSPad + 4 * ty);
+      const float4 bb = *reinterpret_cast<const float4*>(Bs + c * kSPad + 4 * tx);
+      const uint64_t b01 = tc::f32x2(bb.x, bb.y), b23 = tc::f32x2(bb.z, bb.w);
       const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-      const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], bv[b], acc[a][b]);
+      for (int a = 0; a < 4; ++a) {
+        const uint64_t qq = tc::f32x2(qv[a], qv[a]);
+        acc[a][0] = tc::fma_x2(qq, b01, acc[a][0]);
+        acc[a][1] = tc::fma_x2(qq, b23, acc[a][1]);
+      }
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       int i = i0 + 4 * ty + a;
       if (i >= P.s) continue;
       float* row = S + ((size_t)h * P.s + i) * P.Nb;
+      const float2 p01 = tc::f32x2_split(acc[a][0]), p23 = tc::f32x2_split(acc[a][1]);
+      const float av[4] = {p01.x, p01.y, p23.x, p23.y};
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         int j = j0 + 4 * tx + b;
         if (j < P.Nb) {
-          float x = acc[a][b] * scale;
+          float x = av[b] * scale;
           row[j] = x;
           vmax = fmaxf(vmax, x);
         }
