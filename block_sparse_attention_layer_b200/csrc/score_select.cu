@@ -60,20 +60,22 @@ __global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
 }
 
 // ---------------------------------------------------------------- scores
-// 64 queries x 64 blocks per CTA step, 256 threads, 4x4 outputs per thread,
-// fp32 FMA over d in pairs (fma.rn.f32x2: two round-to-nearest FMAs, the same
-// results as scalar ones in the same order).  Q tile and B chunk are staged
-// transposed in shared memory: 16-byte global loads, one row per lane, so the
-// transposed stores hit 32 distinct banks (row pitch 68 floats).
-constexpr int kSQ = 64, kSB = 64, kSPad = 68;
+// 128 queries x 64 blocks per CTA step, 256 threads (16 x 16), 8 queries x
+// 4 blocks per thread, fp32 FMA over d in pairs of queries (fma.rn.f32x2:
+// two round-to-nearest FMAs, the same results as scalar ones in the same
+// order).  Q tile and B chunk are staged transposed in shared memory: 16-byte
+// global loads, one row per lane, so the transposed stores hit 32 distinct
+// banks (row pitches 132 and 68 floats).  Per d step a thread reads two
+// query float4s (a broadcast across its half-warp) and one block float4.
+constexpr int kSQ = 128, kSB = 64, kQPad = 132, kBPad = 68;
 
 template <typename E, int D>
 __global__ void __launch_bounds__(256)
 k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scale,
         float* __restrict__ S, SelState* __restrict__ st) {
   extern __shared__ __align__(16) float sm[];
-  float* Qs = sm;                  // [D][kSPad]
-  float* Bs = sm + D * kSPad;      // [D][kSPad]
+  float* Qs = sm;                  // [D][kQPad]
+  float* Bs = sm + D * kQPad;      // [D][kBPad]
   const int i0 = blockIdx.x * kSQ, h = blockIdx.y;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 
@@ -92,7 +94,7 @@ k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scal
       for (int k = 0; k < V; ++k) x[k] = 0.f;
     }
 #pragma unroll
-    for (int k = 0; k < V; ++k) Qs[(g * V + k) * kSPad + r] = x[k];
+    for (int k = 0; k < V; ++k) Qs[(g * V + k) * kQPad + r] = x[k];
   }
   float vmax = -INFINITY;
   const float* Bh = B + (size_t)h * P.Nb * D;
@@ -102,42 +104,48 @@ k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scal
       const int r = id % kSB, g = id / kSB, j = j0 + r;
       const float4 v = j < P.Nb ? __ldg(reinterpret_cast<const float4*>(Bh + (size_t)j * D) + g)
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      Bs[(4 * g + 0) * kSPad + r] = v.x;
-      Bs[(4 * g + 1) * kSPad + r] = v.y;
-      Bs[(4 * g + 2) * kSPad + r] = v.z;
-      Bs[(4 * g + 3) * kSPad + r] = v.w;
+      Bs[(4 * g + 0) * kBPad + r] = v.x;
+      Bs[(4 * g + 1) * kBPad + r] = v.y;
+      Bs[(4 * g + 2) * kBPad + r] = v.z;
+      Bs[(4 * g + 3) * kBPad + r] = v.w;
     }
     __syncthreads();
-    uint64_t acc[4][2];            // [query a][block pair (0,1) / (2,3)]
+    uint64_t acc[4][4];            // [query pair (2a, 2a+1)][block b]
 #pragma unroll
-    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0ull;
-#pragma unroll 8
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0ull;
+#pragma unroll 4
     for (int c = 0; c < D; ++c) {
-      const float4 qa = *reinterpret_cast<const float4*>(Qs + c * kSPad + 4 * ty);
-      const float4 bb = *reinterpret_cast<const float4*>(Bs + c * kSPad + 4 * tx);
-      const uint64_t b01 = tc::f32x2(bb.x, bb.y), b23 = tc::f32x2(bb.z, bb.w);
-      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float4 q0 = *reinterpret_cast<const float4*>(Qs + c * kQPad + 8 * ty);
+      const float4 q1 = *reinterpret_cast<const float4*>(Qs + c * kQPad + 8 * ty + 4);
+      const float4 bb = *reinterpret_cast<const float4*>(Bs + c * kBPad + 4 * tx);
+      const uint64_t qp[4] = {tc::f32x2(q0.x, q0.y), tc::f32x2(q0.z, q0.w),
+                              tc::f32x2(q1.x, q1.y), tc::f32x2(q1.z, q1.w)};
+      const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const uint64_t qq = tc::f32x2(qv[a], qv[a]);
-        acc[a][0] = tc::fma_x2(qq, b01, acc[a][0]);
-        acc[a][1] = tc::fma_x2(qq, b23, acc[a][1]);
+      for (int b = 0; b < 4; ++b) {
+        const uint64_t b2 = tc::f32x2(bv[b], bv[b]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) acc[a][b] = tc::fma_x2(qp[a], b2, acc[a][b]);
       }
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-      int i = i0 + 4 * ty + a;
-      if (i >= P.s) continue;
-      float* row = S + ((size_t)h * P.s + i) * P.Nb;
-      const float2 p01 = tc::f32x2_split(acc[a][0]), p23 = tc::f32x2_split(acc[a][1]);
-      const float av[4] = {p01.x, p01.y, p23.x, p23.y};
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        int j = j0 + 4 * tx + b;
-        if (j < P.Nb) {
-          float x = av[b] * scale;
-          row[j] = x;
-          vmax = fmaxf(vmax, x);
+      for (int e = 0; e < 2; ++e) {
+        const int i = i0 + 8 * ty + 2 * a + e;
+        if (i >= P.s) continue;
+        float* row = S + ((size_t)h * P.s + i) * P.Nb;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int j = j0 + 4 * tx + b;
+          if (j < P.Nb) {
+            const float2 pr = tc::f32x2_split(acc[a][b]);
+            const float x = (e ? pr.y : pr.x) * scale;
+            row[j] = x;
+            vmax = fmaxf(vmax, x);
+          }
         }
       }
     }
@@ -428,7 +436,7 @@ __global__ void k_stats(Prob P, const SelState* __restrict__ st, vmoba_head_stat
 template <typename E, int D>
 cudaError_t launch_score(const Prob& P, const void* q, const float* B, float scale, float* S,
                          SelState* st, cudaStream_t stream) {
-  const size_t smem = sizeof(float) * 2 * D * kSPad;
+  const size_t smem = sizeof(float) * D * (kQPad + kBPad);
   cudaError_t e = cudaFuncSetAttribute(k_score<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
