@@ -21,10 +21,11 @@
 // K / V chunk it loads serves 256 queries; CTA b takes pairs b, b + G, ...
 // (static round-robin: all pairs of a layer cost about the same).
 // Roles (384 threads):
-//   warp 0      TMA producer: the pair's two query tiles (item-ordered copy
-//               of Q, gather.cu) and the block's K / V chunks (2-stage rings);
+//   warp 0      TMA producer: the block's K / V chunks (2-stage rings);
 //   warp 1      TMEM owner (512 columns) and single-thread MMA issuer;
-//   (warps 2-3 idle: a softmax warpgroup must start at a multiple of 4)
+//   warps 2-3   query gather: the pair's two query tiles straight from Q by
+//               cp.async (a softmax warpgroup must start at a multiple of 4,
+//               which leaves these two warps to the copy);
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one query
 //               row per thread, lazy 2^8 rescale of O, then the tile's
 //               epilogue (partials out through a per-warp staging tile and
