@@ -42,6 +42,12 @@ step open, the reading taken is stated in the function's docstring:
     pairs of the head's pool (global) or k blocks per query row (local) --
     ranked like the method, ties by index.  The pages give no k; it is a
     parameter here.
+11. The other reading of "normalised similarity", rejected for the method
+    and kept as a variant: each query's scores are normalised by a softmax
+    over that query's own N_b blocks and divided by s, so every query row
+    carries mass 1/s of the head's total 1; the head's whole pool is ranked
+    by that value (ties by query, then block) and key design 3's cumulative
+    rule is applied to it.
 
 Pins (what ties each function to something other than itself) are in
 ``tests/test_oracle_pins.py``; each function's docstring lists them.
@@ -233,6 +239,40 @@ def topk_global_select(S_h: np.ndarray, k: int):
 def _row_softmax(row: np.ndarray) -> np.ndarray:
     e = np.exp(row - row.max())
     return e / e.sum()
+
+
+def rownorm_global_select(S_h: np.ndarray, tau: float):
+    """"threshold + global" under the per-query reading of the normalised
+    similarity (reading 11): p_ij = softmax_j(S_i.) / s over the head's whole
+    pool, ranked by p descending (ties: query asc, block asc); keep the
+    shortest prefix whose mass reaches tau (every pair if rounding leaves the
+    total short) -- key design 3's rule on this normalisation.
+
+    Returns (mask [s][N_b] bool, stats) with stats = dict(k, cut_logp, mass):
+    cut_logp = S_ij - logsumexp_j' S_ij' of the last kept pair (its log row
+    softmax), mass = the kept p.
+    Pinned: one query row, and a pool whose rows are all equal, give
+    threshold_select's set; invariant under adding a constant to a row
+    (threshold_select is not); brute-force subset enumeration on tiny pools;
+    minimality.
+    """
+    if not (tau > 0.0) or math.isnan(tau):
+        raise ValueError("tau must be > 0")
+    s, nb = S_h.shape
+    logp = np.empty((s, nb))
+    for i in range(s):
+        m = S_h[i].max()
+        logp[i] = S_h[i] - (m + math.log(np.exp(S_h[i] - m).sum()))
+    flat = logp.reshape(-1)
+    p = np.exp(flat) / s
+    order = np.argsort(-flat, kind="stable")       # descending, ties by flat index
+    c = np.cumsum(p[order])
+    reached = np.flatnonzero(c >= tau)
+    k = int(reached[0]) + 1 if reached.size else flat.size
+    mask = np.zeros(flat.size, dtype=bool)
+    mask[order[:k]] = True
+    stats = dict(k=k, cut_logp=float(flat[order[k - 1]]), mass=float(c[k - 1]))
+    return mask.reshape(S_h.shape), stats
 
 
 def threshold_local_select(S_h: np.ndarray, tau: float):

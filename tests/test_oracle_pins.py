@@ -303,6 +303,63 @@ def test_topk_local_brute_force_and_counts(seed):
     assert mask.tolist() == [[True, True, False, False]] * 2
 
 
+@pytest.mark.parametrize("tau", [0.1, 0.37, 0.8])
+def test_rownorm_global_reduces_to_the_method(tau):
+    rng = np.random.default_rng(11)
+    # one query row: the row softmax is the pool softmax
+    S = rng.standard_normal((1, 9)) * 2.0
+    assert np.array_equal(O.rownorm_global_select(S, tau)[0], O.threshold_select(S, tau)[0])
+    # all rows equal: p_ij = softmax(row)_j / s is the pool softmax too
+    S = np.tile(rng.standard_normal(7) * 2.0, (5, 1))
+    m, st = O.rownorm_global_select(S, tau)
+    m_ref, st_ref = O.threshold_select(S, tau)
+    assert np.array_equal(m, m_ref) and st["k"] == st_ref["k"]
+    assert math.isclose(st["mass"], st_ref["mass"], rel_tol=1e-12)
+
+
+def test_rownorm_global_row_shift_invariance():
+    rng = np.random.default_rng(12)
+    S = rng.standard_normal((6, 5)) * 1.5
+    shifted = S + np.array([8.0, -3.0, 0.0, 1.5, -6.0, 2.0])[:, None]
+    for tau in (0.2, 0.5, 0.9):
+        assert np.array_equal(O.rownorm_global_select(S, tau)[0],
+                              O.rownorm_global_select(shifted, tau)[0])
+    # the method's pool softmax moves with the shift: the two readings differ
+    assert not np.array_equal(O.threshold_select(S, 0.5)[0], O.threshold_select(shifted, 0.5)[0])
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("tau", [0.1, 0.25, 0.5, 0.8])
+def test_rownorm_global_brute_force_on_tiny_pools(seed, tau):
+    rng = np.random.default_rng(700 + seed)
+    s, nb = (4, 3) if seed % 2 else (3, 4)
+    S = rng.standard_normal((s, nb)) * (0.5 + seed)
+    mask, st = O.rownorm_global_select(S, tau)
+    e = np.exp(S - S.max(axis=1, keepdims=True))
+    p = (e / e.sum(axis=1, keepdims=True) / s).reshape(-1)
+    assert math.isclose(p.sum(), 1.0, rel_tol=1e-12)
+    k_bf, best = _brute_force_min_card(p, tau)
+    assert st["k"] == k_bf == mask.sum()
+    assert math.isclose(p[mask.reshape(-1)].sum(), best, rel_tol=1e-12)
+    assert math.isclose(st["mass"], best, rel_tol=1e-12)
+    # minimality: without its least kept pair the mass falls short of tau
+    assert best - p[mask.reshape(-1)].min() < tau
+    # the cut is the last kept pair's log row softmax
+    logp = np.log(p * s).reshape(S.shape)
+    assert math.isclose(st["cut_logp"], logp[mask].min(), rel_tol=1e-12, abs_tol=1e-12)
+
+
+def test_rownorm_global_ties_and_arguments():
+    mask, st = O.rownorm_global_select(np.zeros((3, 2)), 0.5)   # p = 1/6 each
+    assert st["k"] == 3
+    assert mask.reshape(-1).tolist() == [True, True, True, False, False, False]
+    assert O.rownorm_global_select(np.random.default_rng(1).standard_normal((4, 3)), 1.0)[0].all()
+    with pytest.raises(ValueError):
+        O.rownorm_global_select(np.zeros((2, 2)), 0.0)
+    with pytest.raises(ValueError):
+        O.rownorm_global_select(np.zeros((2, 2)), float("nan"))
+
+
 # ---------------------------------------------------------------- attention
 
 def _sdpa(Qh, Kh, Vh, allow, scale):
