@@ -2,8 +2,9 @@
 //
 // Work item n of a head (block j, query tile g of block j's list) covers rows
 // [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
-// rows past the list end are zero.  The attention kernels then fetch query
-// tiles with plain 2-D TMA instead of scattered loads.  One warp per item;
+// rows past the list end are zero.  The backward kernels (dQ pass, dK/dV
+// pass) then fetch query tiles with plain 2-D TMA instead of scattered loads;
+// the forward gathers its own query rows from Q.  One warp per item;
 // 16 lanes x 16 bytes move a 256-byte row, sixteen rows in flight.
 #include "common.cuh"
 #include "pairs.cuh"
