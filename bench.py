@@ -444,27 +444,22 @@ def paper_block_counts(V, w, tensors, stream, warm=2, reps=3):
 
 
 def kernel_traffic(name, w):
-    """DRAM bytes per launch of ``name`` from the committed ncu summary, or None
-    when the kernel's source changed since the counters were taken."""
+    """DRAM bytes per launch of ``name`` from the committed data file of ncu
+    counters (kernel_traffic.json), or None when there is no capture of the
+    kernel or its source changed since the counters were taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "kernel_traffic.md")
-    if not os.path.exists(path):
+    path = os.path.join(ROOT, "kernel_traffic.json")
+    try:
+        with open(path) as f:
+            ent = json.load(f)["kernels"][name]
+    except (OSError, KeyError, ValueError):
         return None
-    for line in open(path):
-        parts = line.split("|")
-        if len(parts) < 6 or parts[1].strip() != name:
-            continue
-        src, digest, nbytes = parts[2].strip(), parts[3].strip(), parts[4].strip()
-        fpath = os.path.join(ROOT, "block_sparse_attention_layer_b200", "csrc", src)
-        if not os.path.exists(fpath):
-            return None
-        if hashlib.sha256(open(fpath, "rb").read()).hexdigest()[:16] != digest:
-            return None
-        try:
-            return float(nbytes)
-        except ValueError:
-            return None
-    return None
+    fpath = os.path.join(ROOT, "block_sparse_attention_layer_b200", "csrc", ent["source"])
+    if not os.path.exists(fpath):
+        return None
+    if hashlib.sha256(open(fpath, "rb").read()).hexdigest()[:16] != ent["sha16"]:
+        return None
+    return float(ent["bytes_per_launch"])
 
 
 def run_e2e(args, layers, host, flops_step, world):

@@ -26,6 +26,15 @@ class VMoBAFunction(torch.autograd.Function):
 
     q, k, v: [s][n_heads][head_dim] contiguous CUDA tensors of the layer's
     dtype.  ``full`` selects every pair (dense attention over the blocks).
+
+    The backward kernels read state the forward left in the layer's buffers
+    (permuted keys and values, pair lists, LSE, the fp32 output copy).  Each
+    call keeps its own selection bitmap and records the layer's forward
+    generation; if another forward ran on the same layer in between (two
+    micro-batches, activation checkpointing, a full-attention call), the
+    backward first restores this call's state by re-running partition, plan
+    and forward on its saved inputs and selection -- the same deterministic
+    kernels, so the restored state is bit-identical -- and then runs.
     """
 
     @staticmethod
@@ -42,13 +51,21 @@ class VMoBAFunction(torch.autograd.Function):
             layer.select(q, k, v, tau, scale)
         out, _ = layer.forward(q, scale)
         ctx.layer, ctx.scale = layer, scale
-        ctx.save_for_backward(q)
+        ctx.generation = layer.generation
+        ctx.save_for_backward(q, k, v, layer.sel.clone())
         return out.clone()
 
     @staticmethod
     def backward(ctx, dout):
-        (q,) = ctx.saved_tensors
-        dq, dk, dv = ctx.layer.backward(q, dout.contiguous(), ctx.scale)
+        q, k, v, sel = ctx.saved_tensors
+        layer = ctx.layer
+        if layer.generation != ctx.generation:
+            # another forward replaced this call's state: rebuild it
+            layer.partition_only(k, v)
+            layer.use_selection(sel)
+            layer.forward(q, ctx.scale)
+            ctx.generation = layer.generation
+        dq, dk, dv = layer.backward(q, dout.contiguous(), ctx.scale)
         return dq.clone(), dk.clone(), dv.clone(), None, None, None, None
 
 

@@ -142,6 +142,7 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
   int rc = make_prob(shape, &P);
   if (rc != VMOBA_OK) return rc;
   if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(blocks)) return VMOBA_ERR_ARG;   // 16-byte vector loads
   if (!(tau > 0.0f) || std::isnan(tau)) return VMOBA_ERR_ARG;
   if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
   WsLayout L;
@@ -162,6 +163,7 @@ int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const fl
   int rc = make_prob(shape, &P);
   if (rc != VMOBA_OK) return rc;
   if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(blocks)) return VMOBA_ERR_ARG;   // 16-byte vector loads
   if (std::isnan(param) || std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
   const bool topk = variant == VMOBA_SELECT_TOPK_GLOBAL || variant == VMOBA_SELECT_TOPK_LOCAL;
   if (variant < VMOBA_SELECT_THRESHOLD_GLOBAL || variant > VMOBA_SELECT_TOPK_LOCAL)
@@ -357,6 +359,7 @@ int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const flo
   int rc = make_prob(shape, &P);
   if (rc != VMOBA_OK) return rc;
   if (!q || !blocks || !sel_bits || !stats) return VMOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(blocks)) return VMOBA_ERR_ARG;   // 16-byte vector loads
   if (!(tau > 0.0f) || std::isnan(tau)) return VMOBA_ERR_ARG;
   if (std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
   const WsLayout L = static_select_layout(P);

@@ -39,6 +39,9 @@ class VMoBALayer:
         self.dq = torch.empty((s, h, d), dtype=dt, device=dev)
         self.dk = torch.empty((s, h, d), dtype=dt, device=dev)
         self.dv = torch.empty((s, h, d), dtype=dt, device=dev)
+        # forwards run so far: lets a caller tell whether the forward state in
+        # the buffers (LSE, fp32 output copy, pair lists) is still its own
+        self.generation = 0
 
     def select(self, q, k, v, tau, scale=0.0):
         sh = self.shape
@@ -67,6 +70,7 @@ class VMoBALayer:
     def forward(self, q, scale=0.0):
         _lib.attn_fwd(self.shape, q, self.k_perm, self.v_perm, self.sel, self.ws, scale,
                       self.out, self.lse)
+        self.generation += 1
         return self.out, self.lse
 
     def backward(self, q, dout, scale=0.0):

@@ -117,10 +117,11 @@ int vmoba_partition(const vmoba_shape* shape, const void* k, const void* v,
  * 3: k = min{k' : cumulative normalised similarity >= tau}; digest 3.3-3.4).
  * q: [s][n_heads][d] (dtype); blocks from vmoba_partition.  tau in (0, 1]
  * (tau >= the pool's total keeps every pair; tau <= 0 or NaN ->
- * VMOBA_ERR_ARG).  scale <= 0 selects 1/sqrt(head_dim).  Writes sel_bits
- * (layout above, fully overwritten) and stats[n_heads] (device).  The pool
- * is ranked by an exact on-device radix select over (score desc, index asc);
- * no host sort and no host round trip. */
+ * VMOBA_ERR_ARG).  scale <= 0 selects 1/sqrt(head_dim).  q and blocks must
+ * be 16-byte aligned (VMOBA_ERR_ARG otherwise: the kernels read them in
+ * 16-byte vectors).  Writes sel_bits (layout above, fully overwritten) and
+ * stats[n_heads] (device).  The pool is ranked by an exact on-device radix
+ * select over (score desc, index asc); no host sort and no host round trip. */
 int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blocks,
                        float tau, float scale, uint32_t* sel_bits,
                        vmoba_head_stats* stats, void* ws, size_t ws_bytes,
@@ -144,7 +145,7 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
  *                                  min(param = k, N_b) blocks.
  * tau must be > 0 (>= 1 keeps everything); k a whole number >= 1 (at or
  * above the pool / N_b keeps everything); anything else, or an unknown
- * variant, -> VMOBA_ERR_ARG.  Same buffers and outputs as
+ * variant, -> VMOBA_ERR_ARG.  Same buffers, alignment rule and outputs as
  * vmoba_score_select.  stats of the local variants: n_selected = pairs,
  * mass = mean kept mass per row under the row softmax, cut_score = NaN
  * (each row has its own cut); the per-row bookkeeping uses workspace that
@@ -174,7 +175,12 @@ int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits,
  * O = 0 and LSE = -inf.  q: [s][n_heads][d]; k_perm, v_perm from
  * vmoba_partition; sel_bits the bitmap the plan was built from.  Writes
  * out [s][n_heads][d] (dtype) and lse [n_heads][s] fp32 (natural log), and
- * keeps an fp32 copy of O in the workspace for vmoba_attn_bwd. */
+ * keeps an fp32 copy of O in the workspace for vmoba_attn_bwd.
+ * Range: the bf16 / head_dim 128 path keeps each (query, block) partial
+ * result as O/l in fp16 (a convex combination of V rows, so |O/l| <= max|V|);
+ * inputs with |V| above 65504, the largest finite fp16, are outside its
+ * contract (their partials overflow to inf).  The fp32 path has no such
+ * limit. */
 int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    const void* v_perm, const uint32_t* sel_bits, void* ws,
                    size_t ws_bytes, float scale, void* out, float* lse,
@@ -202,20 +208,26 @@ int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream);
 /* Selection for callers that cannot allocate device memory.
  * Same contract and results as vmoba_score_select, but the score pool, the
  * radix histograms and the per-head search state live in a fixed 16 MiB
- * array of device memory owned by the library (reserved on every GPU where
- * the library's device code is loaded, until the process exits), so no
- * workspace is passed and nothing is allocated.  Meant for callers such as
- * an engine that has pooled all device memory at start-up and forbids later
+ * array of device memory owned by the library, so no workspace is passed
+ * and nothing is allocated by the call.  Meant for callers such as an
+ * engine that has pooled all device memory at start-up and forbids later
  * cudaMalloc, or a plugin that is given no allocator.  This entry point has
  * no counterpart in the paper: it only changes where scratch memory lives.
+ * - The array is committed on a device when the CUDA runtime loads the
+ *   library's device code there.  With lazy module loading (the CUDA 12
+ *   default) that can happen at this entry point's first call on the
+ *   device, so make one warm-up call on each device before reserving a
+ *   memory pool that leaves no room for 16 MiB; the array then stays
+ *   committed until the process exits.
  * - Problems whose scratch exceeds VMOBA_STATIC_SELECT_SCRATCH_BYTES return
  *   VMOBA_ERR_WORKSPACE without launching anything.  The scratch is the fp32
  *   score pool (4*n_heads*s*N_b bytes) plus about 24.6 KB per head of
  *   histograms and search state; e.g. 4 heads x 2048 tokens x 64 blocks
  *   (2.1 MB) fits, 12 heads x 55296 tokens x 24 blocks (64 MB) does not.
  * - The first call on a device looks up the array's device address on that
- *   device (a CUDA runtime query); make that first call before any stream
- *   capture.
+ *   device (a CUDA runtime query) and caches it; make that first call before
+ *   any stream capture.  cudaDeviceReset invalidates the cached address:
+ *   do not call this entry point on a device after resetting it.
  * - Every call on a device shares the one array: calls that may run at the
  *   same time on the GPU (different streams, other host threads) race and
  *   corrupt each other's results.  Serialise them.

@@ -486,8 +486,3 @@ def io_excess_error(stored: np.ndarray, exact: np.ndarray, dtype: str) -> float:
     err = np.abs(np.asarray(stored, np.float64) - exact) - io_half_ulp(exact, dtype)
     return float(max(err.max(), 0.0)) if err.size else 0.0
 
-
-def selected_pair_density(sel_h: np.ndarray, L: int) -> float:
-    """Fraction of query-key token pairs attended in one head (the pages' "sparsity")."""
-    s = sel_h.shape[0]
-    return float(sel_h.sum()) * L / (s * s)

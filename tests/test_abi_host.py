@@ -97,6 +97,22 @@ def test_null_and_misaligned_pointers_rejected():
                             BAD, None) == -1
 
 
+def test_selection_calls_reject_misaligned_q_and_blocks():
+    """The selection kernels read q and the block means in 16-byte vectors: an
+    element-offset view must come back as VMOBA_ERR_ARG, with nothing launched."""
+    sh = _shape().c()
+    L = V.lib()
+    odd = ctypes.c_void_p(0x100004)
+    ws = 1 << 30
+    for q, b in ((odd, BAD), (BAD, odd)):
+        assert L.vmoba_score_select(ctypes.byref(sh), q, b, 0.5, 0.0, BAD, BAD, BAD, ws,
+                                    None) == -1
+        assert L.vmoba_score_select_variant(ctypes.byref(sh), q, b, 0, 0.5, 0.0, BAD, BAD,
+                                            BAD, ws, None) == -1
+        assert L.vmoba_score_select_static(ctypes.byref(sh), q, b, 0.5, 0.0, BAD, BAD,
+                                           None) == -1
+
+
 @pytest.mark.parametrize("tau", [0.0, -0.5, float("nan")])
 def test_tau_out_of_range_rejected(tau):
     sh = _shape().c()

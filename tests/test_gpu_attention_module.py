@@ -84,3 +84,40 @@ def test_self_attention_module_layers_and_switch():
             assert (y.double().cpu() - y_ref).abs().max().item() <= 0.05
             m.zero_grad()
             x.grad = None
+
+
+def test_two_forwards_before_the_backwards():
+    """Two micro-batches through one layer object: forward A, forward B,
+    backward B, backward A.  Each backward must see its own forward's
+    selection and state, so every gradient equals the one a fresh layer gives
+    for that input alone (the kernels are deterministic: bit-identical)."""
+    mode = 2
+    shape = LayerShape(T, H, W, NH, D, mode, *BOXES[mode], "bf16")
+    scale = 1 / math.sqrt(D)
+    inputs = []
+    for seed in (150, 151):
+        q, k, v = synth.make_qkv(seed, 0, T, H, W, NH, D)
+        dout = synth.make_dout(seed, 0, T * H * W, NH, D)
+        inputs.append([to_device(round_to(x, "bf16"), "bf16") for x in (q, k, v, dout)])
+
+    def grads(layer, q, k, v, dout, full=False):
+        qt, kt, vt = (x.clone().requires_grad_(True) for x in (q, k, v))
+        out = VMoBAFunction.apply(qt, kt, vt, layer, 0.4, full, scale)
+        return out, (qt, kt, vt), dout
+
+    ref = []
+    for q, k, v, dout in inputs:
+        out, leaves, d = grads(VMoBALayer(shape), q, k, v, dout)
+        out.backward(d)
+        ref.append([out.detach().clone()] + [x.grad.clone() for x in leaves])
+
+    shared = VMoBALayer(shape)
+    runs = [grads(shared, *inp) for inp in inputs]       # forward A, forward B
+    for idx in (1, 0):                                    # backward B, backward A
+        out, leaves, d = runs[idx]
+        out.backward(d)
+    torch.cuda.synchronize()
+    for idx, (out, leaves, _) in enumerate(runs):
+        assert torch.equal(out.detach(), ref[idx][0])
+        for x, r in zip(leaves, ref[idx][1:]):
+            assert torch.equal(x.grad, r)

@@ -46,15 +46,24 @@ def test_static_scratch_selection_matches_workspace_selection(wid, mode, tau):
     ref_bits = L.sel.clone()
     ref_stats = _lib.decode_stats(L.stats)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for _ in range(2):
+    for call in range(2):
         bits = torch.full_like(L.sel, -1)
         stats = torch.zeros_like(L.stats)
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        reserved0 = torch.cuda.memory_reserved()
         rc = _lib.lib().vmoba_score_select_static(
             ctypes.byref(sh.c()), ctypes.c_void_p(qd.data_ptr()),
             ctypes.c_void_p(L.blocks.data_ptr()), tau, 0.0, ctypes.c_void_p(bits.data_ptr()),
             ctypes.c_void_p(stats.data_ptr()), stream)
         assert rc == 0
         torch.cuda.synchronize()
+        if call == 1:
+            # after the first call (which may load the module holding the array),
+            # a call takes no device memory from the driver or from torch's pool
+            free1, _ = torch.cuda.mem_get_info()
+            assert free1 == free0
+            assert torch.cuda.memory_reserved() == reserved0
         # the pair set is an integer result: bit-exact
         assert torch.equal(bits, ref_bits)
         st = _lib.decode_stats(stats)
