@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_attn_fwd": (I, [S, P, P, P, P, P, Z, F, P, P, P]),
         "vmoba_attn_bwd": (I, [S, P, P, P, P, P, Z, F, P, P, P, P, P, P, Z, P]),
         "vmoba_get_status": (I, [P, ctypes.POINTER(I), P]),
+        "vmoba_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "vmoba_status_string": (ctypes.c_char_p, [I]),
         "vmoba_last_cuda_error": (ctypes.c_char_p, []),
         "vmoba_kernel_launches": (ctypes.c_ulonglong, []),
@@ -288,6 +289,14 @@ def attn_bwd(shape, q, k_perm, v_perm, sel_bits, ws, scale, lse, dout, dq, dk, d
         ws.numel() * ws.element_size(), float(scale), _ptr(lse), _ptr(dout),
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws_bwd), ws_bwd.numel() * ws_bwd.element_size(),
         _stream(stream)))
+
+
+def debug_set_wait(wait_cycles: int = 0, skip_forward_loads: bool = False) -> None:
+    """Diagnostics for tests of the bounded-wait path (vmoba_debug_set_wait):
+    a spin budget in SM cycles (0 = the default) and whether the forward's
+    key/value producer issues nothing, so that the waits run out."""
+    _check("vmoba_debug_set_wait",
+           lib().vmoba_debug_set_wait(int(wait_cycles), 1 if skip_forward_loads else 0))
 
 
 def get_status(ws, stream=None) -> int:

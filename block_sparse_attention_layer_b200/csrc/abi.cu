@@ -93,8 +93,15 @@ int num_sms() {
 
 }  // namespace
 
+namespace {
+std::atomic<long long> g_wait_budget{0};
+std::atomic<int> g_skip_loads{0};
+}  // namespace
+
 namespace vmoba {
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
+long long debug_wait_budget() { return g_wait_budget.load(); }
+int debug_skip_loads() { return g_skip_loads.load(); }
 }  // namespace vmoba
 
 extern "C" {
@@ -275,6 +282,14 @@ int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream) {
 }
 
 const char* vmoba_last_cuda_error(void) { return cudaGetErrorName(g_last_cuda_error); }
+
+int vmoba_debug_set_wait(long long wait_cycles, int skip_forward_loads) {
+  if (wait_cycles < 0 || (skip_forward_loads != 0 && skip_forward_loads != 1))
+    return VMOBA_ERR_ARG;
+  g_wait_budget.store(wait_cycles);
+  g_skip_loads.store(skip_forward_loads);
+  return VMOBA_OK;
+}
 
 const char* vmoba_status_string(int status) {
   switch (status) {

@@ -86,7 +86,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
              const __grid_constant__ CUtensorMap tm_pd, Prob P, int h, PairsView pv,
              const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
-             int* __restrict__ status) {
+             Watch wt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -139,7 +139,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       bool ok = true;
       for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
         const WorkItem it = decode_item<false>(pv, P, h, n, hint);
-        if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, status, abort);
+        if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, wt, abort);
         if (!ok) break;
         mbar_expect_tx(&bars->qd_full, 2 * kTileB);
         tma_load_2d(sQ, &tm_q, &bars->qd_full, 0, n * kTile);
@@ -149,12 +149,12 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + it.j * P.L + c * kTile;
           const int st = J & 1;
-          if (J >= 2) ok = mbar_wait(&bars->empty_k[st], ((J >> 1) - 1) & 1, status, abort);
+          if (J >= 2) ok = mbar_wait(&bars->empty_k[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_k[st], kTileB);
           tma_load_2d(sK + st * kTileB, &tm_k, &bars->full_k[st], 0, row);
           tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
-          if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, status, abort);
+          if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_v[st], kTileB);
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
@@ -182,10 +182,10 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       // S(J) = Q K^T into S[J & 1]; the chunk's first S of an item waits for its Q / dO
       auto issue_s = [&](int J) -> bool {
         const int st = J & 1, c = J % nch, itl = J / nch;
-        if (c == 0 && !mbar_wait(&bars->qd_full, itl & 1, status, abort)) return false;
-        if (J >= 2 && !mbar_wait(&bars->s_free[st], ((J >> 1) - 1) & 1, status, abort))
+        if (c == 0 && !mbar_wait(&bars->qd_full, itl & 1, wt, abort)) return false;
+        if (J >= 2 && !mbar_wait(&bars->s_free[st], ((J >> 1) - 1) & 1, wt, abort))
           return false;
-        if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, status, abort)) return false;
+        if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, wt, abort)) return false;
         tc_fence_after();
         const uint32_t kb = smem_u32(sK + st * kTileB);
         const uint32_t idc = c == nch - 1 ? idSS_last : idSS;   // N = the chunk's keys
@@ -201,7 +201,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       // dP(J) = dO V^T; overwrites dS(J-1), whose dQ MMA was issued before
       auto issue_dp = [&](int J) -> bool {
         const int st = J & 1, c = J % nch;
-        if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, status, abort)) return false;
+        if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, wt, abort)) return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(sV + st * kTileB);
         const uint32_t idc = c == nch - 1 ? idSS_last : idSS;
@@ -219,8 +219,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       // dQ += dS(J) K(J); dS packed over the dP columns
       auto issue_dq = [&](int J) -> bool {
         const int st = J & 1, c = J % nch, itl = J / nch;
-        if (!mbar_wait(&bars->ds_full, J & 1, status, abort)) return false;
-        if (c == 0 && itl > 0 && !mbar_wait(&bars->dq_free, (itl - 1) & 1, status, abort))
+        if (!mbar_wait(&bars->ds_full, J & 1, wt, abort)) return false;
+        if (c == 0 && itl > 0 && !mbar_wait(&bars->dq_free, (itl - 1) & 1, wt, abort))
           return false;
         tc_fence_after();
         const uint32_t kb = smem_u32(sK + st * kTileB);
@@ -267,7 +267,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       const uint64_t nl2x2 = f32x2(nx_l2, nx_l2), Dx2 = f32x2(nx_d, nx_d);
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, status, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, wt, abort));
         if (!ok) break;
         tc_fence_after();
         const int lim = (c == nch - 1 ? kc_last : kTile) - cb;   // valid columns of this group
@@ -275,7 +275,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           // no key of this chunk in the group's columns: the dQ MMA reads none of them
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->s_free[b]);
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, status, abort));
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, wt, abort));
           if (!ok) break;
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->ds_full);
@@ -298,7 +298,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[b]);    // S[b] may be overwritten now
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, status, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, wt, abort));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -328,7 +328,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       }
       if (!ok) break;
       if (n + G < n_items) fetch(n + G, nx_l2, nx_d);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
@@ -423,7 +423,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                Prob P, int h, PairsView pv, const float* __restrict__ dg,
                const float* __restrict__ l2g, float sl2, float scale,
                __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-               int* __restrict__ status) {
+               Watch wt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -481,7 +481,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       bool ok = true;
       for (int g = 0; g < ng && ok; ++g) {
         const int b = g & 1;
-        if (g >= 2) ok = mbar_wait(&bars->qd_empty[b], ((g >> 1) - 1) & 1, status, abort);
+        if (g >= 2) ok = mbar_wait(&bars->qd_empty[b], ((g >> 1) - 1) & 1, wt, abort);
         if (!ok) break;
         const int qrow = (item0 + g) * kTile;
         mbar_expect_tx(&bars->qd_full[b], 2 * kTileB + 2 * kTile * sizeof(float));
@@ -514,8 +514,8 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           mma_ts(tD, tA + packed_col(kk), desc_sw128(bb + kk * 2048, kHalf, 1024), idAcc,
                  (g > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(&bars->kv_full, 0, status, abort) &&
-                mbar_wait(&bars->qd_full[0], 0, status, abort);
+      bool ok = mbar_wait(&bars->kv_full, 0, wt, abort) &&
+                mbar_wait(&bars->qd_full[0], 0, wt, abort);
       if (ok) {
         tc_fence_after();
         issue_ss(tS, kb, smem_u32(sQ));
@@ -527,11 +527,11 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int b = g & 1;
         const bool more = g + 1 < ng;
         const uint32_t qb = smem_u32(sQ + b * kTileB), ob = smem_u32(sO + b * kTileB);
-        if (!mbar_wait(&bars->p_full, g & 1, status, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->p_full, g & 1, wt, abort)) { ok = false; break; }
         tc_fence_after();
         issue_acc(tV, tS, ob, g);                       // dV += P^T dO
         if (more) {
-          if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, status, abort)) {
+          if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, wt, abort)) {
             ok = false;
             break;
           }
@@ -539,7 +539,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           issue_ss(tS, kb, smem_u32(sQ + (b ^ 1) * kTileB));   // S^T(g+1)
           mma_commit(&bars->st_full);
         }
-        if (!mbar_wait(&bars->ds_full, g & 1, status, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->ds_full, g & 1, wt, abort)) { ok = false; break; }
         tc_fence_after();
         issue_acc(tK, tP, qb, g);                       // dK += dS^T Q
         mma_commit(&bars->qd_empty[b]);
@@ -561,9 +561,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     for (int g = 0; g < ng && ok; ++g) {
       const int b = g & 1;
       // qd_full also covers sL / sD of this tile
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, wt, abort));
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
       const float* NL = sL + b * kTile + cb;
@@ -601,7 +601,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
       // dS^T = P^T (dP^T - D)
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dpt_full, g & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dpt_full, g & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -634,7 +634,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
     // epilogue: dK (x scale) and dV of the tile's keys, original key order
     const bool have = ng > 0 && ok &&
-                      __all_sync(0xffffffffu, mbar_wait(&bars->acc_final, 0, status, abort));
+                      __all_sync(0xffffffffu, mbar_wait(&bars->acc_final, 0, wt, abort));
     if (ng == 0 || have) {
       if (have) tc_fence_after();
       const int pk = key0 + c;
@@ -725,7 +725,7 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
       k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, tpd, P, h, pv, ib.dg,
-                                                        ib.l2g, sl2, status);
+                                                        ib.l2g, sl2, make_watch(status));
     }
     {
       VMOBA_TRACE("k_bwd_dq_merge", st);
@@ -736,7 +736,7 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
       VMOBA_TRACE("k_bwd_dkdv_blk", st);
       k_bwd_dkdv_blk<<<P.Nb * nkt, kThreads, kKvSmem, st>>>(
           tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
-          static_cast<__nv_bfloat16*>(dv), status);
+          static_cast<__nv_bfloat16*>(dv), make_watch(status));
     }
   }
   count_launches(1 + 3 * P.n_h);

@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const __grid_constant__ CUtensorMap tm_po, const __nv_bfloat16* __restrict__ q,
           Prob P, int h, PairsView pv, float sl2, float2* __restrict__ part_ml,
-          int* __restrict__ status) {
+          Watch wt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -169,7 +169,9 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // (wt.skip_loads: diagnostics for the timeout path -- nothing is issued,
+    // so the MMA warp's first wait runs out with no copy in flight)
+    if (lane == 0 && !wt.skip_loads) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int J = 0, hint = 0;
@@ -181,12 +183,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + a.j * P.L + c * kTile;
           const int st = J & 1;
-          if (J >= 2) ok = mbar_wait(&bars->empty_k[st], ((J >> 1) - 1) & 1, status, abort);
+          if (J >= 2) ok = mbar_wait(&bars->empty_k[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_k[st], kTileB);
           tma_load_2d(sK + st * kTileB, &tm_k, &bars->full_k[st], 0, row);
           tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
-          if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, status, abort);
+          if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_v[st], kTileB);
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
@@ -217,7 +219,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         const WorkItem m = t == 0 ? ta : tb;
         if (it_local >= 1)
           ok = __all_sync(0xffffffffu,
-                          mbar_wait(&bars->q_empty[t], (it_local - 1) & 1, status, abort));
+                          mbar_wait(&bars->q_empty[t], (it_local - 1) & 1, wt, abort));
         if (!ok) break;
         if (m.count == 0) {                        // no tile B in this pair
           mbar_arrive(&bars->q_full[t]);
@@ -283,12 +285,12 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         const int nt = b.count > 0 ? 2 : 1;
         {
           const int st = Jk & 1;
-          if (!mbar_wait(&bars->full_k[st], (Jk >> 1) & 1, status, abort)) { ok = false; break; }
+          if (!mbar_wait(&bars->full_k[st], (Jk >> 1) & 1, wt, abort)) { ok = false; break; }
           const uint32_t kb = smem_u32(sK + st * kTileB);
           for (int t = 0; t < 2 && ok; ++t) {
             // every pair passes both tiles' barriers; an absent tile B is
             // released at once
-            if (!mbar_wait(&bars->q_full[t], it_local & 1, status, abort)) { ok = false; break; }
+            if (!mbar_wait(&bars->q_full[t], it_local & 1, wt, abort)) { ok = false; break; }
             tc_fence_after();
             if (t < nt) issue_s(t, kb, nch == 1);
             if (t >= nt || nch == 1) mma_commit(&bars->q_empty[t]);
@@ -299,18 +301,18 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         for (int c = 0; c < nch && ok; ++c) {
           const int Jc = Jk + c, stc = Jc & 1, st1 = (Jc + 1) & 1;
           const bool more = c + 1 < nch;
-          if (!mbar_wait(&bars->full_v[stc], (Jc >> 1) & 1, status, abort)) { ok = false; break; }
+          if (!mbar_wait(&bars->full_v[stc], (Jc >> 1) & 1, wt, abort)) { ok = false; break; }
           uint32_t kb1 = 0;
           for (int t = 0; t < nt && ok; ++t) {
             if (c == 0 && It[t] > 0 &&
-                !mbar_wait(&bars->o_free[t], (It[t] - 1) & 1, status, abort)) { ok = false; break; }
-            if (!mbar_wait(&bars->p_full[t], Js[t] & 1, status, abort)) { ok = false; break; }
+                !mbar_wait(&bars->o_free[t], (It[t] - 1) & 1, wt, abort)) { ok = false; break; }
+            if (!mbar_wait(&bars->p_full[t], Js[t] & 1, wt, abort)) { ok = false; break; }
             ++Js[t];
             tc_fence_after();
             issue_pv(t, smem_u32(sV + stc * kTileB), c);
             if (more) {
               if (t == 0) {
-                if (!mbar_wait(&bars->full_k[st1], ((Jc + 1) >> 1) & 1, status, abort)) {
+                if (!mbar_wait(&bars->full_k[st1], ((Jc + 1) >> 1) & 1, wt, abort)) {
                   ok = false;
                   break;
                 }
@@ -359,7 +361,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       const bool valid = r < cnt;
       float m_run = -INFINITY, l_run = 0.f;
       for (int c = 0; c < nch; ++c, ++Js) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], Js & 1, status, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], Js & 1, wt, abort));
         if (!ok) break;
         tc_fence_after();
         const int kc = c == nch - 1 ? kc_last : kTile;
@@ -372,7 +374,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       if (!ok) break;
       if (p + G < n_pairs) fetch(p + G, nx_n, nx_cnt);
       // epilogue: partial state of (query, block j) into the item's rows
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[t], It & 1, status, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[t], It & 1, wt, abort));
       ++It;
       if (!ok) break;
       tc_fence_after();
@@ -518,7 +520,8 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
     {
       VMOBA_TRACE("k_fwd_blk", st);
       k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(
-          tk, tv, tpo, static_cast<const __nv_bfloat16*>(q), P, h, pv, sl2, part_ml, status);
+          tk, tv, tpo, static_cast<const __nv_bfloat16*>(q), P, h, pv, sl2, part_ml,
+          make_watch(status));
     }
     {
       VMOBA_TRACE("k_fwd_merge", st);

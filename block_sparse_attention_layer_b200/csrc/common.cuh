@@ -148,6 +148,10 @@ class TraceScope {
 // vmoba_kernel_launches).  Every launch wrapper adds what it launched.
 void count_launches(int n);
 
+// Wait settings of vmoba_debug_set_wait (0 = defaults).
+long long debug_wait_budget();
+int debug_skip_loads();
+
 // ---- launch wrappers (one per kernel family; defined in the .cu files) ----
 cudaError_t launch_partition(const Prob& P, const void* k, const void* v, void* kp, void* vp,
                              float* blocks, cudaStream_t st);

@@ -16,7 +16,9 @@ namespace vmoba {
 namespace {
 
 __global__ void k_plan_clear(uint32_t* __restrict__ kt_qt, uint32_t* __restrict__ kt_work,
-                             size_t n_bits_words, size_t n_work) {
+                             size_t n_bits_words, size_t n_work, int* __restrict__ status) {
+  // a new plan starts with a clean device status word
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = VMOBA_OK;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_bits_words;
        i += (size_t)gridDim.x * blockDim.x)
     kt_qt[i] = 0u;
@@ -93,7 +95,7 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   const size_t nw = (size_t)P.n_h * P.n_qt;
   {
     VMOBA_TRACE("k_plan_clear", st);
-    k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw);
+    k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw, ws_ptr<int>(ws, L.status));
   }
   dim3 grid(P.n_qt, P.n_h);
   {

@@ -13,10 +13,19 @@
 namespace vmoba {
 namespace tc {
 
-// Spin budget of every bounded wait (~1 s at 1.9 GHz); on expiry the waiting
-// thread latches VMOBA_ERR_TIMEOUT in the workspace status word and the
-// kernel unwinds without further waits on that barrier.
+// Default spin budget of every bounded wait (~1 s at 1.9 GHz); on expiry the
+// waiting thread latches VMOBA_ERR_TIMEOUT in the workspace status word and
+// the kernel unwinds without further waits on that barrier.
 constexpr long long kWaitCycles = 2000000000LL;
+
+// What a kernel's bounded waits report to: the workspace status word, the
+// spin budget (kWaitCycles unless vmoba_debug_set_wait changed it) and the
+// diagnostics switch that makes the forward's K/V producer issue nothing.
+struct Watch {
+  int* status;
+  long long budget;
+  int skip_loads;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -53,16 +62,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete.  Returns false
-// (after latching the timeout in *status and raising *abort) if the budget
-// runs out or another role already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+// (after latching the timeout in *wt.status and raising *abort) if the
+// budget runs out or another role already gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watch& wt,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      atomicExch(status, (int)VMOBA_ERR_TIMEOUT);
+    if (clock64() - t0 > wt.budget) {
+      atomicExch(wt.status, (int)VMOBA_ERR_TIMEOUT);
       *abort = 1;
       return false;
     }
@@ -317,5 +326,15 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
 // The bf16 case: 64-column x box_rows box.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows);
+
+// Watch of a launch: the status word plus the process-wide wait settings.
+inline tc::Watch make_watch(int* status) {
+  tc::Watch w;
+  w.status = status;
+  const long long b = debug_wait_budget();
+  w.budget = b > 0 ? b : tc::kWaitCycles;
+  w.skip_loads = debug_skip_loads();
+  return w;
+}
 
 }  // namespace vmoba

@@ -202,8 +202,20 @@ int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    cudaStream_t stream);
 
 /* Reads the workspace's device status word (synchronises the stream) into
- * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it. */
+ * *device_status (VMOBA_OK or VMOBA_ERR_TIMEOUT) and clears it.
+ * vmoba_build_plan also clears it (a new plan starts clean). */
 int vmoba_get_status(void* ws, int* device_status, cudaStream_t stream);
+
+/* Diagnostics for tests of the bounded-wait path.  wait_cycles > 0 replaces
+ * the spin budget of every bounded device wait (about one second of SM clock
+ * by default) for attention launches made after the call; 0 restores it.
+ * skip_forward_loads = 1 makes the tensor-core forward's key/value producer
+ * issue no loads, so that its consumers' waits run out with no copy or MMA
+ * in flight and latch VMOBA_ERR_TIMEOUT (the outputs of such a call are
+ * garbage); 0 restores normal operation.  Process-wide, meant for tests:
+ * set it only while no other thread launches.  Returns VMOBA_ERR_ARG for a
+ * negative budget or a flag other than 0 / 1. */
+int vmoba_debug_set_wait(long long wait_cycles, int skip_forward_loads);
 
 /* Selection for callers that cannot allocate device memory.
  * Same contract and results as vmoba_score_select, but the score pool, the

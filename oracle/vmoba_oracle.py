@@ -392,6 +392,52 @@ def attention_bwd_rows(Qh, Kh, Vh, sel_h, blk, scale, rows, dOh_rows):
     return dQ, dK, dV
 
 
+def attention_bwd_block_keys(Qh, Kh, Vh, sel_h, blk, scale, dOh, j):
+    """dK and dV of block j's keys in one head (mask held constant, reading 8).
+
+    Only the queries that selected block j reach its keys.  Each of them
+    needs its LSE_i and O_i over all of its own selected keys; those sums are
+    taken block by block over the blocks the query selected -- the same
+    terms as attention_fwd_rows, grouped by block, with masked keys (whose
+    terms are exactly 0) never formed, so the cost follows the selected pairs
+    instead of s x s.  Two passes: the row maxima, then the sums.  Then for
+    the keys n of block j: P_in = exp(scale q_i.k_n - LSE_i),
+    D_i = dO_i . O_i, dS = P (dO_i.v_n - D_i), dK_n = scale sum_i dS_in q_i,
+    dV_n = sum_i P_in dO_i.
+    Pinned: equals the rows of attention_bwd's dK, dV for every block, and
+    torch autograd through masked SDPA.
+    Returns (keys of block j in original order, dK [len][d], dV [len][d]).
+    """
+    keys_j = np.flatnonzero(blk == j)
+    d = Qh.shape[1]
+    rows = np.flatnonzero(sel_h[:, j])
+    if rows.size == 0:
+        return keys_j, np.zeros((keys_j.size, d)), np.zeros((keys_j.size, d))
+    n_blocks = sel_h.shape[1]
+    members = [np.flatnonzero(blk == b) for b in range(n_blocks)]
+    sub = sel_h[rows]
+    m = np.full(rows.size, -np.inf)
+    for b in range(n_blocks):
+        r = np.flatnonzero(sub[:, b])
+        if r.size:
+            m[r] = np.maximum(m[r], (scale * (Qh[rows[r]] @ Kh[members[b]].T)).max(axis=1))
+    l = np.zeros(rows.size)
+    O = np.zeros((rows.size, d))
+    for b in range(n_blocks):
+        r = np.flatnonzero(sub[:, b])
+        if r.size:
+            P = np.exp(scale * (Qh[rows[r]] @ Kh[members[b]].T) - m[r, None])
+            l[r] += P.sum(axis=1)
+            O[r] += P @ Vh[members[b]]
+    O /= l[:, None]
+    lse = m + np.log(l)
+    P = np.exp(scale * (Qh[rows] @ Kh[keys_j].T) - lse[:, None])
+    dO = dOh[rows]
+    D = np.sum(dO * O, axis=1)
+    dS = P * (dO @ Vh[keys_j].T - D[:, None])
+    return keys_j, scale * (dS.T @ Qh[rows]), P.T @ dO
+
+
 def _row_chunks(s: int, chunk: int):
     for r0 in range(0, s, chunk):
         yield np.arange(r0, min(s, r0 + chunk))

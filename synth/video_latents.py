@@ -78,25 +78,56 @@ def splitmix64_stream(seed: int, n: int, offset: int = 0) -> np.ndarray:
     return z
 
 
+def _uniform01_into(out: np.ndarray, seed: int, offset: int) -> None:
+    """out[i] = uniform number offset + i of the stream (see uniform01)."""
+    z = splitmix64_stream(seed, out.size, offset)
+    np.right_shift(z, np.uint64(11), out=z)
+    out[:] = z
+    out += 1.0
+    out *= 2.0 ** -53
+
+
+# Streams longer than this are produced in chunks on a thread pool (numpy's
+# ufuncs release the GIL); the stream is counter-based, so every element is
+# the same as in one sequential pass.
+_CHUNK = 1 << 22
+
+
+def _chunked(n: int, fn) -> None:
+    starts = range(0, n, _CHUNK)
+    if n <= _CHUNK:
+        fn(0, n)
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+    with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda a: fn(a, min(n, a + _CHUNK)), starts))
+
+
 def uniform01(seed: int, n: int) -> np.ndarray:
     """n uniforms in (0, 1] as float64."""
-    z = splitmix64_stream(seed, n)
-    np.right_shift(z, np.uint64(11), out=z)
-    u = z.astype(np.float64)
-    u += 1.0
-    u *= 2.0 ** -53
+    u = np.empty(n, dtype=np.float64)
+    _chunked(n, lambda a, b: _uniform01_into(u[a:b], seed, a))
     return u
 
 
 def standard_normal(seed: int, n: int) -> np.ndarray:
     """n N(0,1) float64 draws by Box-Muller on uniform pairs."""
-    u = uniform01(seed, 2 * n).reshape(n, 2)
-    r = np.log(u[:, 0])
-    r *= -2.0
-    np.sqrt(r, out=r)
-    c = u[:, 1] * (2.0 * math.pi)
-    np.cos(c, out=c)
-    r *= c
+    r = np.empty(n, dtype=np.float64)
+
+    def part(a: int, b: int) -> None:
+        u = np.empty(2 * (b - a), dtype=np.float64)
+        _uniform01_into(u, seed, 2 * a)
+        u = u.reshape(b - a, 2)
+        x = r[a:b]
+        np.log(u[:, 0], out=x)
+        x *= -2.0
+        np.sqrt(x, out=x)
+        c = u[:, 1] * (2.0 * math.pi)
+        np.cos(c, out=c)
+        x *= c
+
+    _chunked(n, part)
     return r
 
 

@@ -440,6 +440,39 @@ def test_backward_equals_torch_autograd(tau):
         np.testing.assert_allclose(dV[:, h], v.grad.numpy(), rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("tau", [0.05, 0.3, 1.0])
+def test_block_keys_backward_equals_full_backward(tau):
+    """The per-block dK/dV evaluation (sums grouped by block, masked keys never
+    formed) gives attention_bwd's rows for every block, including blocks no
+    query selected (zeros), and torch autograd's key gradients."""
+    Q, K, V, dO, sel, blk, scale = _case(5, tau=tau)
+    dQ, dK, dV = O.attention_bwd(Q, K, V, sel, blk, scale, dO, chunk=13)
+    n_b = sel.shape[2]
+    seen_empty = False
+    for h in range(Q.shape[1]):
+        allow = sel[h][:, blk]
+        safe = allow.copy()
+        safe[~allow.any(1)] = True
+        k = torch.from_numpy(K[:, h].copy()).requires_grad_()
+        v = torch.from_numpy(V[:, h].copy()).requires_grad_()
+        out = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[:, h].copy())[None, None], k[None, None], v[None, None],
+            attn_mask=torch.from_numpy(safe)[None, None], scale=scale)[0, 0]
+        out.backward(torch.from_numpy(dO[:, h] * allow.any(1)[:, None]))
+        for j in range(n_b):
+            keys, dk, dv = O.attention_bwd_block_keys(Q[:, h], K[:, h], V[:, h], sel[h], blk,
+                                                      scale, dO[:, h], j)
+            assert np.array_equal(keys, np.flatnonzero(blk == j))
+            np.testing.assert_allclose(dk, dK[keys, h], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(dv, dV[keys, h], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(dk, k.grad.numpy()[keys], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(dv, v.grad.numpy()[keys], rtol=1e-10, atol=1e-12)
+            if not sel[h][:, j].any():
+                seen_empty = True
+                assert not dk.any() and not dv.any()
+    assert seen_empty or tau > 0.1
+
+
 def test_backward_central_differences():
     Q, K, V, dO, sel, blk, scale = _case(3, grid=(2, 2, 4), box=(1, 2, 2), n_h=1, d=4, tau=0.4)
     dQ, dK, dV = O.attention_bwd(Q, K, V, sel, blk, scale, dO)
