@@ -46,11 +46,21 @@ def parse_args():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the detail runs of the other workloads (256 / 2048 / 32760 "
+                         "tokens) and of the 30-layer 75600-token stack")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile-layer", type=int, default=None,
                     help="profiling case for ncu: run layer L of the workload (its partition "
                          "mode) twice with --heads heads, print per-call times, no timed bench")
     ap.add_argument("--heads", type=int, default=2)
+    ap.add_argument("--shard", choices=("samples", "heads"), default="samples",
+                    help="N > 1: 'samples' runs one synthetic sample per rank (weak "
+                         "scaling); 'heads' splits the 12 heads of one sample across the "
+                         "ranks (strong scaling).  Neither has a collective in the layer.")
+    ap.add_argument("--plan-only", action="store_true",
+                    help="print how the job is split across ranks (heads, samples) and "
+                         "the report's reduction over ranks, without GPU work")
     return ap.parse_args()
 
 
@@ -144,9 +154,59 @@ def rank_sample(rank: int) -> int:
     return rank
 
 
+def rank_work(rank: int, world: int, shard: str, n_heads: int) -> dict:
+    """What one rank runs: its synthetic sample and its heads [h0, h1)."""
+    from block_sparse_attention_layer_b200.sharding import head_range
+    if shard == "heads":
+        h0, h1 = head_range(rank, world, n_heads)
+        return {"sample": 0, "heads": [h0, h1]}
+    return {"sample": rank_sample(rank), "heads": [0, n_heads]}
+
+
+def launch_ranks(n: int, argv, timeout_s: float = 3600.0) -> int:
+    """Run this script once per GPU: re-executes it under torch.distributed.run
+    (one process per rank, rendezvous on 127.0.0.1) and returns the launcher's
+    exit status.  Rank 0 prints the job's JSON line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__), *argv]
+    try:
+        return subprocess.run(cmd, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        return 124
+
+
+def run_plan_only(args, rank, world):
+    """The job's split across ranks on the host (gloo when N > 1): every rank's
+    sample and heads, and the report's max-time / summed-work reduction of one
+    nominal step (rank r: 10 + r ms, 1 + r units of work)."""
+    import torch.distributed as dist
+    import synth
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    mine = rank_work(rank, world, args.shard, w.n_heads)
+    parts = [mine]
+    if world > 1:
+        parts = [None] * world
+        dist.all_gather_object(parts, mine)
+    el, work = reduce_over_ranks(10.0 + rank, 1.0 + rank, "cpu")
+    if rank == 0:
+        print(json.dumps({"plan": parts, "world": world, "shard": args.shard,
+                          "max_ms": el, "work": work}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- inputs
-def host_inputs(sample: int):
-    """bf16 host tensors (pinned) of one synthetic sample: q, k, v, dout."""
+def host_inputs(sample: int, heads=None):
+    """bf16 host tensors (pinned) of one synthetic sample: q, k, v, dout; with
+    ``heads`` = [h0, h1) only those heads, contiguous."""
     import numpy as np
     import torch
 
@@ -155,22 +215,25 @@ def host_inputs(sample: int):
     w = synth.WORKLOADS[WORKLOAD_ID]
     q, k, v = synth.make_qkv(w.wid, sample, w.T, w.H, w.W, w.n_heads, w.head_dim, kind=w.kind)
     dout = synth.make_dout(w.wid, sample, w.s, w.n_heads, w.head_dim)
+    h0, h1 = heads if heads is not None else (0, w.n_heads)
     out = []
     for x in (q, k, v, dout):
+        x = np.ascontiguousarray(x[:, h0:h1])
         t = torch.from_numpy(round_to(x, "bf16").astype(np.float32)).to(torch.bfloat16)
         out.append(t.pin_memory())
     return out
 
 
-def layer_shapes():
+def layer_shapes(n_heads=None):
     import synth
     from block_sparse_attention_layer_b200 import LayerShape
     w = synth.WORKLOADS[WORKLOAD_ID]
+    nh = w.n_heads if n_heads is None else n_heads
     shapes = []
     for l in LAYERS:
         mode = l % 3
         bt, bh, bw = w.boxes[mode]
-        shapes.append(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, bt, bh, bw, "bf16"))
+        shapes.append(LayerShape(w.T, w.H, w.W, nh, w.head_dim, mode, bt, bh, bw, "bf16"))
     return w, shapes
 
 
@@ -187,10 +250,15 @@ def run_ours(args, rank, world, local):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    w, shapes = layer_shapes()
+    import synth
+    job = rank_work(rank, world, args.shard, synth.WORKLOADS[WORKLOAD_ID].n_heads)
+    h0, h1 = job["heads"]
+    if h1 <= h0:
+        raise SystemExit(f"rank {rank}: no head to run (more ranks than heads)")
+    w, shapes = layer_shapes(n_heads=h1 - h0)
     peaks = load_peaks()
     t0 = time.time()
-    hq, hk, hv, hdo = host_inputs(sample=rank_sample(rank))
+    hq, hk, hv, hdo = host_inputs(sample=job["sample"], heads=(h0, h1))
     gen_s = time.time() - t0
     q, k, v, dout = (x.cuda(non_blocking=False) for x in (hq, hk, hv, hdo))
     layers = [VMoBALayer(sh) for sh in shapes]
@@ -265,6 +333,7 @@ def run_ours(args, rank, world, local):
     # the headline: density and ms per layer beside the main workload's
     second = paper_block_counts(V, w, (q, k, v, dout), stream)
     variants = selection_variants(V, w, layers, q, density, stream)
+    others = other_configs(V, stream) if not args.no_sweeps else None
 
     # per-call device times (ms, summed over layers, averaged over steps)
     call_ms = {c: 0.0 for c in CALLS}
@@ -282,7 +351,7 @@ def run_ours(args, rank, world, local):
 
     # roofline of the dominant kernel (by device time over the timed region):
     # algorithmic work per launch summed over the step / its traced time
-    s, nh = w.s, w.n_heads
+    s, nh = w.s, h1 - h0
     flops_per_pair = {"k_fwd_blk": 4 * d, "k_bwd_dq_blk": 6 * d, "k_bwd_dkdv_blk": 8 * d}
     tot_pairs = sum(pairs)
     kern = {}
@@ -315,6 +384,11 @@ def run_ours(args, rank, world, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, layers, (hq, hk, hv, hdo), flops_step, world)
+    sweep = None
+    if not args.no_sweeps:
+        del layers
+        torch.cuda.empty_cache()
+        sweep = stack_sweep(V, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -324,15 +398,20 @@ def run_ours(args, rank, world, local):
         line = {
             "metric": METRIC, "value": round(value, 4), "unit": "TFLOP/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(elapsed_max / K, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded smooth+noise video-latent Q/K/V, dO ~ N(0,1))",
             "config": {
                 "workload": "train-55296tok: T24xH36xW64 latent, 12 heads x 128, bf16, "
                             "tau 0.25, layers l=0,1,2 (1D 1-frame / 2D 6x8 / 3D 4x6x8 blocks), "
-                            "fwd+bwd, batch 1 per GPU",
-                "global_batch": world, "seq_len": w.s, "parallelism": f"dp{world}",
+                            "fwd+bwd, batch 1 "
+                            + ("split by heads across GPUs" if args.shard == "heads"
+                               else "per GPU"),
+                "global_batch": 1 if args.shard == "heads" else world, "seq_len": w.s,
+                "parallelism": f"heads{world}" if args.shard == "heads" else f"dp{world}",
                 "l2": "inputs larger than L2 (170 MB per tensor), no flush"},
-            "ms_per_layer": round(elapsed_max / K / len(layers), 4),
+            "ms_per_layer": round(elapsed_max / K / len(shapes), 4),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -342,6 +421,8 @@ def run_ours(args, rank, world, local):
                 "call_ms_per_step": {c: round(call_ms[c], 4) for c in CALLS},
                 "kernel_ms_per_layer": kern_layer,
                 "blocks_8_48_72": second,
+                "other_configs": others,
+                "stack_75600tok_30_layers": sweep,
                 "selection_variants": variants,
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
                                   for i, l in enumerate(LAYERS)},
@@ -397,6 +478,135 @@ def selection_variants(V, w, layers, q, density, stream, warm=1, reps=3):
             gbs_l.append(round(metrics.select_bytes(sh.s, sh.n_heads, nb) / (ms * 1e-3) / 1e9, 1))
         res[name] = {"ms_per_layer": ms_l, "pair_density": dens_l, "select_GBps": gbs_l}
     return res
+
+
+def _time_layer_calls(V, L, q, k, v, tau, dout, stream, warm=1, reps=3):
+    """Device ms of one layer's calls (select = partition + score/select +
+    plan; fwd; bwd if dout is given), averaged over ``reps`` after ``warm``."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    acc = [0.0, 0.0, 0.0]
+    for it in range(warm + reps):
+        ev[0].record(stream)
+        V.partition(L.shape, k, v, L.k_perm, L.v_perm, L.blocks)
+        V.score_select(L.shape, q, L.blocks, tau, 0.0, L.sel, L.stats, L.ws)
+        V.build_plan(L.shape, L.sel, L.ws)
+        ev[1].record(stream)
+        L.forward(q)
+        ev[2].record(stream)
+        if dout is not None:
+            L.backward(q, dout)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        if it >= warm:
+            for i in range(3):
+                acc[i] += ev[i].elapsed_time(ev[i + 1]) / reps
+    return acc
+
+
+def _layer_record(V, L, ms, d, backward):
+    """Density, ms and throughputs of one timed layer (see _time_layer_calls)."""
+    from block_sparse_attention_layer_b200 import metrics
+    sh = L.shape
+    st = L.head_stats()
+    pairs = metrics.token_pairs_from_stats(st["n_selected"], L.block_len)
+    nb = L.n_blocks
+    ms_sel, ms_fwd, ms_bwd = ms
+    fl = metrics.attention_flops(pairs, d, True, backward)
+    ms_attn = ms_fwd + (ms_bwd if backward else 0.0)
+    esize = 2 if sh.dtype == "bf16" else 4
+    return {"density": round(pairs / (sh.s * sh.s * sh.n_heads), 5),
+            "ms_layer": round(ms_sel + ms_attn, 4), "ms_select": round(ms_sel, 4),
+            "ms_fwd": round(ms_fwd, 4), "ms_bwd": round(ms_bwd, 4) if backward else None,
+            "attn_tflops": round(fl / (ms_attn * 1e-3) / 1e12, 2) if ms_attn > 0 else None,
+            "select_GBps_incl_partition_plan": round(
+                (metrics.partition_bytes(sh.s, sh.n_heads, d, esize, nb)
+                 + metrics.select_bytes(sh.s, sh.n_heads, nb)) / (ms_sel * 1e-3) / 1e9, 1)}
+
+
+def other_configs(V, stream):
+    """The small and inference workloads: 256 tokens (fp32, 2 x 64, forward),
+    2048 tokens (bf16, 4 x 64, tau 0.25 / 0.5 / 0.75, forward + backward) and
+    32760 tokens (Wan-1.3B shape, 12 x 128, tau 0.25, forward): every
+    partition mode (layers l = 0, 1, 2), device ms per call and per layer,
+    selected-pair density, attention TFLOP/s on selected pairs."""
+    import numpy as np
+    import torch
+
+    import synth
+    from synth import torch_latents as TL
+    from synth.video_latents import round_to
+    from block_sparse_attention_layer_b200 import LayerShape
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+    res = {}
+    for wid in (1, 2, 3):
+        w = synth.WORKLOADS[wid]
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        rows = []
+        for mode in range(3):
+            if wid == 3:
+                q, k, v = TL.make_qkv(w.wid, mode, w.T, w.H, w.W, w.n_heads, w.head_dim,
+                                      kind=w.kind, dtype=tdt)
+                dout = None
+            else:
+                arrs = synth.make_qkv(w.wid, mode, w.T, w.H, w.W, w.n_heads, w.head_dim,
+                                      kind=w.kind)
+                arrs = list(arrs) + [synth.make_dout(w.wid, mode, w.s, w.n_heads, w.head_dim)]
+                q, k, v, dout = (torch.from_numpy(round_to(x, w.dtype).astype(np.float32))
+                                 .to(tdt).cuda() for x in arrs)
+                if not w.backward:
+                    dout = None
+            sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *w.boxes[mode],
+                            w.dtype)
+            L = VMoBALayer(sh)
+            for tau in w.taus:
+                ms = _time_layer_calls(V, L, q, k, v, tau, dout, stream)
+                rec = _layer_record(V, L, ms, w.head_dim, dout is not None)
+                rec.update(mode=mode, tau=tau, n_blocks=L.n_blocks)
+                rows.append(rec)
+            del L
+        res[w.name] = rows
+    torch.cuda.empty_cache()
+    return res
+
+
+def stack_sweep(V, stream):
+    """The 30-layer stack at 75600 tokens (T21 x H45 x W80, 12 heads of 128,
+    per-head Q/K gains c_h ~ U[0.5, 2] drawn per layer; layer l partitions by
+    mode l mod 3) at tau 0.1, 0.25 and 0.5, forward + backward: selected-pair
+    density and device ms of every layer.  Inputs are drawn on the device
+    with the generator's torch form (same recipe and seeds as the host one)."""
+    import torch
+
+    import synth
+    from synth import torch_latents as TL
+    from block_sparse_attention_layer_b200 import LayerShape
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+    w = synth.WORKLOADS[5]
+    layers = [VMoBALayer(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, m, *w.boxes[m],
+                                    "bf16")) for m in range(3)]
+    out = {f"tau_{tau}": {"density": [], "ms_layer": [], "attn_tflops": []} for tau in w.taus}
+    t0 = time.time()
+    for layer in range(w.layers):
+        L = layers[layer % 3]
+        q, k, v = TL.make_qkv(w.wid, layer, w.T, w.H, w.W, w.n_heads, w.head_dim,
+                              kind=w.kind, head_gain=w.head_gain)
+        dout = TL.make_dout(w.wid, layer, w.s, w.n_heads, w.head_dim)
+        for tau in w.taus:
+            ms = _time_layer_calls(V, L, q, k, v, tau, dout, stream, warm=1, reps=1)
+            rec = _layer_record(V, L, ms, w.head_dim, True)
+            o = out[f"tau_{tau}"]
+            o["density"].append(rec["density"])
+            o["ms_layer"].append(rec["ms_layer"])
+            o["attn_tflops"].append(rec["attn_tflops"])
+        del q, k, v, dout
+    for o in out.values():
+        o["mean_density"] = round(sum(o["density"]) / len(o["density"]), 5)
+        o["mean_ms_layer"] = round(sum(o["ms_layer"]) / len(o["ms_layer"]), 4)
+    out["wall_s"] = round(time.time() - t0, 1)
+    del layers
+    torch.cuda.empty_cache()
+    return out
 
 
 def paper_block_counts(V, w, tensors, stream, warm=2, reps=3):
@@ -527,9 +737,10 @@ def run_e2e(args, layers, host, flops_step, world):
     b.record(comp)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
-    ms, _ = reduce_over_ranks(ms, 0.0, "cuda")
+    # the job's time is the slowest rank's; its work is every rank's own
+    ms, flops = reduce_over_ranks(ms, flops_step * K, "cuda")
     nbytes = hq.numel() * hq.element_size()
-    return {"value": round(flops_step * K * world / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
             "h2d_bytes_per_step": 4 * nbytes * len(layers),
             "d2h_bytes_per_step": 4 * nbytes * len(layers),
             "ms_per_step": round(ms / K, 3),
@@ -678,7 +889,13 @@ def main():
     if args.profile_layer is not None:
         run_profile_case(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not started by a launcher: start one process per GPU ourselves
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
     rank, world, local = dist_env()
+    if args.plan_only:
+        run_plan_only(args, rank, world)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -3,7 +3,8 @@
 The compute path is libvmoba.so (CUDA, sm_100a) behind the C ABI declared in
 include/vmoba.h; this package is its Python binding (``_lib``), a buffer-
 owning per-layer driver (``layer``), the in-tree build script (``build``) and
-the bench's FLOP-count convention (``metrics``).  Importing the package does
+the bench's FLOP-count convention (``metrics``) and the split of a layer's
+heads across GPUs (``sharding``).  Importing the package does
 not load the library; the first ABI call does, and raises if it is missing.
 """
 from ._lib import (  # noqa: F401
