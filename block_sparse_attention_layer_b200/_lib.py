@@ -223,7 +223,8 @@ def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None)
 
 # selection variants of the ablation (include/vmoba.h: vmoba_score_select_variant)
 SELECT_THRESHOLD_GLOBAL, SELECT_TOPK_GLOBAL, SELECT_THRESHOLD_LOCAL, SELECT_TOPK_LOCAL = 0, 1, 2, 3
-SELECT_VARIANTS = {"threshold_global": 0, "topk_global": 1, "threshold_local": 2, "topk_local": 3}
+SELECT_VARIANTS = {"threshold_global": 0, "topk_global": 1, "threshold_local": 2, "topk_local": 3,
+                   "rownorm_global": 4}
 
 
 def score_select_variant(shape, q, blocks, variant, param, scale, sel_bits, stats, ws,

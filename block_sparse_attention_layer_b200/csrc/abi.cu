@@ -159,7 +159,8 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
   const float tau_dev = tau >= 1.0f ? 2.0f : tau;
   drop_stale_error();
   return cuda_status(
-      launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
+      launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, num_sms(),
+                          stream));
 }
 
 int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const float* blocks,
@@ -173,7 +174,7 @@ int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const fl
   if (!aligned16(q) || !aligned16(blocks)) return VMOBA_ERR_ARG;   // 16-byte vector loads
   if (std::isnan(param) || std::isnan(scale) || std::isinf(scale)) return VMOBA_ERR_ARG;
   const bool topk = variant == VMOBA_SELECT_TOPK_GLOBAL || variant == VMOBA_SELECT_TOPK_LOCAL;
-  if (variant < VMOBA_SELECT_THRESHOLD_GLOBAL || variant > VMOBA_SELECT_TOPK_LOCAL)
+  if (variant < VMOBA_SELECT_THRESHOLD_GLOBAL || variant > VMOBA_SELECT_ROWNORM_GLOBAL)
     return VMOBA_ERR_ARG;
   if (topk ? !(param >= 1.0 && param == std::floor(param) && param < 9.0e15) : !(param > 0.0))
     return VMOBA_ERR_ARG;
@@ -185,15 +186,21 @@ int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const fl
   switch (variant) {
     case VMOBA_SELECT_THRESHOLD_GLOBAL: {
       const float tau_dev = param >= 1.0 ? 2.0f : (float)param;
-      return cuda_status(
-          launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws, L, stream));
+      return cuda_status(launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws,
+                                             L, num_sms(), stream));
+    }
+    case VMOBA_SELECT_ROWNORM_GLOBAL: {
+      const float tau_dev = param >= 1.0 ? 2.0f : (float)param;
+      return cuda_status(launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, ws,
+                                             L, num_sms(), stream, 0, 0.0, true));
     }
     case VMOBA_SELECT_TOPK_GLOBAL:
       // k at or above the pool keeps every pair (the walk can never reach pool + 1)
       return cuda_status(launch_score_select(P, q, blocks, 0.0f, scale, sel_bits, stats, ws, L,
-                                             stream, 1, param >= pool ? pool + 1.0 : param));
+                                             num_sms(), stream, 1,
+                                             param >= pool ? pool + 1.0 : param));
     default: {
-      cudaError_t e = launch_score_pool(P, q, blocks, scale, ws, L, stream);
+      cudaError_t e = launch_score_pool(P, q, blocks, scale, ws, L, num_sms(), stream);
       if (e != cudaSuccess) return cuda_status(e);
       const double p = topk ? param : (param >= 1.0 ? 2.0 : param);
       return cuda_status(launch_select_local(P, topk ? 1 : 0, p, sel_bits, stats, ws, L, stream));
@@ -350,15 +357,22 @@ int static_scratch(void** out) {
   return VMOBA_OK;
 }
 
-// The selection's part of the workspace layout, packed into the static array.
+// The selection's part of the workspace layout, packed into the static array:
+// the device status word, the search state and histograms, and the bf16
+// split of the block means (bf16 inputs; their pool is recomputed, never
+// stored) or the fp32 score pool (fp32 inputs).
 WsLayout static_select_layout(const Prob& P) {
   WsLayout w{};
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  w.status = take(256);
   w.sel_state = take(sizeof(SelState) * P.n_h);
   w.hist_count = take(sizeof(uint32_t) * kHistBins * P.n_h);
   w.hist_mass = take(sizeof(double) * kHistBins * P.n_h);
-  w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
+  if (P.dtype == VMOBA_BF16)
+    w.bsplit = take(sel_split_bytes(P));
+  else
+    w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
   w.total = off;
   return w;
 }
@@ -384,10 +398,11 @@ int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const flo
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   const float tau_dev = tau >= 1.0f ? 2.0f : tau;
   // the first kernel of the selection clears the histograms and the search
-  // state; the score pool is fully overwritten before it is read
+  // state; the split of B (or, for fp32 inputs, the score pool) is fully
+  // overwritten before it is read
   drop_stale_error();
-  return cuda_status(
-      launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, scratch, L, stream));
+  return cuda_status(launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, scratch,
+                                         L, num_sms(), stream));
 }
 
 }  // extern "C"

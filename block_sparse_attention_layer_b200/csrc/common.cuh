@@ -9,6 +9,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -90,6 +91,7 @@ struct SelState {
 // Byte offsets inside the caller's workspace (all 256-byte aligned).
 struct WsLayout {
   size_t status, sel_state, hist_count, hist_mass, scores;
+  size_t bsplit;         // bf16 hi / lo split of the block means (tensor-core score passes)
   size_t qt_kt_bits, qt_work, kt_qt_bits, kt_work;
   size_t o32;            // fp32 copy of the forward output, [s][n_h][d]
   size_t pairs;          // pair lists of the selection (pairs.cu)
@@ -102,6 +104,10 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t pairs_ws_bytes(const Prob& P);
 size_t blk_partial_bytes(const Prob& P);
+// Rows per head and half of the bf16 split of the block means (N_b rounded
+// up to 128) and its bytes ([n_h][hi, lo][rows][d]).
+int sel_split_rows(const Prob& P);
+size_t sel_split_bytes(const Prob& P);
 size_t item_bufs_bytes(const Prob& P);
 // bf16 with head_dim 128 runs the block-major tensor-core kernels; fp32 I/O
 // (whose 1e-4 bar rules out TF32) and head_dim 64 run on the CUDA cores.
@@ -116,6 +122,7 @@ inline WsLayout ws_layout(const Prob& P) {
   w.hist_count = take(sizeof(uint32_t) * kHistBins * P.n_h);
   w.hist_mass = take(sizeof(double) * kHistBins * P.n_h);
   w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
+  w.bsplit = take(sel_split_bytes(P));
   w.qt_kt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
   w.qt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
   w.kt_qt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
@@ -156,14 +163,34 @@ int debug_skip_loads();
 cudaError_t launch_partition(const Prob& P, const void* k, const void* v, void* kp, void* vp,
                              float* blocks, cudaStream_t st);
 // by_count = 0: the method's mass threshold tau; by_count = 1: the kcount
-// highest pairs of each head's pool (top-k global), same ranking and ties.
+// highest pairs of each head's pool (top-k global), same ranking and ties;
+// rownorm: the pool normalised per query row first (a selection variant).
 cudaError_t launch_score_select(const Prob& P, const void* q, const float* blocks, float tau,
                                 float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
-                                const WsLayout& L, cudaStream_t st, int by_count = 0,
-                                double kcount = 0.0);
+                                const WsLayout& L, int num_sms, cudaStream_t st,
+                                int by_count = 0, double kcount = 0.0, bool rownorm = false);
+// What the tensor-core score passes (score_tc.cu) need from the selection
+// around them: the search state and histograms, the outputs, and the
+// one-warp digit walks to run after each histogram pass.
+struct SelPassOps {
+  SelState* st;
+  uint32_t* hc;
+  double* hm;
+  uint32_t* sel;
+  float* pool;
+  void* bsplit;
+  int* status;
+  int num_sms;
+  bool pool_only;       // one pass writing S to `pool`, nothing else
+  std::function<cudaError_t(int, cudaStream_t)> scan, tie_scan;
+};
+// bf16 Q: the score passes of a selection (max, three histogram passes with
+// their scans, the tie passes, the bitmap) or, with pool_only, the pool.
+cudaError_t launch_score_passes_tc(const Prob& P, const void* q, const float* blocks,
+                                   float scale, const SelPassOps& ops, cudaStream_t stream);
 // The score pool S = scale q b^T of every head into the workspace.
 cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks, float scale,
-                              void* ws, const WsLayout& L, cudaStream_t st);
+                              void* ws, const WsLayout& L, int num_sms, cudaStream_t st);
 // Per-query-row selection (threshold local / top-k local); scores in the
 // workspace pool, per-row scratch in the forward-output copy.
 cudaError_t launch_select_local(const Prob& P, int topk, double param, uint32_t* sel,

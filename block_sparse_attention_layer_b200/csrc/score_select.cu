@@ -14,8 +14,13 @@
 // Exact ties at the cut are ranked by flat index i*N_b + j (ascending) with
 // three more count-only radix passes that return at once unless needed.
 //
-// Kernels, in stream order: init -> score -> {hist, scan} x 3 ->
-// {tie_hist, tie_scan} x 3 -> emit (bitmap) -> stats.
+// bf16 inputs (every workload of the method) run the passes on the tensor
+// cores over a pool recomputed tile by tile (score_tc.cu): init -> split of
+// B -> max -> {hist, scan} x 3 -> {tie, tie_scan} x 3 -> emit -> stats, with
+// no pool in memory.  fp32 inputs (whose 1e-4 output bar the bf16 split of
+// Q could not meet) compute the pool once with fp32 FMAs on the CUDA cores
+// and read it in each pass: init -> score -> {hist, scan} x 3 ->
+// {tie_hist, tie_scan} x 3 -> emit -> stats.
 //
 // The ablation's "topk + global" variant (VMoBA notes, ablation table) runs
 // the same passes with the digit walk counting pairs instead of mass: the
@@ -36,12 +41,6 @@ __device__ __forceinline__ float word_elem(const uint32_t* w, int k);
 template <>
 __device__ __forceinline__ float word_elem<float>(const uint32_t* w, int k) {
   return __uint_as_float(w[k]);
-}
-template <>
-__device__ __forceinline__ float word_elem<__nv_bfloat16>(const uint32_t* w, int k) {
-  // bf16 is the top half of an fp32: element 2m in the low 16 bits of word m
-  const uint32_t x = w[k >> 1];
-  return __uint_as_float((k & 1) ? (x & 0xFFFF0000u) : (x << 16));
 }
 
 __global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
@@ -421,6 +420,40 @@ k_emit(Prob P, const float* __restrict__ S, const SelState* __restrict__ st,
   }
 }
 
+// The per-query reading of "normalised similarity" (a selection variant):
+// each row of the stored pool becomes its log softmax over the row's N_b
+// blocks, S_ij <- S_ij - log sum_j' exp S_ij', in place, and the per-head max
+// of the result is recorded.  Ranking the head's pool by this value is
+// ranking it by p_ij = softmax_j(S_i.) / s, and exp(S' - max S') is p up to
+// one factor per head, so the method's passes below then apply the
+// cumulative rule to p unchanged.  One warp per row.
+__global__ void __launch_bounds__(256)
+k_rownorm(Prob P, float* __restrict__ S, SelState* __restrict__ st) {
+  const int lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // h * s + i
+  if (row >= (size_t)P.n_h * P.s) return;
+  const int h = (int)(row / (size_t)P.s);
+  float* r = S + row * P.Nb;
+  float m = -INFINITY;
+  for (int j = lane; j < P.Nb; j += 32) m = fmaxf(m, r[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float z = 0.f;
+  for (int j = lane; j < P.Nb; j += 32) z += expf(r[j] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float lse = m + logf(z);
+  float mx = -INFINITY;
+  for (int j = lane; j < P.Nb; j += 32) {
+    const float v = r[j] - lse;
+    r[j] = v;
+    mx = fmaxf(mx, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) atomicMax(&st[h].max_key, f2key(mx));
+}
+
 __global__ void k_stats(Prob P, const SelState* __restrict__ st, vmoba_head_stats* __restrict__ out) {
   const int h = threadIdx.x;
   if (h >= P.n_h) return;
@@ -451,34 +484,40 @@ cudaError_t launch_score(const Prob& P, const void* q, const float* B, float sca
 }  // namespace
 
 cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks, float scale,
-                              void* ws, const WsLayout& L, cudaStream_t stream) {
+                              void* ws, const WsLayout& L, int num_sms, cudaStream_t stream) {
   SelState* st = ws_ptr<SelState>(ws, L.sel_state);
   {
     VMOBA_TRACE("k_init", stream);
     k_init<<<64, 256, 0, stream>>>(st, ws_ptr<uint32_t>(ws, L.hist_count),
                                    ws_ptr<double>(ws, L.hist_mass), P.n_h);
   }
+  count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   float* S = ws_ptr<float>(ws, L.scores);
-  if (P.dtype == VMOBA_BF16)
-    e = (P.d == 128) ? launch_score<__nv_bfloat16, 128>(P, q, blocks, scale, S, st, stream)
-                     : launch_score<__nv_bfloat16, 64>(P, q, blocks, scale, S, st, stream);
-  else
-    e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
-                     : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
-  count_launches(2);
+  if (P.dtype == VMOBA_BF16) {
+    SelPassOps ops{};
+    ops.st = st;
+    ops.pool = S;
+    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
+    ops.status = ws_ptr<int>(ws, L.status);
+    ops.num_sms = num_sms;
+    ops.pool_only = true;
+    return launch_score_passes_tc(P, q, blocks, scale, ops, stream);
+  }
+  e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
+                   : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
+  count_launches(1);
   return e;
 }
 
 cudaError_t launch_score_select(const Prob& P, const void* q, const float* blocks, float tau,
                                 float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
-                                const WsLayout& L, cudaStream_t stream, int by_count,
-                                double kcount) {
+                                const WsLayout& L, int num_sms, cudaStream_t stream,
+                                int by_count, double kcount, bool rownorm) {
   SelState* st = ws_ptr<SelState>(ws, L.sel_state);
   uint32_t* hc = ws_ptr<uint32_t>(ws, L.hist_count);
   double* hm = ws_ptr<double>(ws, L.hist_mass);
-  float* S = ws_ptr<float>(ws, L.scores);
 
   {
     VMOBA_TRACE("k_init", stream);
@@ -486,74 +525,101 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (P.dtype == VMOBA_BF16)
-    e = (P.d == 128) ? launch_score<__nv_bfloat16, 128>(P, q, blocks, scale, S, st, stream)
-                     : launch_score<__nv_bfloat16, 64>(P, q, blocks, scale, S, st, stream);
-  else
-    e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
-                     : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
-  if (e != cudaSuccess) return e;
+  int launches = 1;
+  auto scan = [&](int pass, cudaStream_t s) -> cudaError_t {
+    VMOBA_TRACE("k_scan", s);
+    if (pass == 0) k_scan<0><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
+    if (pass == 1) k_scan<1><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
+    if (pass == 2) k_scan<2><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
+    ++launches;
+    return cudaGetLastError();
+  };
+  auto tie_scan = [&](int pass, cudaStream_t s) -> cudaError_t {
+    VMOBA_TRACE("k_tie_scan", s);
+    if (pass == 0) k_tie_scan<0><<<P.n_h, 32, 0, s>>>(st, hc);
+    if (pass == 1) k_tie_scan<1><<<P.n_h, 32, 0, s>>>(st, hc);
+    if (pass == 2) k_tie_scan<2><<<P.n_h, 32, 0, s>>>(st, hc);
+    ++launches;
+    return cudaGetLastError();
+  };
 
-  const size_t pool = (size_t)P.s * P.Nb;
-  dim3 hgrid((unsigned)((pool + kHistChunk - 1) / kHistChunk), P.n_h);
-  {
-    VMOBA_TRACE("k_hist", stream);
-    k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+  if (P.dtype == VMOBA_BF16 && rownorm) {
+    // the per-query normalisation needs whole rows: the pool is written once
+    // by the tensor cores and the passes read it (the fp32 path below)
+    SelPassOps ops{};
+    ops.st = st;
+    ops.pool = ws_ptr<float>(ws, L.scores);
+    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
+    ops.status = ws_ptr<int>(ws, L.status);
+    ops.num_sms = num_sms;
+    ops.pool_only = true;
+    e = launch_score_passes_tc(P, q, blocks, scale, ops, stream);
+    if (e != cudaSuccess) return e;
   }
-  {
-    VMOBA_TRACE("k_scan", stream);
-    k_scan<0><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
-  }
-  {
-    VMOBA_TRACE("k_hist", stream);
-    k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-  }
-  {
-    VMOBA_TRACE("k_scan", stream);
-    k_scan<1><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
-  }
-  {
-    VMOBA_TRACE("k_hist", stream);
-    k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-  }
-  {
-    VMOBA_TRACE("k_scan", stream);
-    k_scan<2><<<P.n_h, 32, 0, stream>>>(P, st, hc, hm, tau, by_count, kcount);
-  }
-  {
-    VMOBA_TRACE("k_tie_hist", stream);
-    k_tie_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  }
-  {
-    VMOBA_TRACE("k_tie_scan", stream);
-    k_tie_scan<0><<<P.n_h, 32, 0, stream>>>(st, hc);
-  }
-  {
-    VMOBA_TRACE("k_tie_hist", stream);
-    k_tie_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  }
-  {
-    VMOBA_TRACE("k_tie_scan", stream);
-    k_tie_scan<1><<<P.n_h, 32, 0, stream>>>(st, hc);
-  }
-  {
-    VMOBA_TRACE("k_tie_hist", stream);
-    k_tie_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
-  }
-  {
-    VMOBA_TRACE("k_tie_scan", stream);
-    k_tie_scan<2><<<P.n_h, 32, 0, stream>>>(st, hc);
-  }
-  dim3 egrid((P.s + 31) / 32, P.n_h);
-  {
-    VMOBA_TRACE("k_emit", stream);
-    k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
+  if (P.dtype == VMOBA_BF16 && !rownorm) {
+    // tensor-core passes over the recomputed pool (score_tc.cu)
+    SelPassOps ops{};
+    ops.st = st;
+    ops.hc = hc;
+    ops.hm = hm;
+    ops.sel = sel;
+    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
+    ops.status = ws_ptr<int>(ws, L.status);
+    ops.num_sms = num_sms;
+    ops.scan = scan;
+    ops.tie_scan = tie_scan;
+    e = launch_score_passes_tc(P, q, blocks, scale, ops, stream);
+    if (e != cudaSuccess) return e;
+  } else {
+    // fp32 I/O: the pool is computed once with fp32 FMAs and read by each
+    // pass (bf16 with the per-query normalisation: written above)
+    float* S = ws_ptr<float>(ws, L.scores);
+    if (P.dtype != VMOBA_BF16) {
+      e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
+                       : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
+      if (e != cudaSuccess) return e;
+      ++launches;
+    }
+    if (rownorm) {
+      VMOBA_TRACE("k_rownorm", stream);
+      k_rownorm<<<(unsigned)(((size_t)P.n_h * P.s + 7) / 8), 256, 0, stream>>>(P, S, st);
+      ++launches;
+    }
+    const size_t pool = (size_t)P.s * P.Nb;
+    dim3 hgrid((unsigned)((pool + kHistChunk - 1) / kHistChunk), P.n_h);
+    for (int pass = 0; pass < 3; ++pass) {
+      {
+        VMOBA_TRACE("k_hist", stream);
+        if (pass == 0) k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+        if (pass == 1) k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+        if (pass == 2) k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+      }
+      ++launches;
+      if ((e = scan(pass, stream)) != cudaSuccess) return e;
+    }
+    for (int pass = 0; pass < 3; ++pass) {
+      {
+        VMOBA_TRACE("k_tie_hist", stream);
+        if (pass == 0) k_tie_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+        if (pass == 1) k_tie_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+        if (pass == 2) k_tie_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc);
+      }
+      ++launches;
+      if ((e = tie_scan(pass, stream)) != cudaSuccess) return e;
+    }
+    dim3 egrid((P.s + 31) / 32, P.n_h);
+    {
+      VMOBA_TRACE("k_emit", stream);
+      k_emit<<<egrid, 256, 0, stream>>>(P, S, st, sel);
+    }
+    ++launches;
   }
   {
     VMOBA_TRACE("k_stats", stream);
     k_stats<<<1, 128, 0, stream>>>(P, st, stats);
   }
-  count_launches(16);
+  ++launches;
+  count_launches(launches);
   return cudaGetLastError();
 }
 

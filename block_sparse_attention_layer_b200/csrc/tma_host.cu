@@ -21,9 +21,11 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (cols * elem_bytes) % 16 != 0 ||
       box_cols * elem_bytes != 128)
     return false;
-  // a driver call: make sure this host thread has the device's context bound
-  // (a thread whose first CUDA work is this call would have none)
-  if (cudaFree(nullptr) != cudaSuccess) return false;
+  // a driver call: make sure this host thread has the device's primary
+  // context bound (a thread whose first CUDA work is this call would have
+  // none); cudaSetDevice binds it without allocating anything
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * elem_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};

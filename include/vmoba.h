@@ -142,7 +142,16 @@ int vmoba_score_select(const vmoba_shape* shape, const void* q, const float* blo
  *   VMOBA_SELECT_TOPK_LOCAL        "topk + local" (about MoBA's selection;
  *                                  the training-free runs use it on 3D
  *                                  blocks): per query row its first
- *                                  min(param = k, N_b) blocks.
+ *                                  min(param = k, N_b) blocks;
+ *   VMOBA_SELECT_ROWNORM_GLOBAL    the method's global pool and cumulative
+ *                                  rule under the other reading of
+ *                                  "normalised similarity": each query's
+ *                                  scores normalised by a softmax over its
+ *                                  own N_b blocks and divided by s, so
+ *                                  every query carries 1/s of the head's
+ *                                  mass; param = tau.  Ranked by that value
+ *                                  (ties by index); cut_score is the log row
+ *                                  softmax of the last pair kept.
  * tau must be > 0 (>= 1 keeps everything); k a whole number >= 1 (at or
  * above the pool / N_b keeps everything); anything else, or an unknown
  * variant, -> VMOBA_ERR_ARG.  Same buffers, alignment rule and outputs as
@@ -154,7 +163,8 @@ enum {
   VMOBA_SELECT_THRESHOLD_GLOBAL = 0,
   VMOBA_SELECT_TOPK_GLOBAL = 1,
   VMOBA_SELECT_THRESHOLD_LOCAL = 2,
-  VMOBA_SELECT_TOPK_LOCAL = 3
+  VMOBA_SELECT_TOPK_LOCAL = 3,
+  VMOBA_SELECT_ROWNORM_GLOBAL = 4
 };
 int vmoba_score_select_variant(const vmoba_shape* shape, const void* q, const float* blocks,
                                int variant, double param, float scale, uint32_t* sel_bits,
@@ -225,6 +235,21 @@ int vmoba_debug_set_wait(long long wait_cycles, int skip_forward_loads);
  * engine that has pooled all device memory at start-up and forbids later
  * cudaMalloc, or a plugin that is given no allocator.  This entry point has
  * no counterpart in the paper: it only changes where scratch memory lives.
+ * - The array is committed on a device when the CUDA runtime loads the
+ *   library's device code there.  With lazy module loading (the CUDA 12
+ *   default) that can happen at this entry point's first call on the
+ *   device, so make one warm-up call on each device before reserving a
+ *   memory pool that leaves no room for 16 MiB; the array then stays
+ *   committed until the process exits.
+ * - Problems whose scratch exceeds VMOBA_STATIC_SELECT_SCRATCH_BYTES return
+ *   VMOBA_ERR_WORKSPACE without launching anything.  For bf16 inputs the
+ *   scratch is the bf16 hi / lo split of the block means (4 * n_heads *
+ *   N_b' * head_dim bytes, N_b' = N_b rounded up to 128; the score pool is
+ *   recomputed, never stored) plus about 24.6 KB per head of histograms and
+ *   search state: 12 heads x 288 blocks x 128 (2.7 MB) fits, 128 heads x
+ *   1024 blocks x 128 (67 MB) does not.  For fp32 inputs the fp32 score pool
+ *   (4 * n_heads * s * N_b bytes) takes the split's place: 2 heads x 256
+ *   tokens x 8 blocks fits, 12 heads x 55296 tokens x 24 blocks does not.
  * - The array is committed on a device when the CUDA runtime loads the
  *   library's device code there.  With lazy module loading (the CUDA 12
  *   default) that can happen at this entry point's first call on the

@@ -123,7 +123,7 @@ def test_tau_out_of_range_rejected(tau):
 
 @pytest.mark.parametrize("variant,param", [
     (1, 0.0), (1, 2.5), (1, -3.0), (3, 0.0), (3, 1.5), (0, 0.0), (2, -0.1),
-    (2, float("nan")), (3, float("nan")), (4, 1.0), (-1, 1.0)])
+    (2, float("nan")), (3, float("nan")), (4, 0.0), (4, float("nan")), (5, 1.0), (-1, 1.0)])
 def test_selection_variant_arguments_rejected(variant, param):
     sh = _shape().c()
     rc = V.lib().vmoba_score_select_variant(ctypes.byref(sh), BAD, BAD, variant, param, 0.0,

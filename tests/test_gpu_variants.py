@@ -166,3 +166,43 @@ def test_training_free_setting_attention():
         rows = sample_rows(w.s, 128, seed=700 + h)
         o_ref, _ = O.attention_fwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows)
         assert out_err(got[rows, h], o_ref, "bf16") <= TOL["bf16"]
+
+
+def _rownorm_logp(S_h):
+    m = S_h.max(axis=1, keepdims=True)
+    return S_h - (m + np.log(np.exp(S_h - m).sum(axis=1, keepdims=True)))
+
+
+@pytest.mark.parametrize("wid,mode", SMALL)
+@pytest.mark.parametrize("tau", [0.25, 0.6])
+def test_rownorm_global_small(wid, mode, tau):
+    """The per-query reading of the normalisation as a selection variant: the
+    pair set equals the oracle's outside the 1e-4 band around the cut in its
+    own ranking value (the log row softmax); k and the mass match."""
+    w = WORKLOADS[wid]
+    q, k, v = workload_arrays(w, mode)
+    L, g, st = _run(w, mode, q, k, v, "rownorm_global", tau)
+    S = _scores(w, mode, q, k)
+    for h in range(w.n_heads):
+        m, ost = O.rownorm_global_select(S[h], tau)
+        lp = _rownorm_logp(S[h])
+        assert pair_set_mismatch(g[h], lp, m, ost["cut_logp"]) == 0
+        band = np.abs(lp - ost["cut_logp"]) <= BAND_REL * abs(ost["cut_logp"])
+        assert abs(int(st["n_selected"][h]) - ost["k"]) <= int(band.sum())
+        assert abs(float(st["mass"][h]) - ost["mass"]) < 1e-4
+        assert abs(float(st["cut_score"][h]) - ost["cut_logp"]) <= 1e-4 * abs(ost["cut_logp"]) \
+            + 1e-5
+
+
+@pytest.mark.parametrize("mode", [0, 2])
+def test_rownorm_global_full_size(mode):
+    w = WORKLOADS[4]
+    nh = 2
+    q, k, v = synth.make_qkv(w.wid, 30 + mode, w.T, w.H, w.W, nh, w.head_dim)
+    q, k, v = (round_to(x, "bf16") for x in (q, k, v))
+    L, g, st = _run(w, mode, q, k, v, "rownorm_global", 0.25, heads=nh)
+    S = _scores(w, mode, q, k)
+    for h in range(nh):
+        m, ost = O.rownorm_global_select(S[h], 0.25)
+        lp = _rownorm_logp(S[h])
+        assert pair_set_mismatch(g[h], lp, m, ost["cut_logp"]) == 0
