@@ -334,6 +334,7 @@ def run_ours(args, rank, world, local):
     second = paper_block_counts(V, w, (q, k, v, dout), stream)
     variants = selection_variants(V, w, layers, q, density, stream)
     others = other_configs(V, stream) if not args.no_sweeps else None
+    p10_48_60 = paper_10_48_60(V, stream) if not args.no_sweeps else None
 
     # per-call device times (ms, summed over layers, averaged over steps)
     call_ms = {c: 0.0 for c in CALLS}
@@ -422,6 +423,7 @@ def run_ours(args, rank, world, local):
                 "kernel_ms_per_layer": kern_layer,
                 "blocks_8_48_72": second,
                 "other_configs": others,
+                "blocks_10_48_60": p10_48_60,
                 "stack_75600tok_30_layers": sweep,
                 "selection_variants": variants,
                 "layer_call_ms": {f"l{l}": [round(x, 4) for x in layer_call_ms[i]]
@@ -522,6 +524,35 @@ def _layer_record(V, L, ms, d, backward):
             "select_GBps_incl_partition_plan": round(
                 (metrics.partition_bytes(sh.s, sh.n_heads, d, esize, nb)
                  + metrics.select_bytes(sh.s, sh.n_heads, nb)) / (ms_sel * 1e-3) / 1e9, 1)}
+
+
+def paper_10_48_60(V, stream):
+    """The pre-training runs' 10-48-60 block counts at 11520 and 46080 tokens
+    (12 x 128, bf16, tau 0.25, forward + backward; latents chosen so that the
+    counts come out exactly): per mode, density and device ms."""
+    import torch
+
+    import synth
+    from synth import torch_latents as TL
+    from block_sparse_attention_layer_b200 import LayerShape
+    from block_sparse_attention_layer_b200.layer import VMoBALayer
+    res = {}
+    for name, w in synth.PAPER_10_48_60.items():
+        rows = []
+        for mode in range(3):
+            q, k, v = TL.make_qkv(w.wid, mode, w.T, w.H, w.W, w.n_heads, w.head_dim,
+                                  kind=w.kind)
+            dout = TL.make_dout(w.wid, mode, w.s, w.n_heads, w.head_dim)
+            L = VMoBALayer(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode,
+                                      *w.boxes[mode], "bf16"))
+            ms = _time_layer_calls(V, L, q, k, v, w.taus[0], dout, stream)
+            rec = _layer_record(V, L, ms, w.head_dim, True)
+            rec.update(mode=mode, n_blocks=L.n_blocks, box=list(w.boxes[mode]))
+            rows.append(rec)
+            del L
+        res[name] = rows
+    torch.cuda.empty_cache()
+    return res
 
 
 def other_configs(V, stream):

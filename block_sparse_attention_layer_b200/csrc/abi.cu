@@ -74,9 +74,9 @@ ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
   b.rows = item_rows_capacity(P);
   char* p = ws_ptr<char>(ws, L.items);
   b.qg = reinterpret_cast<__nv_bfloat16*>(p);
-  p += align_up(b.rows * 128 * sizeof(__nv_bfloat16), 256);
+  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
   b.dog = reinterpret_cast<__nv_bfloat16*>(p);
-  p += align_up(b.rows * 128 * sizeof(__nv_bfloat16), 256);
+  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
   b.l2g = reinterpret_cast<float*>(p);
   p += align_up(b.rows * sizeof(float), 256);
   b.dg = reinterpret_cast<float*>(p);
@@ -233,8 +233,8 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
   WsLayout L;
   if ((rc = check_ws(P, ws, ws_bytes, &L)) != VMOBA_OK) return rc;
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
-  // bf16 with head_dim 128 runs on the tensor cores; fp32 I/O (whose 1e-4
-  // bar rules out TF32) and head_dim 64 run on the CUDA cores
+  // bf16 runs on the tensor cores; fp32 I/O (whose 1e-4 bar rules out
+  // TF32) runs on the CUDA cores
   drop_stale_error();
   if (uses_blk_path(P))
     return cuda_status(launch_attn_fwd_blk(

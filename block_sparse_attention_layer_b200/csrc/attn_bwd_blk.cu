@@ -1,5 +1,5 @@
 // Sparse attention backward, block-major, on the 5th-generation tensor cores
-// (bf16, head_dim 128).  The selection mask is held constant (the pages add
+// (bf16, head_dim D = 64 or 128).  The selection mask is held constant (the pages add
 // no loss and route no gradient through it):
 //   P = exp(scale q.k - LSE),  D_i = dO_i . O_i,  dS = P (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO   (selected pairs only).
@@ -24,9 +24,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int kD = 128;
+// 128 rows x 64 bf16: one 128-byte swizzle atom wide; a 128-row tile of
+// head_dim D is D / 64 of them side by side
 constexpr uint32_t kHalf = 128 * 64 * 2;
-constexpr uint32_t kTileB = 2 * kHalf;
+template <int D>
+constexpr uint32_t tile_bytes() { return (D / 64) * kHalf; }
 // 384 threads: warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 two softmax
 // warpgroups that split each tile's 128 columns 64/64 (a warp reaches TMEM
 // lanes 32*(warp % 4) .. +32, so both groups cover all 128 rows).
@@ -41,16 +43,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ------------------------------------------------------------- D_i, lse2
 // rowD[h][i] = dO_i . O_i (fp32 output copy); nlse2[h][i] = -LSE_i * log2(e),
 // so that P = 2^(S scale log2(e) + nlse2) is one fused multiply-add and ex2.
+template <int D>
 __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
                            const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                            float* __restrict__ rowD, float* __restrict__ lse2) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= P.s * P.n_h) return;
   const int i = warp / P.n_h, h = warp - i * P.n_h;
-  const float4 a = reinterpret_cast<const float4*>(o32 + (size_t)warp * kD)[lane];
-  const uint2 b = reinterpret_cast<const uint2*>(dout + (size_t)warp * kD)[lane];
-  float acc = a.x * __uint_as_float(b.x << 16) + a.y * __uint_as_float(b.x & 0xFFFF0000u) +
-              a.z * __uint_as_float(b.y << 16) + a.w * __uint_as_float(b.y & 0xFFFF0000u);
+  float acc;
+  if constexpr (D == 128) {
+    const float4 a = reinterpret_cast<const float4*>(o32 + (size_t)warp * D)[lane];
+    const uint2 b = reinterpret_cast<const uint2*>(dout + (size_t)warp * D)[lane];
+    acc = a.x * __uint_as_float(b.x << 16) + a.y * __uint_as_float(b.x & 0xFFFF0000u) +
+          a.z * __uint_as_float(b.y << 16) + a.w * __uint_as_float(b.y & 0xFFFF0000u);
+  } else {
+    const float2 a = reinterpret_cast<const float2*>(o32 + (size_t)warp * D)[lane];
+    const uint32_t b = reinterpret_cast<const uint32_t*>(dout + (size_t)warp * D)[lane];
+    acc = a.x * __uint_as_float(b << 16) + a.y * __uint_as_float(b & 0xFFFF0000u);
+  }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   if (lane == 0) {
@@ -61,7 +71,7 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
 
 // =====================================================================
 // dQ pass.  TMEM: S0 [0,128), S1 [128,256), dP [256,384) (then dS), dQ
-// [384,512).  Roles: warp 0 TMA (the item's Q and dO tiles from the
+// [384,384+D).  Roles: warp 0 TMA (the item's Q and dO tiles from the
 // item-ordered copies, then the block's K, V chunks), warp 1 MMA, warps
 // 4-7 / 8-11 softmax of key columns 0-63 / 64-127 + epilogue (warps 2-3
 // idle).  Per chunk J the softmax forms P(J) from S(J) and frees S, then
@@ -77,10 +87,14 @@ struct DqBars {
   int abort;
 };
 constexpr uint32_t kStageB = 32 * 32 * 4;     // epilogue staging per softmax warp
-constexpr size_t kDqSmem = 1024 + 2 * kTileB /*Q,dO*/ + 4 * kTileB /*K,V x2*/ + 8 * kStageB +
-                           sizeof(DqBars) + 64;
-static_assert(kDqSmem <= 232448, "shared memory per CTA");
+template <int D>
+constexpr size_t dq_smem() {
+  return 1024 + 2 * tile_bytes<D>() /*Q,dO*/ + 4 * tile_bytes<D>() /*K,V x2*/ + 8 * kStageB +
+         sizeof(DqBars) + 64;
+}
+static_assert(dq_smem<128>() <= 232448, "shared memory per CTA");
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
@@ -90,6 +104,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t kTileB = tile_bytes<D>();
   uint8_t* sQ = smem;
   uint8_t* sO = sQ + kTileB;              // dO tile
   uint8_t* sK = sO + kTileB;              // 2 stages
@@ -143,9 +158,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         if (!ok) break;
         mbar_expect_tx(&bars->qd_full, 2 * kTileB);
         tma_load_2d(sQ, &tm_q, &bars->qd_full, 0, n * kTile);
-        tma_load_2d(sQ + kHalf, &tm_q, &bars->qd_full, 64, n * kTile);
+        if (D == 128) tma_load_2d(sQ + kHalf, &tm_q, &bars->qd_full, 64, n * kTile);
         tma_load_2d(sO, &tm_o, &bars->qd_full, 0, n * kTile);
-        tma_load_2d(sO + kHalf, &tm_o, &bars->qd_full, 64, n * kTile);
+        if (D == 128) tma_load_2d(sO + kHalf, &tm_o, &bars->qd_full, 64, n * kTile);
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + it.j * P.L + c * kTile;
           const int st = J & 1;
@@ -153,19 +168,19 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           if (!ok) break;
           mbar_expect_tx(&bars->full_k[st], kTileB);
           tma_load_2d(sK + st * kTileB, &tm_k, &bars->full_k[st], 0, row);
-          tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
+          if (D == 128) tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
           if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_v[st], kTileB);
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
-          tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
+          if (D == 128) tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
         if (ok && n + G < n_items) {
           // the next item's Q / dO into L2 behind this item's loads (one buffer in smem)
-          tma_prefetch_l2_2d(&tm_q, 0, (n + G) * kTile);
-          tma_prefetch_l2_2d(&tm_q, 64, (n + G) * kTile);
-          tma_prefetch_l2_2d(&tm_o, 0, (n + G) * kTile);
-          tma_prefetch_l2_2d(&tm_o, 64, (n + G) * kTile);
+          for (int x = 0; x < D; x += 64) {
+            tma_prefetch_l2_2d(&tm_q, x, (n + G) * kTile);
+            tma_prefetch_l2_2d(&tm_o, x, (n + G) * kTile);
+          }
         }
       }
     }
@@ -173,7 +188,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (lane == 0) {
       const uint32_t idSS = idesc_bf16(128, 128, false, false);
       const uint32_t idSS_last = idesc_bf16(128, (kc_last + 15) & ~15, false, false);
-      const uint32_t idDQ = idesc_bf16(128, 128, false, true);
+      const uint32_t idDQ = idesc_bf16(128, D, false, true);
       const int ks_last = (kc_last + 15) / 16;
       const uint32_t qb = smem_u32(sQ), ob = smem_u32(sO);
       const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / G + 1 : 0;
@@ -190,7 +205,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         const uint32_t kb = smem_u32(sK + st * kTileB);
         const uint32_t idc = c == nch - 1 ? idSS_last : idSS;   // N = the chunk's keys
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tmem + st * 128, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
                  idc, kk > 0 ? 1u : 0u);
@@ -206,7 +221,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         const uint32_t vb = smem_u32(sV + st * kTileB);
         const uint32_t idc = c == nch - 1 ? idSS_last : idSS;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tdP, desc_sw128(ob + off, 16, 1024), desc_sw128(vb + off, 16, 1024), idc,
                  kk > 0 ? 1u : 0u);
@@ -332,9 +347,10 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {               // this group's 64 dQ columns
+      constexpr int kQc = D / 2;                      // dQ columns of each group
+      for (int cc = 0; cc < kQc / 32; ++cc) {          // this group's D / 2 dQ columns
         uint32_t xr[32];
-        tmem_ld32(tDQ + lane_off + cb + cc * 32, xr);
+        tmem_ld32(tDQ + lane_off + kQc * wg + cc * 32, xr);
         tmem_ld_wait();
         // the staging tile is free once the previous store has read it
         if (lane == 0) bulk_wait_read_all();
@@ -350,7 +366,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         __syncwarp();
         // the warp's 32 item rows, 32 columns, in one asynchronous store
         if (lane == 0) {
-          tma_store_2d(&tm_pd, stg, cb + cc * 32, n * kTile + wq * 32);
+          tma_store_2d(&tm_pd, stg, kQc * wg + cc * 32, n * kTile + wq * 32);
           bulk_commit();
         }
       }
@@ -368,8 +384,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   }
 }
 
-// dQ_i = scale * sum_j partial_ij, blocks in ascending order; one warp per row.
-// The partials sit at the pairs' item rows (slot_row).
+// dQ_i = scale * sum_j partial_ij, blocks in ascending order; one warp per row
+// (D / 32 dims per lane).  The partials sit at the pairs' item rows (slot_row).
+template <int D>
 __global__ void __launch_bounds__(256)
 k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, float scale,
                __nv_bfloat16* __restrict__ dq) {
@@ -378,23 +395,33 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
   const uint32_t off = __ldg(pv.row_off + (size_t)h * (P.s + 1) + i);
   const uint32_t cnt = __ldg(pv.row_cnt + (size_t)h * P.s + i);
   const uint32_t* srow = pv.slot_row + (size_t)h * P.s * P.Nb + off;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  __nv_bfloat16* dst = dq + ((size_t)i * P.n_h + h) * D;
+  if constexpr (D == 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-  for (uint32_t k = 0; k < cnt; ++k) {
-    const uint32_t row = __ldg(srow + k);
-    const float4 o = reinterpret_cast<const float4*>(part_dq + (size_t)row * kD)[lane];
-    acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    for (uint32_t k = 0; k < cnt; ++k) {
+      const uint32_t row = __ldg(srow + k);
+      const float4 o = reinterpret_cast<const float4*>(part_dq + (size_t)row * D)[lane];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    reinterpret_cast<uint2*>(dst)[lane] = make_uint2(pack_bf16x2(acc.x * scale, acc.y * scale),
+                                                     pack_bf16x2(acc.z * scale, acc.w * scale));
+  } else {
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (uint32_t k = 0; k < cnt; ++k) {
+      const uint32_t row = __ldg(srow + k);
+      const float2 o = reinterpret_cast<const float2*>(part_dq + (size_t)row * D)[lane];
+      acc.x += o.x; acc.y += o.y;
+    }
+    reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(acc.x * scale, acc.y * scale);
   }
-  uint2 ob;
-  ob.x = pack_bf16x2(acc.x * scale, acc.y * scale);
-  ob.y = pack_bf16x2(acc.z * scale, acc.w * scale);
-  reinterpret_cast<uint2*>(dq + ((size_t)i * P.n_h + h) * kD)[lane] = ob;
 }
 
 // =====================================================================
 // dK/dV pass.  Item = (key tile kt of block j, head h), one CTA each.
-// TMEM: S^T [0,128) (then P^T), dP^T [128,256) (then dS^T), dV [256,384),
-// dK [384,512).  Two softmax warpgroups split each query tile's columns
+// TMEM: S^T [0,128) (then P^T), dP^T [128,256) (then dS^T), dV [256,256+D),
+// dK [384,384+D).  Two softmax warpgroups split each query tile's columns
 // 64 / 64.  The tile's work is cut where its dependencies allow:
 //   S^T(g)  -> P^T(g) (exponentials)            -> dV(g) += P^T dO
 //   dP^T(g) -> dS^T(g) = P^T (dP^T - D)          -> dK(g) += dS^T Q
@@ -414,9 +441,13 @@ struct KvBars {
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kKvSmem = 1024 + 2 * kTileB /*K,V*/ + 4 * kTileB /*Q,dO x2*/ +
-                           2 * 2 * kTile * sizeof(float) /*nlse2, D x2*/ + sizeof(KvBars) + 64;
+template <int D>
+constexpr size_t kv_smem() {
+  return 1024 + 2 * tile_bytes<D>() /*K,V*/ + 4 * tile_bytes<D>() /*Q,dO x2*/ +
+         2 * 2 * kTile * sizeof(float) /*nlse2, D x2*/ + sizeof(KvBars) + 64;
+}
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
@@ -427,6 +458,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t kTileB = tile_bytes<D>();
   uint8_t* sK = smem;
   uint8_t* sV = sK + kTileB;
   uint8_t* sQ = sV + kTileB;           // 2 buffers
@@ -475,9 +507,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const int row = h * P.s + key0;
       mbar_expect_tx(&bars->kv_full, 2 * kTileB);
       tma_load_2d(sK, &tm_k, &bars->kv_full, 0, row);
-      tma_load_2d(sK + kHalf, &tm_k, &bars->kv_full, 64, row);
+      if (D == 128) tma_load_2d(sK + kHalf, &tm_k, &bars->kv_full, 64, row);
       tma_load_2d(sV, &tm_v, &bars->kv_full, 0, row);
-      tma_load_2d(sV + kHalf, &tm_v, &bars->kv_full, 64, row);
+      if (D == 128) tma_load_2d(sV + kHalf, &tm_v, &bars->kv_full, 64, row);
       bool ok = true;
       for (int g = 0; g < ng && ok; ++g) {
         const int b = g & 1;
@@ -486,9 +518,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int qrow = (item0 + g) * kTile;
         mbar_expect_tx(&bars->qd_full[b], 2 * kTileB + 2 * kTile * sizeof(float));
         tma_load_2d(sQ + b * kTileB, &tm_q, &bars->qd_full[b], 0, qrow);
-        tma_load_2d(sQ + b * kTileB + kHalf, &tm_q, &bars->qd_full[b], 64, qrow);
+        if (D == 128) tma_load_2d(sQ + b * kTileB + kHalf, &tm_q, &bars->qd_full[b], 64, qrow);
         tma_load_2d(sO + b * kTileB, &tm_o, &bars->qd_full[b], 0, qrow);
-        tma_load_2d(sO + b * kTileB + kHalf, &tm_o, &bars->qd_full[b], 64, qrow);
+        if (D == 128) tma_load_2d(sO + b * kTileB + kHalf, &tm_o, &bars->qd_full[b], 64, qrow);
         bulk_load(sL + b * kTile, l2g + qrow, kTile * sizeof(float), &bars->qd_full[b]);
         bulk_load(sD + b * kTile, dg + qrow, kTile * sizeof(float), &bars->qd_full[b]);
       }
@@ -496,12 +528,12 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0 && ng > 0) {
       const uint32_t idSS = idesc_bf16(128, 128, false, false);
-      const uint32_t idAcc = idesc_bf16(128, 128, false, true);
+      const uint32_t idAcc = idesc_bf16(128, D, false, true);
       const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
       // S^T = K Q^T (or dP^T = V dO^T): keys x queries, K-major both sides
       auto issue_ss = [&](uint32_t tD, uint32_t ab, uint32_t bb) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tD, desc_sw128(ab + off, 16, 1024), desc_sw128(bb + off, 16, 1024), idSS,
                  kk > 0 ? 1u : 0u);
@@ -643,9 +675,9 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int half = wg == 0 ? 1 : 0;
         const uint32_t base = half == 0 ? tK : tV;
         const float f = half == 0 ? scale : 1.0f;
-        __nv_bfloat16* dst = (half == 0 ? dk : dv) + ((size_t)n * P.n_h + h) * kD;
+        __nv_bfloat16* dst = (half == 0 ? dk : dv) + ((size_t)n * P.n_h + h) * D;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t xr[32];
           if (have) {
             tmem_ld32(base + lane_off + cc * 32, xr);
@@ -685,18 +717,20 @@ size_t bwd_blk_ws_bytes(const Prob& P) {
   return 2 * align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
 }
 
-cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
-                                const uint32_t* sel, const PairsView& pv, void* part,
-                                const ItemBufs& ib, const float* o32, const float* lse,
-                                const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
-                                float scale, int* status, int num_sms, cudaStream_t st) {
+namespace {
+
+template <int D>
+cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
+                    const PairsView& pv, void* part, const ItemBufs& ib, const float* o32,
+                    const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                    void* ws_bwd, float scale, int* status, int num_sms, cudaStream_t st) {
   CUtensorMap tk, tv, tq, to, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   float* part_dq = static_cast<float*>(part);
-  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
-      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, kD, 128) ||
-      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, kD, 128) ||
-      !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), kD,
+  if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
+      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, D, 128) ||
+      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, D, 128) ||
+      !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), D,
                     32, 32))
     return cudaErrorInvalidValue;
   float* rowD = static_cast<float*>(ws_bwd);
@@ -705,14 +739,15 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
   const int warps = P.s * P.n_h;
   {
     VMOBA_TRACE("k_bwd_rows", st);
-    k_bwd_rows<<<(warps + 7) / 8, 256, 0, st>>>(P, o32, static_cast<const __nv_bfloat16*>(dout),
-                                                lse, rowD, lse2);
+    k_bwd_rows<D><<<(warps + 7) / 8, 256, 0, st>>>(
+        P, o32, static_cast<const __nv_bfloat16*>(dout), lse, rowD, lse2);
   }
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_dq_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kDqSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_dq_blk<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)dq_smem<D>());
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_bwd_dkdv_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kKvSmem);
+  e = cudaFuncSetAttribute(k_bwd_dkdv_blk<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kv_smem<D>());
   if (e != cudaSuccess) return e;
   const float sl2 = scale * kLog2e;
   const int nkt = (P.L + kTile - 1) / kTile;
@@ -724,23 +759,37 @@ cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, co
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
-      k_bwd_dq_blk<<<num_sms, kThreads, kDqSmem, st>>>(tk, tv, tq, to, tpd, P, h, pv, ib.dg,
-                                                        ib.l2g, sl2, make_watch(status));
+      k_bwd_dq_blk<D><<<num_sms, kThreads, dq_smem<D>(), st>>>(
+          tk, tv, tq, to, tpd, P, h, pv, ib.dg, ib.l2g, sl2, make_watch(status));
     }
     {
       VMOBA_TRACE("k_bwd_dq_merge", st);
-      k_bwd_dq_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
-                                                    static_cast<__nv_bfloat16*>(dq));
+      k_bwd_dq_merge<D><<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
+                                                       static_cast<__nv_bfloat16*>(dq));
     }
     {
       VMOBA_TRACE("k_bwd_dkdv_blk", st);
-      k_bwd_dkdv_blk<<<P.Nb * nkt, kThreads, kKvSmem, st>>>(
+      k_bwd_dkdv_blk<D><<<P.Nb * nkt, kThreads, kv_smem<D>(), st>>>(
           tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
           static_cast<__nv_bfloat16*>(dv), make_watch(status));
     }
   }
   count_launches(1 + 3 * P.n_h);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
+                                const uint32_t* sel, const PairsView& pv, void* part,
+                                const ItemBufs& ib, const float* o32, const float* lse,
+                                const void* dout, void* dq, void* dk, void* dv, void* ws_bwd,
+                                float scale, int* status, int num_sms, cudaStream_t st) {
+  (void)sel;
+  return P.d == 128 ? bwd_blk<128>(P, q, kp, vp, pv, part, ib, o32, lse, dout, dq, dk, dv, ws_bwd,
+                                   scale, status, num_sms, st)
+                    : bwd_blk<64>(P, q, kp, vp, pv, part, ib, o32, lse, dout, dq, dk, dv, ws_bwd,
+                                  scale, status, num_sms, st);
 }
 
 }  // namespace vmoba

@@ -1,5 +1,5 @@
 // Sparse attention forward, block-major, on the 5th-generation tensor cores
-// (bf16, head_dim 128).
+// (bf16, head_dim D = 64 or 128).
 //
 // VMoBA notes, overall framework: attention only over the selected
 // (query, block) pairs.  A work item is (block j, one tile of 128 queries
@@ -30,7 +30,7 @@
 //               row per thread, lazy 2^8 rescale of O, then the tile's
 //               epilogue (partials out through a per-warp staging tile and
 //               an asynchronous TMA store).
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 // The MMA issue order per chunk c is PV_A(c), S_A(c+1), PV_B(c), S_B(c+1):
 // while one warpgroup computes exponentials the tensor core serves the other.
 // P is written as bf16 pairs over the first half of its own S columns; the
@@ -46,9 +46,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int kD = 128;
+// 128 rows x 64 bf16: one 128-byte swizzle atom wide; a 128-row tile of
+// head_dim D is D / 64 of them side by side
 constexpr uint32_t kHalf = 128 * 64 * 2;
-constexpr uint32_t kTileB = 2 * kHalf;
+template <int D>
+constexpr uint32_t tile_bytes() { return (D / 64) * kHalf; }
 constexpr int kThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
@@ -63,15 +65,18 @@ struct Bars {
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + 2 * kTileB /*Q pair*/ + 2 * kTileB /*K*/ + 2 * kTileB /*V*/ +
-                              8 * kStageB + sizeof(Bars) + 64;
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+template <int D>
+constexpr size_t fwd_smem() {
+  return 1024 + 2 * tile_bytes<D>() /*Q pair*/ + 2 * tile_bytes<D>() /*K*/ +
+         2 * tile_bytes<D>() /*V*/ + 8 * kStageB + sizeof(Bars) + 64;
+}
+static_assert(fwd_smem<128>() <= 232448, "shared memory per CTA");
 
 // One chunk of softmax for one row: P = 2^(S sl2 - m) over the chunk's kc
 // valid keys (NC columns loaded), written as bf16 pairs over S's first NC/2
 // columns; running max / sum updated, O rescaled when the max grew by more
 // than 2^8.
-template <int NC>
+template <int NC, int D>
 __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, float sl2,
                                               float& m_run, float& l_run) {
   uint32_t xr[NC];
@@ -109,7 +114,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, 
   if (__any_sync(0xffffffffu, rescale)) {
     f = rescale ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t ob[32];
       tmem_ld32(tO + cc * 32, ob);
       tmem_ld_wait();
@@ -123,6 +128,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t tS, uint32_t tO, int kc, 
   tmem_st_wait();
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
           const __grid_constant__ CUtensorMap tm_po, const __nv_bfloat16* __restrict__ q,
@@ -131,6 +137,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t kTileB = tile_bytes<D>();
   uint8_t* sQ = smem;                       // tiles A, B
   uint8_t* sK = sQ + 2 * kTileB;            // 2 stages
   uint8_t* sV = sK + 2 * kTileB;            // 2 stages
@@ -187,23 +194,24 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
           if (!ok) break;
           mbar_expect_tx(&bars->full_k[st], kTileB);
           tma_load_2d(sK + st * kTileB, &tm_k, &bars->full_k[st], 0, row);
-          tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
+          if (D == 128) tma_load_2d(sK + st * kTileB + kHalf, &tm_k, &bars->full_k[st], 64, row);
           if (J >= 2) ok = mbar_wait(&bars->empty_v[st], ((J >> 1) - 1) & 1, wt, abort);
           if (!ok) break;
           mbar_expect_tx(&bars->full_v[st], kTileB);
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
-          tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
+          if (D == 128) tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
       }
     }
   } else if (warp == 2 || warp == 3) {
     // -------------------------------------------------------- query gather
     // The pair's query rows straight from Q (one head's rows stay in L2):
-    // warp w copies rows [64 w, 64 w + 64) of each tile, two rows per step
-    // (16 lanes x 16 bytes per 256-byte row), into the 128-byte-swizzled
-    // layout the MMA descriptors read (16-byte granule g of row r at
-    // g ^ (r & 7)); rows past the tile's queries are zero-filled.
-    const int w = warp - 2, c = lane & 15, hr = lane >> 4;
+    // warp w copies rows [64 w, 64 w + 64) of each tile, kRps rows per step
+    // (D / 8 lanes x 16 bytes per row), into the 128-byte-swizzled layout
+    // the MMA descriptors read (16-byte granule g of row r at g ^ (r & 7));
+    // rows past the tile's queries are zero-filled.
+    constexpr int kLpr = D / 8, kRps = 32 / kLpr;     // lanes per row, rows per step
+    const int w = warp - 2, c = lane % kLpr, hr = lane / kLpr;
     const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
     const uint32_t qbase = smem_u32(sQ);
     int it_local = 0, hint = 0;
@@ -233,15 +241,15 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
             base + 32 + lane < m.count ? __ldg(col_rows + m.first + base + 32 + lane) : 0u;
         const uint32_t tbase = qbase + t * kTileB + (c >> 3) * kHalf;
 #pragma unroll 4
-        for (int k = 0; k < 32; ++k) {
-          const int rr = 2 * k + hr;                // row within the warp's 64
+        for (int k = 0; k < 64 / kRps; ++k) {
+          const int rr = kRps * k + hr;             // row within the warp's 64
           const uint32_t i0 = __shfl_sync(0xffffffffu, idx0, rr & 31);
           const uint32_t i1 = __shfl_sync(0xffffffffu, idx1, rr & 31);
           const int r = base + rr;
           const bool in = r < m.count;
           const uint32_t i = in ? (rr < 32 ? i0 : i1) : 0u;
           cp_async16(tbase + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                     q + ((size_t)i * P.n_h + h) * kD + c * 8, in ? 16u : 0u);
+                     q + ((size_t)i * P.n_h + h) * D + c * 8, in ? 16u : 0u);
         }
         // copies landed, made visible to the tensor core's (async) proxy
         cp_async_wait_all();
@@ -254,7 +262,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idS_last = idesc_bf16(128, (kc_last + 15) & ~15, false, false);
-      const uint32_t idPV = idesc_bf16(128, 128, false, true);
+      const uint32_t idPV = idesc_bf16(128, D, false, true);
       const int ks_last = (kc_last + 15) / 16;
       int Jk = 0;                 // chunks through the K / V rings
       int Js[2] = {0, 0};         // S / P rounds per tile
@@ -263,7 +271,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       auto issue_s = [&](int t, uint32_t kb, bool last) {
         const uint32_t qbase = smem_u32(sQ + t * kTileB);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
           mma_ss(tmem + t * 128, desc_sw128(qbase + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
                  last ? idS_last : idS, kk > 0 ? 1u : 0u);
@@ -365,8 +373,8 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
         if (!ok) break;
         tc_fence_after();
         const int kc = c == nch - 1 ? kc_last : kTile;
-        if (kc > 64) softmax_chunk<128>(tS, tO, kc, sl2, m_run, l_run);
-        else softmax_chunk<64>(tS, tO, kc, sl2, m_run, l_run);
+        if (kc > 64) softmax_chunk<128, D>(tS, tO, kc, sl2, m_run, l_run);
+        else softmax_chunk<64, D>(tS, tO, kc, sl2, m_run, l_run);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[t]);
@@ -382,7 +390,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       uint32_t* stw = reinterpret_cast<uint32_t*>(stg);
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {               // 64 columns: 128 fp16 bytes per row
+      for (int cc = 0; cc < D / 64; ++cc) {          // 64 columns: 128 fp16 bytes per row
         uint32_t ob[64];
         tmem_ld32(tO + cc * 64, ob);
         tmem_ld32(tO + cc * 64 + 32, ob + 32);
@@ -429,8 +437,9 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 // Combine the partial (m, l, O / l) of every query's selected blocks:
 // O_i = sum_j 2^(m_j - M) l_j (O / l)_j / sum_j 2^(m_j - M) l_j,
 // LSE_i = (M + log2 sum_j 2^(m_j - M) l_j) ln 2.
-// One warp per query row, four dims per lane, blocks in ascending order; the
-// partials sit at the pairs' item rows (slot_row).
+// One warp per query row, D / 32 dims per lane, blocks in ascending order;
+// the partials sit at the pairs' item rows (slot_row).
+template <int D>
 __global__ void __launch_bounds__(256)
 k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
             const float2* __restrict__ part_ml, __nv_bfloat16* __restrict__ out,
@@ -452,7 +461,10 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
   for (uint32_t b = 32 + lane; b < cnt; b += 32) M = fmaxf(M, part_ml[__ldg(srow + b)].x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int V = D / 32;                  // dims per lane: V / 2 fp16 pairs
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   for (uint32_t b = 0; b < cnt; b += 32) {
     uint32_t my_row = row0;
@@ -472,20 +484,34 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
       const uint32_t row = __shfl_sync(0xffffffffu, my_row, k);
       const float wl = __shfl_sync(0xffffffffu, my_w, k);
       Lsum += wl;
-      const uint2 u = reinterpret_cast<const uint2*>(part_o + (size_t)row * 128)[lane];
-      const float2 a = unpack_f16x2(u.x), c = unpack_f16x2(u.y);
-      acc.x = fmaf(wl, a.x, acc.x); acc.y = fmaf(wl, a.y, acc.y);
-      acc.z = fmaf(wl, c.x, acc.z); acc.w = fmaf(wl, c.y, acc.w);
+      uint32_t u[V / 2];                     // this lane's V fp16 values, one vector load
+      if constexpr (V == 4) {
+        const uint2 x = reinterpret_cast<const uint2*>(part_o + (size_t)row * D)[lane];
+        u[0] = x.x;
+        u[1] = x.y;
+      } else {
+        u[0] = reinterpret_cast<const uint32_t*>(part_o + (size_t)row * D)[lane];
+      }
+#pragma unroll
+      for (int e = 0; e < V / 2; ++e) {
+        const float2 a = unpack_f16x2(u[e]);
+        acc[2 * e] = fmaf(wl, a.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wl, a.y, acc[2 * e + 1]);
+      }
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-  const size_t row = ((size_t)i * P.n_h + h) * 128;
-  reinterpret_cast<float4*>(o32 + row)[lane] = acc;
-  uint2 ob;
-  ob.x = pack_bf16x2(acc.x, acc.y);
-  ob.y = pack_bf16x2(acc.z, acc.w);
-  reinterpret_cast<uint2*>(out + row)[lane] = ob;
+  const size_t row = ((size_t)i * P.n_h + h) * D;
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] *= inv;
+  if constexpr (V == 4) {
+    reinterpret_cast<float4*>(o32 + row)[lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    reinterpret_cast<uint2*>(out + row)[lane] =
+        make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+  } else {
+    reinterpret_cast<float2*>(o32 + row)[lane] = make_float2(acc[0], acc[1]);
+    reinterpret_cast<uint32_t*>(out + row)[lane] = pack_bf16x2(acc[0], acc[1]);
+  }
   if (lane == 0)
     lse[(size_t)h * P.s + i] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY;
 }
@@ -494,43 +520,57 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
 
 size_t blk_partial_bytes(const Prob& P) {
   // one head's partials, one row per work-item row (item_rows_capacity rows):
-  // 128 fp32 (dQ pass) or 128 fp16 (forward O / l), then the forward's (m, l)
+  // d fp32 (dQ pass) or d fp16 (forward O / l), then the forward's (m, l)
   const size_t rows = item_rows_capacity(P);
-  return align_up(rows * 128 * sizeof(float), 256) + align_up(rows * sizeof(float2), 256);
+  return align_up(rows * P.d * sizeof(float), 256) + align_up(rows * sizeof(float2), 256);
 }
 
-cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
-                                const uint32_t* sel, const PairsView& pv, void* part,
-                                const ItemBufs& ib, float scale, void* out, float* o32,
-                                float* lse, int* status, int num_sms, cudaStream_t st) {
+namespace {
+
+template <int D>
+cudaError_t fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
+                    const PairsView& pv, void* part, float scale, void* out, float* o32,
+                    float* lse, int* status, int num_sms, cudaStream_t st) {
   CUtensorMap tk, tv, tpo;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   const size_t prows = item_rows_capacity(P);
   __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
   float2* part_ml = reinterpret_cast<float2*>(
-      static_cast<char*>(part) + align_up(prows * 128 * sizeof(float), 256));
-  if (!make_tmap_bf16_2d(&tk, kp, rows, kD, 128) || !make_tmap_bf16_2d(&tv, vp, rows, kD, 128) ||
-      !make_tmap_2d(&tpo, part_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, prows, kD, 64, 32))
+      static_cast<char*>(part) + align_up(prows * D * sizeof(float), 256));
+  if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
+      !make_tmap_2d(&tpo, part_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, prows, D, 64, 32))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_blk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_blk<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)fwd_smem<D>());
   if (e != cudaSuccess) return e;
   const float sl2 = scale * 1.4426950408889634f;
   for (int h = 0; h < P.n_h; ++h) {
     {
       VMOBA_TRACE("k_fwd_blk", st);
-      k_fwd_blk<<<num_sms, kThreads, kSmemBytes, st>>>(
+      k_fwd_blk<D><<<num_sms, kThreads, fwd_smem<D>(), st>>>(
           tk, tv, tpo, static_cast<const __nv_bfloat16*>(q), P, h, pv, sl2, part_ml,
           make_watch(status));
     }
     {
       VMOBA_TRACE("k_fwd_merge", st);
-      k_fwd_merge<<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_o, part_ml,
-                                                 static_cast<__nv_bfloat16*>(out), o32, lse);
+      k_fwd_merge<D><<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_o, part_ml,
+                                                    static_cast<__nv_bfloat16*>(out), o32, lse);
     }
   }
   count_launches(2 * P.n_h);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
+                                const uint32_t* sel, const PairsView& pv, void* part,
+                                const ItemBufs& ib, float scale, void* out, float* o32,
+                                float* lse, int* status, int num_sms, cudaStream_t st) {
+  (void)sel;
+  (void)ib;
+  return P.d == 128 ? fwd_blk<128>(P, q, kp, vp, pv, part, scale, out, o32, lse, status, num_sms, st)
+                    : fwd_blk<64>(P, q, kp, vp, pv, part, scale, out, o32, lse, status, num_sms, st);
 }
 
 }  // namespace vmoba

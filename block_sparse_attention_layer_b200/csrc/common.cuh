@@ -109,9 +109,9 @@ size_t blk_partial_bytes(const Prob& P);
 int sel_split_rows(const Prob& P);
 size_t sel_split_bytes(const Prob& P);
 size_t item_bufs_bytes(const Prob& P);
-// bf16 with head_dim 128 runs the block-major tensor-core kernels; fp32 I/O
-// (whose 1e-4 bar rules out TF32) and head_dim 64 run on the CUDA cores.
-inline bool uses_blk_path(const Prob& P) { return P.dtype == VMOBA_BF16 && P.d == 128; }
+// bf16 (head_dim 64 or 128) runs the block-major tensor-core kernels; fp32
+// I/O (whose 1e-4 bar rules out TF32) runs on the CUDA cores.
+inline bool uses_blk_path(const Prob& P) { return P.dtype == VMOBA_BF16; }
 
 inline WsLayout ws_layout(const Prob& P) {
   WsLayout w{};
@@ -123,10 +123,11 @@ inline WsLayout ws_layout(const Prob& P) {
   w.hist_mass = take(sizeof(double) * kHistBins * P.n_h);
   w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
   w.bsplit = take(sel_split_bytes(P));
-  w.qt_kt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
-  w.qt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
-  w.kt_qt_bits = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt);
-  w.kt_work = take(sizeof(uint32_t) * (size_t)P.n_h * P.n_qt);
+  const bool tiles = !uses_blk_path(P);     // tile plan of the CUDA-core kernels
+  w.qt_kt_bits = take(tiles ? sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt : 0);
+  w.qt_work = take(tiles ? sizeof(uint32_t) * (size_t)P.n_h * P.n_qt : 0);
+  w.kt_qt_bits = take(tiles ? sizeof(uint32_t) * (size_t)P.n_h * P.n_qt * P.Wqt : 0);
+  w.kt_work = take(tiles ? sizeof(uint32_t) * (size_t)P.n_h * P.n_qt : 0);
   w.o32 = take(sizeof(float) * (size_t)P.n_h * P.s * P.d);
   w.pairs = take(pairs_ws_bytes(P));
   w.part = take(uses_blk_path(P) ? blk_partial_bytes(P) : 0);

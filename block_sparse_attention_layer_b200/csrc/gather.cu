@@ -4,16 +4,17 @@
 // [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
 // rows past the list end are zero.  The backward kernels (dQ pass, dK/dV
 // pass) then fetch query tiles with plain 2-D TMA instead of scattered loads;
-// the forward gathers its own query rows from Q.  One warp per item;
-// 16 lanes x 16 bytes move a 256-byte row, sixteen rows in flight.
+// the forward gathers its own query rows from Q.  One warp per item; D / 8
+// lanes x 16 bytes move a row of head_dim D, 8 instructions in flight.
 #include "common.cuh"
 #include "pairs.cuh"
 
 namespace vmoba {
 namespace {
 
-constexpr int kPairsInFlight = 8;        // two rows per warp instruction
+constexpr int kInFlight = 8;             // warp instructions in flight per batch
 
+template <int D>
 __global__ void __launch_bounds__(256)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
                const __nv_bfloat16* __restrict__ b, __nv_bfloat16* __restrict__ ag,
@@ -23,7 +24,8 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
   const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
   const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4, c = lane & 15;     // row of the instruction's two, 16-byte chunk
+  constexpr int kLpr = D / 8, kRpi = 32 / kLpr;  // lanes per row, rows per instruction
+  const int half = lane / kLpr, c = lane % kLpr;  // row of the instruction's kRpi, 16-byte chunk
   const int warps = (gridDim.x * blockDim.x) >> 5;
   int hint = 0;
   for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < n_items; n += warps) {
@@ -31,22 +33,22 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
     const int count = it.count;
     const uint32_t* rows = col_rows + it.first;
     const size_t base = (size_t)n * kTile;
-    for (int r0 = 0; r0 < kTile; r0 += 2 * kPairsInFlight) {
-      uint4 va[kPairsInFlight], vb[kPairsInFlight];
+    for (int r0 = 0; r0 < kTile; r0 += kRpi * kInFlight) {
+      uint4 va[kInFlight], vb[kInFlight];
 #pragma unroll
-      for (int u = 0; u < kPairsInFlight; ++u) {
-        const int r = r0 + 2 * u + half;
+      for (int u = 0; u < kInFlight; ++u) {
+        const int r = r0 + kRpi * u + half;
         va[u] = make_uint4(0u, 0u, 0u, 0u);
         vb[u] = make_uint4(0u, 0u, 0u, 0u);
         if (r < count) {
-          const size_t src = ((size_t)__ldg(rows + r) * P.n_h + h) * 128;
+          const size_t src = ((size_t)__ldg(rows + r) * P.n_h + h) * D;
           va[u] = __ldg(reinterpret_cast<const uint4*>(a + src) + c);
           if (b) vb[u] = __ldg(reinterpret_cast<const uint4*>(b + src) + c);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kPairsInFlight; ++u) {
-        const size_t dst = (base + r0 + 2 * u + half) * 128;
+      for (int u = 0; u < kInFlight; ++u) {
+        const size_t dst = (base + r0 + kRpi * u + half) * D;
         reinterpret_cast<uint4*>(ag + dst)[c] = va[u];
         if (b) reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
       }
@@ -80,7 +82,12 @@ cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 int num_sms, cudaStream_t st) {
   {
     VMOBA_TRACE("k_gather_items", st);
-    k_gather_items<<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg, fa_pad);
+    if (P.d == 128)
+      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg,
+                                                       fa_pad);
+    else
+      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg,
+                                                      fa_pad);
   }
   count_launches(1);
   return cudaGetLastError();
@@ -92,7 +99,7 @@ namespace vmoba {
 
 size_t item_bufs_bytes(const Prob& P) {
   const size_t rows = item_rows_capacity(P);
-  return 2 * align_up(rows * 128 * sizeof(__nv_bfloat16), 256) +
+  return 2 * align_up(rows * P.d * sizeof(__nv_bfloat16), 256) +
          2 * align_up(rows * sizeof(float), 256);
 }
 

@@ -91,18 +91,22 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   uint32_t* qt_work = ws_ptr<uint32_t>(ws, L.qt_work);
   uint32_t* kt_qt = ws_ptr<uint32_t>(ws, L.kt_qt_bits);
   uint32_t* kt_work = ws_ptr<uint32_t>(ws, L.kt_work);
-  const size_t nbw = (size_t)P.n_h * P.n_qt * P.Wqt;
-  const size_t nw = (size_t)P.n_h * P.n_qt;
+  // the tile bitmaps serve the CUDA-core kernels only; the tensor-core
+  // kernels walk the pair lists
+  const bool tiles = !uses_blk_path(P);
+  const size_t nbw = tiles ? (size_t)P.n_h * P.n_qt * P.Wqt : 0;
+  const size_t nw = tiles ? (size_t)P.n_h * P.n_qt : 0;
   {
     VMOBA_TRACE("k_plan_clear", st);
-    k_plan_clear<<<148, 256, 0, st>>>(kt_qt, kt_work, nbw, nw, ws_ptr<int>(ws, L.status));
+    k_plan_clear<<<tiles ? 148 : 1, 256, 0, st>>>(kt_qt, kt_work, nbw, nw,
+                                                   ws_ptr<int>(ws, L.status));
   }
-  dim3 grid(P.n_qt, P.n_h);
-  {
+  if (tiles) {
+    dim3 grid(P.n_qt, P.n_h);
     VMOBA_TRACE("k_plan_tiles", st);
     k_plan_tiles<<<grid, kTile, 0, st>>>(P, sel, qt_kt, qt_work, kt_qt, kt_work);
   }
-  count_launches(2);
+  count_launches(tiles ? 2 : 1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_pairs(P, sel, pairs_view(P, ws_ptr<char>(ws, L.pairs)), st);

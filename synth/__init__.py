@@ -13,4 +13,4 @@ from .video_latents import (  # noqa: F401
     make_dout,
     seed_for,
 )
-from .workloads import BOXES_8_48_72, WORKLOADS, Workload  # noqa: F401
+from .workloads import BOXES_8_48_72, PAPER_10_48_60, WORKLOADS, Workload  # noqa: F401

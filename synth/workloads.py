@@ -59,3 +59,21 @@ WORKLOADS = {
 # 4; 3D is workload 4's 4x6x8 box doubled in height and width (4x12x16).
 BOXES_8_48_72 = ((3, 36, 64), (24, 6, 8), (4, 12, 16))
 
+
+# The 10-48-60 setting of the pages' pre-training runs (digest, App. C: 11K
+# and 46K tokens, 1D / 2D / 3D block counts 10, 48 and 60, tau 0.25, the Wan
+# 2.1 architecture).  The pages give neither the latents' T, H, W nor the
+# boxes; these latents are chosen so that the three counts come out exactly:
+#   11520 tokens = T10 x H32 x W36: 1D one frame (10 blocks of 1152), 2D 4x6
+#     (8 x 6 = 48 blocks of 240), 3D 2x8x12 (5 x 4 x 3 = 60 blocks of 192);
+#   46080 tokens = T30 x H32 x W48: 1D three frames (10 blocks of 4608), 2D
+#     4x8 (8 x 6 = 48 blocks of 960), 3D 6x8x16 (5 x 4 x 3 = 60 blocks of 768).
+# 12 heads of 128 (the Wan 2.1 1.3B attention shape), bf16, fwd + bwd.
+PAPER_10_48_60 = {
+    "11520tok": Workload(60, "pretrain-11520tok", 10, 32, 36, 12, 128, "bf16", "smooth",
+                         ((1, 32, 36), (10, 4, 6), (2, 8, 12)), (0.25,), True,
+                         notes="10-48-60 block counts at 11K tokens"),
+    "46080tok": Workload(61, "pretrain-46080tok", 30, 32, 48, 12, 128, "bf16", "smooth",
+                         ((3, 32, 48), (30, 4, 8), (6, 8, 16)), (0.25,), True,
+                         notes="10-48-60 block counts at 46K tokens"),
+}

@@ -255,3 +255,55 @@ def test_paper_block_counts_fwd_bwd(mode):
                                                               blk, scale, dout[:, h], j)
             assert out_err(gk[keys, h], dk_ref, "bf16") <= TOL["bf16"]
             assert out_err(gv[keys, h], dv_ref, "bf16") <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", ["11520tok", "46080tok"])
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_paper_10_48_60_setting(name, mode):
+    """The pre-training runs' 10-48-60 block counts at 11K and 46K tokens
+    (latents chosen so the counts come out exactly; see synth.workloads):
+    full pair sets of two heads, then forward and dQ on sampled rows and
+    dK/dV on every key of the most- and least-selected block, on the
+    oracle's pairs."""
+    w = synth.PAPER_10_48_60[name]
+    nh, tau, scale = 2, 0.25, 1 / math.sqrt(128)
+    q, k, v = synth.make_qkv(w.wid, mode, w.T, w.H, w.W, nh, w.head_dim)
+    dout = synth.make_dout(w.wid, mode, w.s, nh, w.head_dim)
+    q, k, v, dout = (round_to(x, "bf16") for x in (q, k, v, dout))
+    sh = LayerShape(w.T, w.H, w.W, nh, w.head_dim, mode, *w.boxes[mode], "bf16")
+    L = VMoBALayer(sh)
+    assert L.n_blocks == (10, 48, 60)[mode]
+    qd = to_device(q, "bf16")
+    L.select(qd, to_device(k, "bf16"), to_device(v, "bf16"), tau)
+    torch.cuda.synchronize()
+    box = O.mode_box(mode, w.T, w.H, w.W, *w.boxes[mode])
+    B = O.pool_blocks(k, w.T, w.H, w.W, box)
+    blk = O.block_of_token(w.T, w.H, w.W, box)
+    bits = L.sel.cpu().numpy().copy()
+    g = unpack_bits(bits, L.n_blocks)
+    for h in range(nh):
+        S_h = O.block_scores(q[:, h:h + 1], B[h:h + 1], scale)[0]
+        m, st = O.threshold_select(S_h, tau)
+        assert pair_set_mismatch(g[h], S_h, m, st["cut_score"]) == 0
+        bits[h] = pack_bits(m)
+        g[h] = m
+    L.use_selection(torch.from_numpy(bits).cuda())
+    out, _ = L.forward(qd)
+    dq, dk, dv = L.backward(qd, to_device(dout, "bf16"))
+    torch.cuda.synchronize()
+    go, gq, gk, gv = from_device(out), from_device(dq), from_device(dk), from_device(dv)
+    for h in range(nh):
+        empty = np.flatnonzero(~g[h].any(axis=1))[:8]
+        rows = sample_rows(w.s, 96, seed=400 + h, must=empty)
+        o_ref, _ = O.attention_fwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows)
+        assert out_err(go[rows, h], o_ref, "bf16") <= TOL["bf16"]
+        dq_ref, _, _ = O.attention_bwd_rows(q[:, h], k[:, h], v[:, h], g[h], blk, scale, rows,
+                                            dout[rows, h])
+        assert out_err(gq[rows, h], dq_ref, "bf16") <= TOL["bf16"]
+        counts = g[h].sum(axis=0)
+        order = [j for j in np.argsort(counts, kind="stable") if counts[j] > 0]
+        for j in (int(np.argmax(counts)), order[0]):
+            keys, dk_ref, dv_ref = O.attention_bwd_block_keys(q[:, h], k[:, h], v[:, h], g[h],
+                                                              blk, scale, dout[:, h], j)
+            assert out_err(gk[keys, h], dk_ref, "bf16") <= TOL["bf16"]
+            assert out_err(gv[keys, h], dv_ref, "bf16") <= TOL["bf16"]
