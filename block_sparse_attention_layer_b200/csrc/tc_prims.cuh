@@ -215,6 +215,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// The same with fp16 A and B (format code 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor of a 128-byte-swizzled tile: start address,
 // leading / stride byte offsets (>> 4), version 1 at bits [46,48), layout
 // SWIZZLE_128B (2) at bits [61,64).  Tile bases are 1024-byte aligned, so the
@@ -306,6 +312,19 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
   return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+
+// Eight bf16 values (one 16-byte vector) as eight fp16 values, rounded to
+// nearest: exact for magnitudes in [2^-14, 65504] (bf16 carries 8
+// significant bits, fp16 11), gradual underflow below, inf above.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi);
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    o[k] = pack_f16x2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
