@@ -261,7 +261,9 @@ def run_ours(args, rank, world, local):
     hq, hk, hv, hdo = host_inputs(sample=job["sample"], heads=(h0, h1))
     gen_s = time.time() - t0
     q, k, v, dout = (x.cuda(non_blocking=False) for x in (hq, hk, hv, hdo))
-    layers = [VMoBALayer(sh) for sh in shapes]
+    # workspaces sized for the method's selection at tau (fewer than
+    # tau * s * N_b + 1 pairs per head)
+    layers = [VMoBALayer(sh, max_pair_fraction=TAU) for sh in shapes]
     stream = torch.cuda.current_stream()
 
     def one_step(events=None, only=None):
@@ -544,7 +546,7 @@ def paper_10_48_60(V, stream):
                                   kind=w.kind)
             dout = TL.make_dout(w.wid, mode, w.s, w.n_heads, w.head_dim)
             L = VMoBALayer(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode,
-                                      *w.boxes[mode], "bf16"))
+                                      *w.boxes[mode], "bf16"), max_pair_fraction=w.taus[0])
             ms = _time_layer_calls(V, L, q, k, v, w.taus[0], dout, stream)
             rec = _layer_record(V, L, ms, w.head_dim, True)
             rec.update(mode=mode, n_blocks=L.n_blocks, box=list(w.boxes[mode]))
@@ -589,7 +591,7 @@ def other_configs(V, stream):
                     dout = None
             sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *w.boxes[mode],
                             w.dtype)
-            L = VMoBALayer(sh)
+            L = VMoBALayer(sh, max_pair_fraction=max(w.taus))
             for tau in w.taus:
                 ms = _time_layer_calls(V, L, q, k, v, tau, dout, stream)
                 rec = _layer_record(V, L, ms, w.head_dim, dout is not None)
@@ -615,7 +617,7 @@ def stack_sweep(V, stream):
     from block_sparse_attention_layer_b200.layer import VMoBALayer
     w = synth.WORKLOADS[5]
     layers = [VMoBALayer(LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, m, *w.boxes[m],
-                                    "bf16")) for m in range(3)]
+                                    "bf16"), max_pair_fraction=max(w.taus)) for m in range(3)]
     out = {f"tau_{tau}": {"density": [], "ms_layer": [], "attn_tflops": []} for tau in w.taus}
     t0 = time.time()
     for layer in range(w.layers):
@@ -654,7 +656,7 @@ def paper_block_counts(V, w, tensors, stream, warm=2, reps=3):
            "ms_per_layer": [], "tflops": []}
     for mode, box in enumerate(synth.BOXES_8_48_72):
         sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *box, "bf16")
-        L = VMoBALayer(sh)
+        L = VMoBALayer(sh, max_pair_fraction=TAU)
 
         def layer():
             V.partition(L.shape, k, v, L.k_perm, L.v_perm, L.blocks)

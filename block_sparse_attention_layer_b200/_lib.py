@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
         "vmoba_mode_for_layer": (I, [I]),
         "vmoba_num_blocks": (I, [S]),
         "vmoba_workspace_size": (Z, [S]),
+        "vmoba_workspace_size_bounded": (Z, [S, ctypes.c_double]),
         "vmoba_bwd_workspace_size": (Z, [S]),
         "vmoba_partition": (I, [S, P, P, P, P, P, P]),
         "vmoba_score_select": (I, [S, P, P, F, F, P, P, P, Z, P]),
@@ -165,8 +166,13 @@ def num_blocks(shape: LayerShape) -> int:
     return n
 
 
-def workspace_size(shape: LayerShape) -> int:
-    return lib().vmoba_workspace_size(ctypes.byref(shape.c()))
+def workspace_size(shape: LayerShape, max_pair_fraction: float | None = None) -> int:
+    """Workspace bytes of a layer: for every pair selected, or (with
+    max_pair_fraction) for selections keeping at most that share of each
+    head's pool -- tau for the method's threshold selection."""
+    if max_pair_fraction is None:
+        return lib().vmoba_workspace_size(ctypes.byref(shape.c()))
+    return lib().vmoba_workspace_size_bounded(ctypes.byref(shape.c()), float(max_pair_fraction))
 
 
 def bwd_workspace_size(shape: LayerShape) -> int:
@@ -204,8 +210,8 @@ def _check_common(shape, q=None, k_perm=None, v_perm=None, sel_bits=None, ws=Non
         _expect(v_perm, (h, s, d), dt, "v_perm")
     if sel_bits is not None:
         _expect(sel_bits, (h, s, sel_words(shape)), torch.int32, "sel_bits")
-    if ws is not None and ws.numel() * ws.element_size() < workspace_size(shape):
-        raise ValueError("workspace smaller than vmoba_workspace_size")
+    if ws is not None and ws.numel() * ws.element_size() < workspace_size(shape, 1e-300):
+        raise ValueError("workspace smaller than the smallest vmoba_workspace_size_bounded")
 
 
 def score_select(shape, q, blocks, tau, scale, sel_bits, stats, ws, stream=None):

@@ -44,13 +44,34 @@ int make_prob(const vmoba_shape* sh, Prob* P) {
   p.Wb = (p.Nb + 31) / 32;
   p.n_qt = (p.s + kTile - 1) / kTile;
   p.Wqt = (p.n_qt + 31) / 32;
+  p.cap = (uint32_t)((long long)p.s * p.Nb);     // every pair of a head (at most)
   *P = p;
   return VMOBA_OK;
 }
 
-int check_ws(const Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
+// Pair slots per head that a workspace of ws_bytes holds: every pair of the
+// head if it fits, else the largest capacity whose layout fits (the layout
+// grows with the capacity), 0 if not even one pair does.  Every call of a
+// layer passes the same ws_bytes, so all derive the same layout.
+uint32_t fit_capacity(Prob P, size_t ws_bytes) {
+  const uint32_t full = P.cap;
+  if (ws_layout(P).total <= ws_bytes) return full;
+  uint32_t lo = 0, hi = full;
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo + 1) / 2;
+    P.cap = mid;
+    if (ws_layout(P).total <= ws_bytes) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Checks the workspace and fixes the layer's pair capacity from its size.
+int check_ws(Prob& P, const void* ws, size_t ws_bytes, WsLayout* L) {
+  if (!ws || !aligned16(ws)) return VMOBA_ERR_WORKSPACE;
+  const uint32_t cap = fit_capacity(P, ws_bytes);
+  if (cap == 0) return VMOBA_ERR_WORKSPACE;
+  P.cap = cap;
   *L = ws_layout(P);
-  if (!ws || ws_bytes < L->total || !aligned16(ws)) return VMOBA_ERR_WORKSPACE;
   return VMOBA_OK;
 }
 
@@ -73,10 +94,10 @@ ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
   ItemBufs b{};
   b.rows = item_rows_capacity(P);
   char* p = ws_ptr<char>(ws, L.items);
-  b.qg = reinterpret_cast<__half*>(p);
-  p += align_up(b.rows * P.d * sizeof(__half), 256);
-  b.dog = reinterpret_cast<__half*>(p);
-  p += align_up(b.rows * P.d * sizeof(__half), 256);
+  b.qg = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
+  b.dog = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
   b.l2g = reinterpret_cast<float*>(p);
   p += align_up(b.rows * sizeof(float), 256);
   b.dg = reinterpret_cast<float*>(p);
@@ -120,6 +141,18 @@ int vmoba_num_blocks(const vmoba_shape* shape) {
 size_t vmoba_workspace_size(const vmoba_shape* shape) {
   Prob P;
   if (make_prob(shape, &P) != VMOBA_OK) return 0;
+  return ws_layout(P).total;
+}
+
+size_t vmoba_workspace_size_bounded(const vmoba_shape* shape, double max_pair_fraction) {
+  Prob P;
+  if (make_prob(shape, &P) != VMOBA_OK) return 0;
+  if (!(max_pair_fraction > 0.0) || std::isnan(max_pair_fraction)) return 0;
+  // fraction of the pool, a relative margin for rounding in the selection's
+  // mass sums and a few pairs more; never beyond the whole pool
+  const double pool = (double)P.s * (double)P.Nb;
+  const double want = std::floor(max_pair_fraction * pool * (1.0 + 1e-4)) + 64.0;
+  if (want < pool) P.cap = (uint32_t)want;
   return ws_layout(P).total;
 }
 
@@ -358,9 +391,8 @@ int static_scratch(void** out) {
 }
 
 // The selection's part of the workspace layout, packed into the static array:
-// the device status word, the search state and histograms, and the bf16
-// split of the block means (bf16 inputs; their pool is recomputed, never
-// stored) or the fp32 score pool (fp32 inputs).
+// the device status word, the search state and histograms, the fp32 score
+// pool and, for bf16 inputs, the bf16 split of the block means.
 WsLayout static_select_layout(const Prob& P) {
   WsLayout w{};
   size_t off = 0;
@@ -369,10 +401,8 @@ WsLayout static_select_layout(const Prob& P) {
   w.sel_state = take(sizeof(SelState) * P.n_h);
   w.hist_count = take(sizeof(uint32_t) * kHistBins * P.n_h);
   w.hist_mass = take(sizeof(double) * kHistBins * P.n_h);
-  if (P.dtype == VMOBA_BF16)
-    w.bsplit = take(sel_split_bytes(P));
-  else
-    w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
+  w.scores = take(sizeof(float) * (size_t)P.n_h * P.s * P.Nb);
+  if (P.dtype == VMOBA_BF16) w.bsplit = take(sel_split_bytes(P));
   w.total = off;
   return w;
 }
@@ -398,8 +428,8 @@ int vmoba_score_select_static(const vmoba_shape* shape, const void* q, const flo
   if (scale <= 0.0f) scale = 1.0f / std::sqrt((float)P.d);
   const float tau_dev = tau >= 1.0f ? 2.0f : tau;
   // the first kernel of the selection clears the histograms and the search
-  // state; the split of B (or, for fp32 inputs, the score pool) is fully
-  // overwritten before it is read
+  // state; the score pool and the split of B are fully overwritten before
+  // they are read
   drop_stale_error();
   return cuda_status(launch_score_select(P, q, blocks, tau_dev, scale, sel_bits, stats, scratch,
                                          L, num_sms(), stream));

@@ -19,10 +19,13 @@
 //    block's list (tens of thousands in the large layers), and with P and
 //    dS rounded to bf16 (8 significant bits) the rounding alone moves
 //    them by more than 2e-2; fp16 (11 bits) keeps it near 1/8 of that.
-//    The K / V tile is converted in shared memory once per CTA and the
-//    query tiles come from fp16 item-ordered copies (exact conversions of
-//    the bf16 inputs within fp16's range, |x| <= 65504; P is in [0, 1] and
-//    dS = P (dP - D) must stay below 65504 too).
+//    The K / V tile is converted in shared memory once per CTA and each
+//    query tile as it lands (exact conversions of the bf16 inputs within
+//    fp16's range, |x| <= 65504; P is in [0, 1] and dS = P (dP - D) must
+//    stay below 65504 too).  Its D_i is the sum of P dP over the row's
+//    selected keys, accumulated by the dQ pass, not dO_i . O_i from the
+//    forward's output copy: dK sums D's error times P q over every query of
+//    the list, and the output copy carries the forward's bf16 P.
 // D_i comes from the forward's fp32 output copy.
 #include "tc_prims.cuh"
 #include "pairs.cuh"
@@ -79,14 +82,14 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
 
 // =====================================================================
 // dQ pass.  TMEM: S0 [0,128), S1 [128,256), dP [256,384) (then dS), dQ
-// [384,384+D).  Roles: warp 0 TMA (the block's K, V chunks), warps 2-3 the
-// item's Q and dO rows straight from the inputs (cp.async), warp 1 MMA,
-// warps 4-7 / 8-11 softmax of key columns 0-63 / 64-127 + epilogue.  Per chunk J the softmax forms P(J) from S(J) and frees S, then
+// [384,384+D).  Roles: warp 0 TMA (the item's Q and dO tiles from the
+// item-ordered copies, then the block's K, V chunks), warp 1 MMA, warps
+// 4-7 / 8-11 softmax of key columns 0-63 / 64-127 + epilogue (warps 2-3
+// idle).  Per chunk J the softmax forms P(J) from S(J) and frees S, then
 // dS(J) = P (dP - D) once dP(J) is there; the MMA issue order S(J+1),
 // dQ(J) += dS(J) K, dP(J+1) lets S(J+1) run while dS(J) is formed and
 // dP(J+1) while P(J+1) is.
 // =====================================================================
-constexpr int kGatherThreads = 64;            // warps 2-3 gather the query tiles
 struct DqBars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
   uint64_t s_full[2], s_free[2], dp_full, ds_full;
@@ -105,10 +108,10 @@ static_assert(dq_smem<128>() <= 232448, "shared memory per CTA");
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-             const __grid_constant__ CUtensorMap tm_pd, const __nv_bfloat16* __restrict__ q,
-             const __nv_bfloat16* __restrict__ dout, Prob P, int h, PairsView pv,
-             const float* __restrict__ rowD, const float* __restrict__ lse2, float sl2,
-             Watch wt) {
+             const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+             const __grid_constant__ CUtensorMap tm_pd, Prob P, int h, PairsView pv,
+             const float* __restrict__ dg, const float* __restrict__ l2g, float sl2,
+             float* __restrict__ part_d, Watch wt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -135,7 +138,7 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     }
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->ds_full, kSoftmaxWarps);
-    mbar_init(&bars->qd_full, kGatherThreads);
+    mbar_init(&bars->qd_full, 1);
     mbar_init(&bars->qd_empty, 1);
     mbar_init(&bars->dq_final, 1);
     mbar_init(&bars->dq_free, kSoftmaxWarps);
@@ -156,10 +159,19 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int J = 0, hint = 0;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_o);
+      int J = 0, it_local = 0, hint = 0;
       bool ok = true;
-      for (int n = blockIdx.x; n < n_items && ok; n += G) {
+      for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
         const WorkItem it = decode_item<false>(pv, P, h, n, hint);
+        if (it_local >= 1) ok = mbar_wait(&bars->qd_empty, (it_local - 1) & 1, wt, abort);
+        if (!ok) break;
+        mbar_expect_tx(&bars->qd_full, 2 * kTileB);
+        tma_load_2d(sQ, &tm_q, &bars->qd_full, 0, n * kTile);
+        if (D == 128) tma_load_2d(sQ + kHalf, &tm_q, &bars->qd_full, 64, n * kTile);
+        tma_load_2d(sO, &tm_o, &bars->qd_full, 0, n * kTile);
+        if (D == 128) tma_load_2d(sO + kHalf, &tm_o, &bars->qd_full, 64, n * kTile);
         for (int c = 0; c < nch && ok; ++c, ++J) {
           const int row = h * P.s + it.j * P.L + c * kTile;
           const int st = J & 1;
@@ -174,47 +186,14 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           tma_load_2d(sV + st * kTileB, &tm_v, &bars->full_v[st], 0, row);
           if (D == 128) tma_load_2d(sV + st * kTileB + kHalf, &tm_v, &bars->full_v[st], 64, row);
         }
+        if (ok && n + G < n_items) {
+          // the next item's Q / dO into L2 behind this item's loads (one buffer in smem)
+          for (int x = 0; x < D; x += 64) {
+            tma_prefetch_l2_2d(&tm_q, x, (n + G) * kTile);
+            tma_prefetch_l2_2d(&tm_o, x, (n + G) * kTile);
+          }
+        }
       }
-    }
-  } else if (warp == 2 || warp == 3) {
-    // The item's query rows of Q and dO straight from the inputs (one head's
-    // rows stay in L2): warp w copies rows [64 w, 64 w + 64) of both tiles,
-    // kRps rows per step (D / 8 lanes x 16 bytes per row), into the
-    // 128-byte-swizzled layout the MMA descriptors read (16-byte granule g of
-    // row r at g ^ (r & 7)); rows past the tile's queries are zero-filled.
-    constexpr int kLpr = D / 8, kRps = 32 / kLpr;     // lanes per row, rows per step
-    const int w = warp - 2, c = lane % kLpr, hr = lane / kLpr;
-    const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
-    const uint32_t qbase = smem_u32(sQ) + (c >> 3) * kHalf, obase = smem_u32(sO) + (c >> 3) * kHalf;
-    int hint = 0;
-    bool ok = true;
-    for (int n = blockIdx.x, it_local = 0; n < n_items && ok; n += G, ++it_local) {
-      const WorkItem m = decode_item<true>(pv, P, h, n, hint);
-      if (it_local >= 1)
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars->qd_empty, (it_local - 1) & 1, wt, abort));
-      if (!ok) break;
-      const int base = 64 * w;
-      const uint32_t idx0 = base + lane < m.count ? __ldg(col_rows + m.first + base + lane) : 0u;
-      const uint32_t idx1 =
-          base + 32 + lane < m.count ? __ldg(col_rows + m.first + base + 32 + lane) : 0u;
-#pragma unroll 4
-      for (int k = 0; k < 64 / kRps; ++k) {
-        const int rr = kRps * k + hr;               // row within the warp's 64
-        const uint32_t i0 = __shfl_sync(0xffffffffu, idx0, rr & 31);
-        const uint32_t i1 = __shfl_sync(0xffffffffu, idx1, rr & 31);
-        const int r = base + rr;
-        const bool in = r < m.count;
-        const uint32_t i = in ? (rr < 32 ? i0 : i1) : 0u;
-        const uint32_t off = r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        const size_t src = ((size_t)i * P.n_h + h) * D + c * 8;
-        cp_async16(qbase + off, q + src, in ? 16u : 0u);
-        cp_async16(obase + off, dout + src, in ? 16u : 0u);
-      }
-      // copies landed, made visible to the tensor core's (async) proxy
-      cp_async_wait_all();
-      fence_proxy_async();
-      mbar_arrive(&bars->qd_full);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -301,25 +280,22 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const uint64_t sl2x2 = f32x2(sl2, sl2);
     int J = 0, it_local = 0;
     bool ok = true;
-    // -LSE log2(e) and D of this thread's query in item nn (-inf and 0 past
-    // the tile's queries, so that P is exactly 0 there); loaded one item
-    // ahead, before the epilogue, so their latency is off the critical path
-    const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
-    int hint = 0;
+    // -LSE log2(e) and D of the row in item nn (the item-ordered copies hold
+    // -inf and 0 past the tile's queries); loaded one item ahead, before the
+    // epilogue, so their latency is off the critical path
     auto fetch = [&](int nn, float& l2, float& d) {
-      const WorkItem m = decode_item<true>(pv, P, h, nn, hint);
-      l2 = -INFINITY;
-      d = 0.f;
-      if (r < m.count) {
-        const uint32_t i = __ldg(col_rows + m.first + r);
-        l2 = __ldg(lse2 + (size_t)h * P.s + i);
-        d = __ldg(rowD + (size_t)h * P.s + i);
-      }
+      l2 = __ldg(l2g + (size_t)nn * kTile + r);
+      d = __ldg(dg + (size_t)nn * kTile + r);
     };
     float nx_l2 = -INFINITY, nx_d = 0.f;
     if (blockIdx.x < n_items) fetch(blockIdx.x, nx_l2, nx_d);
     for (int n = blockIdx.x; n < n_items && ok; n += G, ++it_local) {
       const uint64_t nl2x2 = f32x2(nx_l2, nx_l2), Dx2 = f32x2(nx_d, nx_d);
+      // sum of P dP over the group's keys of this block: the block's share of
+      // D_i = dO_i . O_i = sum_k P_ik dP_ik, exact to fp32 (the D used above
+      // comes from the forward's output copy); the dQ merge adds the shares
+      // up and the dK/dV pass uses that sum
+      uint64_t dacc = f32x2(0.f, 0.f);
       for (int c = 0; c < nch; ++c, ++J) {
         const int b = J & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, wt, abort));
@@ -368,10 +344,14 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             // dP past the chunk's keys is stale; P = 0 there must not meet it
             const uint64_t dd = sub_x2(f32x2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
                                        Dx2);
-            const float2 ds = f32x2_split(
-                mul_x2(f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1])), dd));
+            const uint64_t p2 = f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1]));
+            const float2 ds = f32x2_split(mul_x2(p2, dd));
             pk[e >> 1] = pack_bf16x2((full || x < lim) ? ds.x : 0.f,
                                      (full || x + 1 < lim) ? ds.y : 0.f);
+            dacc = fma_x2(p2,
+                          f32x2((full || x < lim) ? __uint_as_float(dp[e]) : 0.f,
+                                (full || x + 1 < lim) ? __uint_as_float(dp[e + 1]) : 0.f),
+                          dacc);
           }
           // dS into the group's columns [cb + 16 hh, +16): dP columns already read
           tmem_st16(tdP + lane_off + cb + hh * 16, pk);
@@ -383,6 +363,10 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       }
       if (!ok) break;
       if (n + G < n_items) fetch(n + G, nx_l2, nx_d);
+      {
+        const float2 dsum = f32x2_split(dacc);
+        part_d[((size_t)n * kTile + r) * 2 + wg] = dsum.x + dsum.y;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
@@ -428,13 +412,24 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 // (D / 32 dims per lane).  The partials sit at the pairs' item rows (slot_row).
 template <int D>
 __global__ void __launch_bounds__(256)
-k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, float scale,
-               __nv_bfloat16* __restrict__ dq) {
+k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq,
+               const float2* __restrict__ part_d, float scale, __nv_bfloat16* __restrict__ dq,
+               float* __restrict__ rowD) {
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (i >= P.s) return;
   const uint32_t off = __ldg(pv.row_off + (size_t)h * (P.s + 1) + i);
   const uint32_t cnt = __ldg(pv.row_cnt + (size_t)h * P.s + i);
-  const uint32_t* srow = pv.slot_row + (size_t)h * P.s * P.Nb + off;
+  const uint32_t* srow = pv.slot_row + (size_t)h * P.cap + off;
+  // D_i as the sum of the pass's P dP shares (lane-parallel over the pairs,
+  // then a warp sum), replacing the value computed from the output copy
+  float dsum = 0.f;
+  for (uint32_t k = lane; k < cnt; k += 32) {
+    const float2 v = part_d[__ldg(srow + k)];
+    dsum += v.x + v.y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  if (lane == 0 && cnt > 0) rowD[(size_t)h * P.s + i] = dsum;
   __nv_bfloat16* dst = dq + ((size_t)i * P.n_h + h) * D;
   if constexpr (D == 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -475,7 +470,7 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq, f
 // =====================================================================
 struct KvBars {
   uint64_t kv_full, kv_conv;           // K / V tile landed (bf16) / converted to fp16
-  uint64_t qd_full[2], qd_empty[2];
+  uint64_t qd_full[2], qd_conv[2], qd_empty[2];   // query tile landed / converted / free
   uint64_t st_full, dpt_full, p_full, ds_full;
   uint64_t acc_final;
   uint32_t tmem_base;
@@ -524,7 +519,11 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->kv_conv, 64);
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->qd_full[i], 1);
+      mbar_init(&bars->qd_conv[i], 64);
+      mbar_init(&bars->qd_empty[i], 1);
+    }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
     mbar_init(&bars->p_full, kSoftmaxWarps);
@@ -588,7 +587,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                  (g > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&bars->kv_conv, 0, wt, abort) &&
-                mbar_wait(&bars->qd_full[0], 0, wt, abort);
+                mbar_wait(&bars->qd_conv[0], 0, wt, abort);
       if (ok) {
         tc_fence_after();
         issue_ss(tS, kb, smem_u32(sQ));
@@ -604,7 +603,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc_fence_after();
         issue_acc(tV, tS, ob, g);                       // dV += P^T dO
         if (more) {
-          if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, wt, abort)) {
+          if (!mbar_wait(&bars->qd_conv[b ^ 1], ((g + 1) >> 1) & 1, wt, abort)) {
             ok = false;
             break;
           }
@@ -624,18 +623,30 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (ok) mma_commit(&bars->acc_final);
     }
   } else if (warp == 2 || warp == 3) {
-    // the K / V tile, once landed, to fp16 in place (the swizzled layout is a
-    // permutation of 16-byte granules, so converting granule by granule keeps
-    // it), then made visible to the tensor core's proxy
-    if (ng > 0) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->kv_full, 0, wt, abort));
-      if (ok) {
-        uint4* g = reinterpret_cast<uint4*>(sK);           // K then V: 2 * kTileB bytes
-        for (int x = threadIdx.x - 64; x < (int)(2 * kTileB / 16); x += 64)
-          g[x] = bf16x8_to_f16x8(g[x]);
-        fence_proxy_async();
-        mbar_arrive(&bars->kv_conv);
+    // operands to fp16 in place as they land: the K / V tile once, then each
+    // query tile's Q and dO (the swizzled layout is a permutation of 16-byte
+    // granules, so converting granule by granule keeps it), each made
+    // visible to the tensor core's proxy before its barrier
+    const int x0 = threadIdx.x - 64;
+    bool ok = ng > 0 && __all_sync(0xffffffffu, mbar_wait(&bars->kv_full, 0, wt, abort));
+    if (ok) {
+      uint4* gkv = reinterpret_cast<uint4*>(sK);             // K then V: 2 * kTileB bytes
+      for (int x = x0; x < (int)(2 * kTileB / 16); x += 64) gkv[x] = bf16x8_to_f16x8(gkv[x]);
+      fence_proxy_async();
+      mbar_arrive(&bars->kv_conv);
+    }
+    for (int g = 0; g < ng && ok; ++g) {
+      const int b = g & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, wt, abort));
+      if (!ok) break;
+      uint4* gq = reinterpret_cast<uint4*>(sQ + b * kTileB);
+      uint4* go = reinterpret_cast<uint4*>(sO + b * kTileB);
+      for (int x = x0; x < (int)(kTileB / 16); x += 64) {
+        gq[x] = bf16x8_to_f16x8(gq[x]);
+        go[x] = bf16x8_to_f16x8(go[x]);
       }
+      fence_proxy_async();
+      mbar_arrive(&bars->qd_conv[b]);
     }
   } else if (warp >= 4) {
     const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
@@ -647,8 +658,8 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool ok = true;
     for (int g = 0; g < ng && ok; ++g) {
       const int b = g & 1;
-      // qd_full also covers sL / sD of this tile
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, wt, abort));
+      // qd_conv follows qd_full, which also covers sL / sD of this tile
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_conv[b], (g >> 1) & 1, wt, abort));
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, wt, abort));
       if (!ok) break;
@@ -782,9 +793,13 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   CUtensorMap tk, tv, tq, to, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   float* part_dq = static_cast<float*>(part);
+  // the dQ pass's per-pair shares of D (two per item row), where the
+  // forward kept its (m, l)
+  float* part_d = reinterpret_cast<float*>(
+      static_cast<char*>(part) + align_up(item_rows_capacity(P) * D * sizeof(float), 256));
   if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
-      !make_tmap_2d(&tq, ib.qg, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
-      !make_tmap_2d(&to, ib.dog, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
+      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, D, 128) ||
+      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, D, 128) ||
       !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), D,
                     32, 32))
     return cudaErrorInvalidValue;
@@ -815,14 +830,18 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
       k_bwd_dq_blk<D><<<num_sms, kThreads, dq_smem<D>(), st>>>(
-          tk, tv, tpd, static_cast<const __nv_bfloat16*>(q),
-          static_cast<const __nv_bfloat16*>(dout), P, h, pv, rowD, lse2, sl2, make_watch(status));
+          tk, tv, tq, to, tpd, P, h, pv, ib.dg, ib.l2g, sl2, part_d, make_watch(status));
     }
     {
       VMOBA_TRACE("k_bwd_dq_merge", st);
-      k_bwd_dq_merge<D><<<(P.s + 7) / 8, 256, 0, st>>>(P, h, pv, part_dq, scale,
-                                                       static_cast<__nv_bfloat16*>(dq));
+      k_bwd_dq_merge<D><<<(P.s + 7) / 8, 256, 0, st>>>(
+          P, h, pv, part_dq, reinterpret_cast<const float2*>(part_d), scale,
+          static_cast<__nv_bfloat16*>(dq), rowD);
     }
+    // the exact D of this head into item order for the dK/dV pass
+    e = launch_gather_items(P, h, pv, nullptr, nullptr, nullptr, nullptr, lse2, rowD, ib.l2g,
+                            ib.dg, -INFINITY, num_sms, st);
+    if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dkdv_blk", st);
       k_bwd_dkdv_blk<D><<<P.Nb * nkt, kThreads, kv_smem<D>(), st>>>(
@@ -830,7 +849,7 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
           static_cast<__nv_bfloat16*>(dv), make_watch(status));
     }
   }
-  count_launches(1 + 3 * P.n_h);
+  count_launches(1 + 4 * P.n_h);
   return cudaGetLastError();
 }
 

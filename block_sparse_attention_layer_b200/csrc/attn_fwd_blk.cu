@@ -212,7 +212,7 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
     // rows past the tile's queries are zero-filled.
     constexpr int kLpr = D / 8, kRps = 32 / kLpr;     // lanes per row, rows per step
     const int w = warp - 2, c = lane % kLpr, hr = lane / kLpr;
-    const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
+    const uint32_t* col_rows = pv.col_rows + (size_t)h * P.cap;
     const uint32_t qbase = smem_u32(sQ);
     int it_local = 0, hint = 0;
     bool ok = true;
@@ -448,7 +448,7 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
   if (i >= P.s) return;
   const uint32_t off = __ldg(pv.row_off + (size_t)h * (P.s + 1) + i);
   const uint32_t cnt = __ldg(pv.row_cnt + (size_t)h * P.s + i);
-  const uint32_t* srow = pv.slot_row + (size_t)h * P.s * P.Nb + off;
+  const uint32_t* srow = pv.slot_row + (size_t)h * P.cap + off;
   // lane k takes pairs k, k + 32, ...: item rows and (m, l) are loaded
   // lane-parallel and broadcast to the warp by shuffles
   uint32_t row0 = 0u;

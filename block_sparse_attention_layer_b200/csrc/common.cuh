@@ -32,6 +32,7 @@ struct Prob {
   int Wb;                           // bitmap words per query row
   int n_qt;                         // 128-row tiles (queries and keys alike)
   int Wqt;                          // words of a tile bitmap (ceil(n_qt/32))
+  uint32_t cap;                     // (query, block) pair slots per head in the workspace
 };
 
 // Original token of partition position p.

@@ -1,12 +1,11 @@
-// Item-ordered copies of the rows the dK/dV pass reads as tiles.
+// Item-ordered copies of the rows the backward kernels read as tiles.
 //
 // Work item n of a head (block j, query tile g of block j's list) covers rows
 // [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
-// rows past the list end are zero.  The dK/dV pass re-reads every query tile
-// of a block once per key tile, so it fetches them with plain 2-D TMA from
-// these copies instead of scattered loads; Q and dO are stored in fp16 (the
-// bf16 inputs converted, exact within fp16's range), the operand type of its
-// MMAs.  The forward and the dQ pass gather their own query rows.  One warp per item; D / 8
+// rows past the list end are zero.  The backward kernels (dQ pass, dK/dV
+// pass) then fetch query tiles with plain 2-D TMA instead of scattered
+// loads; the forward gathers its own query rows from Q.  With no row source
+// (a == nullptr) only the per-row values are rewritten.  One warp per item; D / 8
 // lanes x 16 bytes move a row of head_dim D, 8 instructions in flight.
 #include "tc_prims.cuh"
 #include "pairs.cuh"
@@ -19,11 +18,11 @@ constexpr int kInFlight = 8;             // warp instructions in flight per batc
 template <int D>
 __global__ void __launch_bounds__(256)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
-               const __nv_bfloat16* __restrict__ b, __half* __restrict__ ag,
-               __half* __restrict__ bg, const float* __restrict__ fa,
+               const __nv_bfloat16* __restrict__ b, __nv_bfloat16* __restrict__ ag,
+               __nv_bfloat16* __restrict__ bg, const float* __restrict__ fa,
                const float* __restrict__ fb, float* __restrict__ fag, float* __restrict__ fbg,
                float fa_pad) {
-  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.s * P.Nb;
+  const uint32_t* col_rows = pv.col_rows + (size_t)h * P.cap;
   const int n_items = (int)__ldg(pv.head_totals + 4 * h + 1);
   const int lane = threadIdx.x & 31;
   constexpr int kLpr = D / 8, kRpi = 32 / kLpr;  // lanes per row, rows per instruction
@@ -35,7 +34,7 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
     const int count = it.count;
     const uint32_t* rows = col_rows + it.first;
     const size_t base = (size_t)n * kTile;
-    for (int r0 = 0; r0 < kTile; r0 += kRpi * kInFlight) {
+    for (int r0 = 0; a != nullptr && r0 < kTile; r0 += kRpi * kInFlight) {
       uint4 va[kInFlight], vb[kInFlight];
 #pragma unroll
       for (int u = 0; u < kInFlight; ++u) {
@@ -51,8 +50,8 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
 #pragma unroll
       for (int u = 0; u < kInFlight; ++u) {
         const size_t dst = (base + r0 + kRpi * u + half) * D;
-        reinterpret_cast<uint4*>(ag + dst)[c] = tc::bf16x8_to_f16x8(va[u]);
-        if (b) reinterpret_cast<uint4*>(bg + dst)[c] = tc::bf16x8_to_f16x8(vb[u]);
+        reinterpret_cast<uint4*>(ag + dst)[c] = va[u];
+        if (b) reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
       }
     }
     if (fa) {
@@ -74,12 +73,12 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
 
 size_t item_rows_capacity(const Prob& P) {
   // at most one partial tile per block beyond the pairs themselves
-  return (size_t)P.s * P.Nb + (size_t)kTile * P.Nb;
+  return (size_t)P.cap + (size_t)kTile * P.Nb;
 }
 
 cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 const __nv_bfloat16* a, const __nv_bfloat16* b,
-                                __half* ag, __half* bg, const float* fa,
+                                __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st) {
   {
@@ -101,7 +100,7 @@ namespace vmoba {
 
 size_t item_bufs_bytes(const Prob& P) {
   const size_t rows = item_rows_capacity(P);
-  return 2 * align_up(rows * P.d * sizeof(__half), 256) +
+  return 2 * align_up(rows * P.d * sizeof(__nv_bfloat16), 256) +
          2 * align_up(rows * sizeof(float), 256);
 }
 

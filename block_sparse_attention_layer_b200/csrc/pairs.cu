@@ -87,10 +87,11 @@ __device__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh, uint32_t* total) {
 // One CTA (1024 threads) per head: column totals and offsets, chunk bases,
 // work-item offsets, and the row offsets (CSR).
 __global__ void __launch_bounds__(1024)
-k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict__ chunk_cnt,
+k_pairs_scan(Prob P, uint32_t* __restrict__ row_cnt, uint32_t* __restrict__ chunk_cnt,
              int n_chunks, uint32_t* __restrict__ row_off, uint32_t* __restrict__ col_off,
              uint32_t* __restrict__ item_off, uint32_t* __restrict__ pitem_off,
-             uint32_t* __restrict__ head_totals, uint32_t* __restrict__ blk_order) {
+             uint32_t* __restrict__ head_totals, uint32_t* __restrict__ blk_order,
+             int* __restrict__ status) {
   __shared__ uint32_t sh[32];
   __shared__ uint32_t len[kMaxBlocks];
   const int h = blockIdx.x, t = threadIdx.x;
@@ -101,6 +102,28 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
     for (int c = 0; c < n_chunks; ++c) tot += cc[(size_t)c * P.Nb + t];
   uint32_t all;
   const uint32_t off = block_excl_scan(t < P.Nb ? tot : 0u, sh, &all);
+  if (all > P.cap) {
+    // more pairs than the workspace holds: the head is left empty (every
+    // count and offset 0, so the attention kernels do nothing for it and its
+    // outputs are zero) and the device status word says why
+    for (int j = t; j <= P.Nb; j += blockDim.x) {
+      col_off[(size_t)h * (P.Nb + 1) + j] = 0u;
+      item_off[(size_t)h * (P.Nb + 1) + j] = 0u;
+      pitem_off[(size_t)h * (P.Nb + 1) + j] = 0u;
+      if (j < P.Nb) blk_order[(size_t)h * P.Nb + j] = (uint32_t)j;
+    }
+    for (int i = t; i < P.s; i += blockDim.x) {
+      row_cnt[(size_t)h * P.s + i] = 0u;
+      row_off[(size_t)h * (P.s + 1) + i] = 0u;
+    }
+    if (t == 0) {
+      row_off[(size_t)h * (P.s + 1) + P.s] = 0u;
+      head_totals[4 * h] = head_totals[4 * h + 1] = head_totals[4 * h + 2] = 0u;
+      head_totals[4 * h + 3] = 1u;             // overflow: k_pairs_fill skips the head
+      atomicExch(status, (int)VMOBA_ERR_WORKSPACE);
+    }
+    return;
+  }
   const uint32_t tiles = t < P.Nb ? (tot + kTile - 1) / kTile : 0u;
   uint32_t n_items, n_pitems;
   const uint32_t ioff = block_excl_scan(tiles, sh, &n_items);
@@ -152,16 +175,18 @@ k_pairs_scan(Prob P, const uint32_t* __restrict__ row_cnt, uint32_t* __restrict_
 // blocks below j it selected).
 __global__ void __launch_bounds__(kChunkRows)
 k_pairs_fill(Prob P, const uint32_t* __restrict__ sel, const uint32_t* __restrict__ chunk_base,
-             int n_chunks, const uint32_t* __restrict__ row_off,
+             const uint32_t* __restrict__ head_totals, int n_chunks,
+             const uint32_t* __restrict__ row_off,
              const uint32_t* __restrict__ col_off, const uint32_t* __restrict__ item_off,
              uint32_t* __restrict__ col_rows, uint32_t* __restrict__ slot_row) {
   __shared__ uint32_t wcnt[kChunkRows / 32][32];
   const int c = blockIdx.x, h = blockIdx.y;
+  if (head_totals[4 * h + 3] != 0u) return;      // the head overflowed the workspace
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = c * kChunkRows + threadIdx.x;
   const uint32_t* cb = chunk_base + ((size_t)h * n_chunks + c) * P.Nb;
-  uint32_t* rows = col_rows + (size_t)h * P.s * P.Nb;
-  uint32_t* srow = slot_row + (size_t)h * P.s * P.Nb;
+  uint32_t* rows = col_rows + (size_t)h * P.cap;
+  uint32_t* srow = slot_row + (size_t)h * P.cap;
   const uint32_t* coff = col_off + (size_t)h * (P.Nb + 1);
   const uint32_t* ioff = item_off + (size_t)h * (P.Nb + 1);
   uint32_t slot = (i < P.s) ? __ldg(row_off + (size_t)h * (P.s + 1) + i) : 0u;
@@ -211,8 +236,8 @@ size_t pairs_ws_bytes(const Prob& P) {
   take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));          // pitem_off
   take(sizeof(uint32_t) * 4 * P.n_h);                           // head totals
   take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);     // chunk counts / bases
-  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // col_rows (worst case)
-  take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);          // slot_row (worst case)
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.cap);               // col_rows
+  take(sizeof(uint32_t) * (size_t)P.n_h * P.cap);               // slot_row
   take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);                // blk_order
   return b;
 }
@@ -229,14 +254,15 @@ PairsView pairs_view(const Prob& P, void* base) {
   v.pitem_off = take(sizeof(uint32_t) * (size_t)P.n_h * (P.Nb + 1));
   v.head_totals = take(sizeof(uint32_t) * 4 * P.n_h);
   v.chunk = take(sizeof(uint32_t) * (size_t)P.n_h * n_chunks * P.Nb);
-  v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
-  v.slot_row = take(sizeof(uint32_t) * (size_t)P.n_h * P.s * P.Nb);
+  v.col_rows = take(sizeof(uint32_t) * (size_t)P.n_h * P.cap);
+  v.slot_row = take(sizeof(uint32_t) * (size_t)P.n_h * P.cap);
   v.blk_order = take(sizeof(uint32_t) * (size_t)P.n_h * P.Nb);
   v.n_chunks = n_chunks;
   return v;
 }
 
-cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, cudaStream_t st) {
+cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, int* status,
+                         cudaStream_t st) {
   dim3 g(v.n_chunks, P.n_h);
   {
     VMOBA_TRACE("k_pairs_count", st);
@@ -245,11 +271,13 @@ cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v,
   {
     VMOBA_TRACE("k_pairs_scan", st);
     k_pairs_scan<<<P.n_h, 1024, 0, st>>>(P, v.row_cnt, v.chunk, v.n_chunks, v.row_off, v.col_off,
-                                         v.item_off, v.pitem_off, v.head_totals, v.blk_order);
+                                         v.item_off, v.pitem_off, v.head_totals, v.blk_order,
+                                         status);
   }
   {
     VMOBA_TRACE("k_pairs_fill", st);
-    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.n_chunks, v.row_off, v.col_off,
+    k_pairs_fill<<<g, kChunkRows, 0, st>>>(P, sel, v.chunk, v.head_totals, v.n_chunks, v.row_off,
+                                           v.col_off,
                                            v.item_off, v.col_rows, v.slot_row);
   }
   count_launches(3);

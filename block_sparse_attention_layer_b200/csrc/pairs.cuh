@@ -96,11 +96,10 @@ __device__ __forceinline__ WorkItem decode_item_pair(const PairsView& pv, const 
   return a;
 }
 
-// Item-ordered copies (gather.cu) for the dK/dV pass: fp16 rows of Q and dO
-// (the bf16 inputs converted; exact within fp16's range), fp32 -LSE*log2e and D.
+// Item-ordered copies (gather.cu): bf16 rows of Q and dO, fp32 -LSE*log2e and D.
 struct ItemBufs {
-  __half* qg;
-  __half* dog;
+  __nv_bfloat16* qg;
+  __nv_bfloat16* dog;
   float* l2g;
   float* dg;
   size_t rows;   // capacity
@@ -108,7 +107,10 @@ struct ItemBufs {
 
 size_t pairs_ws_bytes(const Prob& P);
 PairsView pairs_view(const Prob& P, void* base);
-cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, cudaStream_t st);
+// Builds the pair lists; a head with more pairs than P.cap is left empty and
+// VMOBA_ERR_WORKSPACE is latched in *status.
+cudaError_t launch_pairs(const Prob& P, const uint32_t* sel, const PairsView& v, int* status,
+                         cudaStream_t st);
 
 cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp,
                                 const uint32_t* sel, const PairsView& pv, void* part,
@@ -118,7 +120,7 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
 size_t item_rows_capacity(const Prob& P);
 cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 const __nv_bfloat16* a, const __nv_bfloat16* b,
-                                __half* ag, __half* bg, const float* fa,
+                                __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st);
 

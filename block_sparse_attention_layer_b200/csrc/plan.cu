@@ -109,7 +109,8 @@ cudaError_t launch_plan(const Prob& P, const uint32_t* sel, void* ws, const WsLa
   count_launches(tiles ? 2 : 1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_pairs(P, sel, pairs_view(P, ws_ptr<char>(ws, L.pairs)), st);
+  return launch_pairs(P, sel, pairs_view(P, ws_ptr<char>(ws, L.pairs)), ws_ptr<int>(ws, L.status),
+                      st);
 }
 
 }  // namespace vmoba

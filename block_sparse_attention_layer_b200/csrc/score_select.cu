@@ -543,9 +543,10 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
     return cudaGetLastError();
   };
 
-  if (P.dtype == VMOBA_BF16 && rownorm) {
-    // the per-query normalisation needs whole rows: the pool is written once
-    // by the tensor cores and the passes read it (the fp32 path below)
+  if (P.dtype == VMOBA_BF16) {
+    // the tensor cores write the pool (and each head's max) once; the radix
+    // passes below read it with many CTAs per SM, whose shared-memory
+    // histogram atomics hide each other's latency
     SelPassOps ops{};
     ops.st = st;
     ops.pool = ws_ptr<float>(ws, L.scores);
@@ -556,21 +557,7 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
     e = launch_score_passes_tc(P, q, blocks, scale, ops, stream);
     if (e != cudaSuccess) return e;
   }
-  if (P.dtype == VMOBA_BF16 && !rownorm) {
-    // tensor-core passes over the recomputed pool (score_tc.cu)
-    SelPassOps ops{};
-    ops.st = st;
-    ops.hc = hc;
-    ops.hm = hm;
-    ops.sel = sel;
-    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
-    ops.status = ws_ptr<int>(ws, L.status);
-    ops.num_sms = num_sms;
-    ops.scan = scan;
-    ops.tie_scan = tie_scan;
-    e = launch_score_passes_tc(P, q, blocks, scale, ops, stream);
-    if (e != cudaSuccess) return e;
-  } else {
+  {
     // fp32 I/O: the pool is computed once with fp32 FMAs and read by each
     // pass (bf16 with the per-query normalisation: written above)
     float* S = ws_ptr<float>(ws, L.scores);
@@ -581,6 +568,12 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
       ++launches;
     }
     if (rownorm) {
+      // the max of the normalised pool replaces the raw one
+      {
+        VMOBA_TRACE("k_init", stream);
+        k_init<<<64, 256, 0, stream>>>(st, hc, hm, P.n_h);
+      }
+      ++launches;
       VMOBA_TRACE("k_rownorm", stream);
       k_rownorm<<<(unsigned)(((size_t)P.n_h * P.s + 7) / 8), 256, 0, stream>>>(P, S, st);
       ++launches;

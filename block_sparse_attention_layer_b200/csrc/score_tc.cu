@@ -20,7 +20,7 @@
 //   kTie0..2    count-only radix histogram of the flat index i*N_b + j of the
 //               elements whose key equals the cut (exact ties);
 //   kEmit       the selection bitmap, one 32-bit word per 32 blocks of a row;
-//   kPool       S itself, written to the workspace pool (selection variants).
+//   kPool       S itself, written to the workspace pool, and the head max.
 // The digit walks between passes are the one-warp scans of score_select.cu.
 //
 // Persistent CTAs, cph per head (CTA b: head b / cph, query tiles b % cph,
@@ -286,6 +286,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 word |= (on ? 1u : 0u) << e;
               } else {                                         // kPool
                 pool[((size_t)h * P.s + i) * P.Nb + j] = x;
+                vmax = fmaxf(vmax, x);
               }
             }
             if (PASS == kEmit && row_ok)
@@ -313,7 +314,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
     }
     if (kTie && ok) ok = epi_sync(&bars->adds_done, n_sync);
-    if (PASS == kMax) {
+    if (PASS == kMax || PASS == kPool) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
       if (lane == 0 && vmax > -INFINITY) atomicMax(&st[h].max_key, f2key(vmax));

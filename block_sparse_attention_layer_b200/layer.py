@@ -16,7 +16,10 @@ from ._lib import LayerShape
 class VMoBALayer:
     """Buffers + calls for one layer shape (reusable across steps)."""
 
-    def __init__(self, shape: LayerShape, device="cuda"):
+    def __init__(self, shape: LayerShape, device="cuda", max_pair_fraction=None):
+        """max_pair_fraction: size the workspace for selections keeping at
+        most that share of each head's pairs (tau for the method's threshold
+        selection); None sizes it for every pair."""
         self.shape = shape
         s, h, d = shape.s, shape.n_heads, shape.head_dim
         dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
@@ -31,7 +34,8 @@ class VMoBALayer:
         self.sel = torch.empty((h, s, (nb + 31) // 32), dtype=torch.int32, device=dev)
         self.stats = torch.empty((h * _lib.HEAD_STATS_DTYPE.itemsize,), dtype=torch.uint8,
                                  device=dev)
-        self.ws = torch.empty((_lib.workspace_size(shape),), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty((_lib.workspace_size(shape, max_pair_fraction),), dtype=torch.uint8,
+                              device=dev)
         self.ws_bwd = torch.empty((_lib.bwd_workspace_size(shape),), dtype=torch.uint8,
                                   device=dev)
         self.out = torch.empty((s, h, d), dtype=dt, device=dev)

@@ -100,8 +100,25 @@ int vmoba_mode_for_layer(int layer_idx);
 int vmoba_num_blocks(const vmoba_shape* shape);
 
 /* Bytes of workspace for score_select / build_plan / attn_fwd / attn_bwd
- * (one buffer serves them all), or 0 for an invalid shape. */
+ * (one buffer serves them all), or 0 for an invalid shape.  This size holds
+ * the pair lists and per-pair buffers for every (query, block) pair of every
+ * head being selected. */
 size_t vmoba_workspace_size(const vmoba_shape* shape);
+
+/* The same for selections that keep at most max_pair_fraction of each head's
+ * s x N_b pairs (plus a small margin), or 0 for an invalid shape or a
+ * fraction <= 0 / NaN; at or above the whole pool it equals
+ * vmoba_workspace_size.  The method's threshold selection keeps fewer than
+ * tau * s * N_b + 1 pairs per head (the cumulative rule stops within the
+ * first tau of the mass, and the sorted prefix carries at least its share of
+ * it), so max_pair_fraction = tau suffices for it; top-k global needs k /
+ * (s N_b); the local variants can keep more.  Every call of a layer derives
+ * the pair capacity from the ws_bytes it is given (the largest the buffer
+ * holds).  If a selection keeps more pairs in a head than that capacity,
+ * vmoba_build_plan leaves the head empty (its attention outputs and
+ * gradients are zero) and latches VMOBA_ERR_WORKSPACE in the device status
+ * word (vmoba_get_status); nothing is read or written past the buffers. */
+size_t vmoba_workspace_size_bounded(const vmoba_shape* shape, double max_pair_fraction);
 
 /* Bytes of the extra backward workspace (row terms D = rowsum(dO*O)), or 0. */
 size_t vmoba_bwd_workspace_size(const vmoba_shape* shape);
@@ -235,6 +252,19 @@ int vmoba_debug_set_wait(long long wait_cycles, int skip_forward_loads);
  * engine that has pooled all device memory at start-up and forbids later
  * cudaMalloc, or a plugin that is given no allocator.  This entry point has
  * no counterpart in the paper: it only changes where scratch memory lives.
+ * - The array is committed on a device when the CUDA runtime loads the
+ *   library's device code there.  With lazy module loading (the CUDA 12
+ *   default) that can happen at this entry point's first call on the
+ *   device, so make one warm-up call on each device before reserving a
+ *   memory pool that leaves no room for 16 MiB; the array then stays
+ *   committed until the process exits.
+ * - Problems whose scratch exceeds VMOBA_STATIC_SELECT_SCRATCH_BYTES return
+ *   VMOBA_ERR_WORKSPACE without launching anything.  The scratch is the fp32
+ *   score pool (4*n_heads*s*N_b bytes), for bf16 inputs the bf16 hi / lo
+ *   split of the block means (4 * n_heads * N_b' * head_dim bytes, N_b' =
+ *   N_b rounded up to 128), and about 24.6 KB per head of histograms and
+ *   search state; e.g. 4 heads x 2048 tokens x 64 blocks (2.2 MB) fits,
+ *   12 heads x 55296 tokens x 24 blocks (64 MB) does not.
  * - The array is committed on a device when the CUDA runtime loads the
  *   library's device code there.  With lazy module loading (the CUDA 12
  *   default) that can happen at this entry point's first call on the

@@ -132,17 +132,21 @@ def test_selection_variant_arguments_rejected(variant, param):
 
 
 def test_small_workspace_rejected():
+    # below the smallest layout (one pair slot per head) every call refuses;
+    # between that and the every-pair size the calls derive a smaller pair
+    # capacity from ws_bytes instead
     sh = _shape()
-    need = V.workspace_size(sh)
+    assert 0 < V.workspace_size(sh, 1e-300) < V.workspace_size(sh)
+    tiny = 4096                           # holds not even the fixed part of the layout
     L = V.lib()
     rc = L.vmoba_score_select(ctypes.byref(sh.c()), BAD, BAD, 0.5, 0.0, BAD, BAD, BAD,
-                              need - 1, None)
+                              tiny, None)
     assert rc == -4
-    rc = L.vmoba_build_plan(ctypes.byref(sh.c()), BAD, None, need, None)
-    assert rc == -4
-    rc = L.vmoba_attn_bwd(ctypes.byref(sh.c()), BAD, BAD, BAD, BAD, BAD, need, 0.0, BAD,
-                          BAD, BAD, BAD, BAD, BAD, 0, None)
-    assert rc == -4
+    rc = L.vmoba_build_plan(ctypes.byref(sh.c()), BAD, None, V.workspace_size(sh), None)
+    assert rc == -4                       # no workspace pointer
+    rc = L.vmoba_attn_bwd(ctypes.byref(sh.c()), BAD, BAD, BAD, BAD, BAD, V.workspace_size(sh),
+                          0.0, BAD, BAD, BAD, BAD, BAD, BAD, 0, None)
+    assert rc == -4                       # backward workspace missing
 
 
 def test_status_strings():
@@ -165,3 +169,20 @@ def test_full_attention_steps_of_the_training_strategy():
     from block_sparse_attention_layer_b200.attention import full_attention_steps
     assert full_attention_steps(50) == 13 and full_attention_steps(40) == 10
     assert full_attention_steps(1) == 1 and full_attention_steps(8, 0.0) == 0
+
+
+@pytest.mark.parametrize("wid", [3, 4, 5])
+def test_bounded_workspace_sizes(wid):
+    """A workspace sized for the method's selection at tau holds a quarter of
+    the pairs: much smaller than the every-pair size, monotone in the
+    fraction, equal to it at the whole pool, invalid fractions give 0."""
+    w = WORKLOADS[wid]
+    sh = V.LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, 2, *w.boxes[2], w.dtype)
+    full = V.workspace_size(sh)
+    sizes = [V.workspace_size(sh, f) for f in (0.05, 0.1, 0.25, 0.5, 1.0, 3.0)]
+    assert sizes == sorted(sizes)
+    assert sizes[-2] == sizes[-1] == full
+    assert sizes[2] < 0.5 * full
+    L = V.lib()
+    for bad in (0.0, -1.0, float("nan")):
+        assert L.vmoba_workspace_size_bounded(ctypes.byref(sh.c()), bad) == 0

@@ -143,3 +143,47 @@ def test_guard_bands_around_outputs_and_workspace(mode, box, d):
     assert out_err(from_device(b["dq"]), dq_ref, "bf16") <= TOL["bf16"]
     assert out_err(from_device(b["dk"]), dk_ref, "bf16") <= TOL["bf16"]
     assert out_err(from_device(b["dv"]), dv_ref, "bf16") <= TOL["bf16"]
+
+
+def _layer_run(sh, q, k, v, dout, tau, frac):
+    L = VMoBALayer(sh, max_pair_fraction=frac)
+    qd = to_device(q, "bf16")
+    L.step(qd, to_device(k, "bf16"), to_device(v, "bf16"), tau, dout=to_device(dout, "bf16"))
+    torch.cuda.synchronize()
+    return L
+
+
+@pytest.mark.parametrize("mode,box", [(0, (1, 16, 16)), (2, (2, 4, 4))])
+def test_workspace_sized_for_tau_gives_the_same_results(mode, box):
+    """A workspace sized for the method's selection at tau (a quarter of the
+    pairs) derives a smaller pair capacity from its size; every output equals
+    the every-pair workspace's bit for bit."""
+    q, k, v, dout = _inputs(190 + mode)
+    sh = LayerShape(T, H, W, NH, D, mode, *box, "bf16")
+    tau = 0.25
+    assert _lib.workspace_size(sh, tau) < _lib.workspace_size(sh)
+    a = _layer_run(sh, q, k, v, dout, tau, None)
+    b = _layer_run(sh, q, k, v, dout, tau, tau)
+    assert _lib.get_status(b.ws) == 0
+    for name in ("sel", "out", "lse", "dq", "dk", "dv"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_selection_beyond_the_workspace_is_refused_on_the_device():
+    """A workspace sized for 1 % of the pairs given a selection that keeps
+    ~40 %: the plan leaves every head empty and latches VMOBA_ERR_WORKSPACE;
+    nothing is written past the buffers (outputs zero, LSE -inf) and the
+    context stays usable for a correct call."""
+    q, k, v, dout = _inputs(195)
+    sh = LayerShape(T, H, W, NH, D, 0, 1, 16, 16, "bf16")
+    L = _layer_run(sh, q, k, v, dout, 0.4, 0.01)
+    assert _lib.get_status(L.ws) == -4           # VMOBA_ERR_WORKSPACE
+    assert not L.out.any() and not L.dq.any() and not L.dk.any() and not L.dv.any()
+    assert torch.isneginf(L.lse).all()
+    good = _layer_run(sh, q, k, v, dout, 0.4, 0.5)
+    assert _lib.get_status(good.ws) == 0
+    from tests.gpu_util import unpack_bits
+    g = unpack_bits(good.sel.cpu().numpy(), good.n_blocks)
+    blk = O.block_of_token(T, H, W, O.mode_box(0, T, H, W, 1, 16, 16))
+    o_ref, _ = O.attention_fwd(q, k, v, g, blk, 1 / math.sqrt(D))
+    assert out_err(from_device(good.out), o_ref, "bf16") <= TOL["bf16"]
