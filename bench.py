@@ -896,7 +896,7 @@ def run_profile_case(args):
     q, k, v, do = (torch.from_numpy(round_to(x, "bf16").astype(np.float32))
                    .to(torch.bfloat16).cuda() for x in (q, k, v, do))
     sh = LayerShape(w.T, w.H, w.W, nh, w.head_dim, mode, *w.boxes[mode], "bf16")
-    L = VMoBALayer(sh)
+    L = VMoBALayer(sh, max_pair_fraction=TAU)      # a few GB on the device at most
     times = []
     for _ in range(2):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
