@@ -98,6 +98,10 @@ ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
   p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
   b.dog = reinterpret_cast<__nv_bfloat16*>(p);
   p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
+  b.qh = reinterpret_cast<__half*>(p);
+  p += align_up(b.rows * P.d * sizeof(__half), 256);
+  b.doh = reinterpret_cast<__half*>(p);
+  p += align_up(b.rows * P.d * sizeof(__half), 256);
   b.l2g = reinterpret_cast<float*>(p);
   p += align_up(b.rows * sizeof(float), 256);
   b.dg = reinterpret_cast<float*>(p);

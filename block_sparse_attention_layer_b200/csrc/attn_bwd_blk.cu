@@ -19,10 +19,10 @@
 //    block's list (tens of thousands in the large layers), and with P and
 //    dS rounded to bf16 (8 significant bits) the rounding alone moves
 //    them by more than 2e-2; fp16 (11 bits) keeps it near 1/8 of that.
-//    The K / V tile is converted in shared memory once per CTA and each
-//    query tile as it lands (exact conversions of the bf16 inputs within
-//    fp16's range, |x| <= 65504; P is in [0, 1] and dS = P (dP - D) must
-//    stay below 65504 too).  Its D_i is the sum of P dP over the row's
+//    The K / V tile is converted in shared memory once per CTA and the
+//    query tiles come from fp16 item-ordered copies (exact conversions of
+//    the bf16 inputs within fp16's range, |x| <= 65504; P is in [0, 1] and
+//    dS = P (dP - D) must stay below 65504 too).  Its D_i is the sum of P dP over the row's
 //    selected keys, accumulated by the dQ pass, not dO_i . O_i from the
 //    forward's output copy: dK sums D's error times P q over every query of
 //    the list, and the output copy carries the forward's bf16 P.
@@ -470,7 +470,7 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq,
 // =====================================================================
 struct KvBars {
   uint64_t kv_full, kv_conv;           // K / V tile landed (bf16) / converted to fp16
-  uint64_t qd_full[2], qd_conv[2], qd_empty[2];   // query tile landed / converted / free
+  uint64_t qd_full[2], qd_empty[2];
   uint64_t st_full, dpt_full, p_full, ds_full;
   uint64_t acc_final;
   uint32_t tmem_base;
@@ -519,11 +519,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->kv_conv, 64);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->qd_full[i], 1);
-      mbar_init(&bars->qd_conv[i], 64);
-      mbar_init(&bars->qd_empty[i], 1);
-    }
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
     mbar_init(&bars->p_full, kSoftmaxWarps);
@@ -587,7 +583,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                  (g > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&bars->kv_conv, 0, wt, abort) &&
-                mbar_wait(&bars->qd_conv[0], 0, wt, abort);
+                mbar_wait(&bars->qd_full[0], 0, wt, abort);
       if (ok) {
         tc_fence_after();
         issue_ss(tS, kb, smem_u32(sQ));
@@ -603,7 +599,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc_fence_after();
         issue_acc(tV, tS, ob, g);                       // dV += P^T dO
         if (more) {
-          if (!mbar_wait(&bars->qd_conv[b ^ 1], ((g + 1) >> 1) & 1, wt, abort)) {
+          if (!mbar_wait(&bars->qd_full[b ^ 1], ((g + 1) >> 1) & 1, wt, abort)) {
             ok = false;
             break;
           }
@@ -623,10 +619,10 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (ok) mma_commit(&bars->acc_final);
     }
   } else if (warp == 2 || warp == 3) {
-    // operands to fp16 in place as they land: the K / V tile once, then each
-    // query tile's Q and dO (the swizzled layout is a permutation of 16-byte
-    // granules, so converting granule by granule keeps it), each made
-    // visible to the tensor core's proxy before its barrier
+    // the K / V tile to fp16 in place once it lands (the swizzled layout is a
+    // permutation of 16-byte granules, so converting granule by granule
+    // keeps it), made visible to the tensor core's proxy before its barrier;
+    // the query tiles arrive in fp16 from the item-ordered copies
     const int x0 = threadIdx.x - 64;
     bool ok = ng > 0 && __all_sync(0xffffffffu, mbar_wait(&bars->kv_full, 0, wt, abort));
     if (ok) {
@@ -634,19 +630,6 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       for (int x = x0; x < (int)(2 * kTileB / 16); x += 64) gkv[x] = bf16x8_to_f16x8(gkv[x]);
       fence_proxy_async();
       mbar_arrive(&bars->kv_conv);
-    }
-    for (int g = 0; g < ng && ok; ++g) {
-      const int b = g & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, wt, abort));
-      if (!ok) break;
-      uint4* gq = reinterpret_cast<uint4*>(sQ + b * kTileB);
-      uint4* go = reinterpret_cast<uint4*>(sO + b * kTileB);
-      for (int x = x0; x < (int)(kTileB / 16); x += 64) {
-        gq[x] = bf16x8_to_f16x8(gq[x]);
-        go[x] = bf16x8_to_f16x8(go[x]);
-      }
-      fence_proxy_async();
-      mbar_arrive(&bars->qd_conv[b]);
     }
   } else if (warp >= 4) {
     const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
@@ -658,14 +641,19 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool ok = true;
     for (int g = 0; g < ng && ok; ++g) {
       const int b = g & 1;
-      // qd_conv follows qd_full, which also covers sL / sD of this tile
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_conv[b], (g >> 1) & 1, wt, abort));
+      // qd_full also covers sL / sD of this tile
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[b], (g >> 1) & 1, wt, abort));
       if (!ok) break;
+      const float* NL = sL + b * kTile + cb;
+      const float* Dq = sD + b * kTile + cb;
+      // -LSE log2(e) of the first 32 query columns read ahead of the S^T wait
+      // (the other 32 are read as they are used; all 64 would spill)
+      float4 nlr[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) nlr[x] = *reinterpret_cast<const float4*>(NL + 4 * x);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, g & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
-      const float* NL = sL + b * kTile + cb;
-      const float* Dq = sD + b * kTile + cb;
       // P^T for the group's 64 query columns (kept in fp32 for dS^T);
       // rows of keys past the tile's end are computed but never stored
       uint32_t pr[64];
@@ -678,7 +666,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int x = hh * 32 + e;
-          const float4 nl = *reinterpret_cast<const float4*>(NL + x);
+          const float4 nl = hh == 0 ? nlr[x >> 2] : *reinterpret_cast<const float4*>(NL + x);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int y = x + 2 * u;
@@ -698,6 +686,10 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
+      // likewise D of the first 32 query columns, ahead of the dP^T wait
+      float4 ddr[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) ddr[x] = *reinterpret_cast<const float4*>(Dq + 4 * x);
       // dS^T = P^T (dP^T - D)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dpt_full, g & 1, wt, abort));
       if (!ok) break;
@@ -711,7 +703,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int x = hh * 32 + e;
-          const float4 dd = *reinterpret_cast<const float4*>(Dq + x);
+          const float4 dd = hh == 0 ? ddr[x >> 2] : *reinterpret_cast<const float4*>(Dq + x);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int y = e + 2 * u;
@@ -790,7 +782,7 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
                     const PairsView& pv, void* part, const ItemBufs& ib, const float* o32,
                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
                     void* ws_bwd, float scale, int* status, int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv, tq, to, tpd;
+  CUtensorMap tk, tv, tq, to, tqh, toh, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   float* part_dq = static_cast<float*>(part);
   // the dQ pass's per-pair shares of D (two per item row), where the
@@ -800,6 +792,8 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
       !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, D, 128) ||
       !make_tmap_bf16_2d(&to, ib.dog, ib.rows, D, 128) ||
+      !make_tmap_2d(&tqh, ib.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
+      !make_tmap_2d(&toh, ib.doh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
       !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), D,
                     32, 32))
     return cudaErrorInvalidValue;
@@ -824,8 +818,8 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   for (int h = 0; h < P.n_h; ++h) {
     // padding rows get -LSE log2(e) = -inf, so their P is exactly 0
     e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q),
-                            static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, lse2, rowD,
-                            ib.l2g, ib.dg, -INFINITY, num_sms, st);
+                            static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, ib.qh, ib.doh,
+                            lse2, rowD, ib.l2g, ib.dg, -INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
@@ -839,13 +833,13 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
           static_cast<__nv_bfloat16*>(dq), rowD);
     }
     // the exact D of this head into item order for the dK/dV pass
-    e = launch_gather_items(P, h, pv, nullptr, nullptr, nullptr, nullptr, lse2, rowD, ib.l2g,
-                            ib.dg, -INFINITY, num_sms, st);
+    e = launch_gather_items(P, h, pv, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, lse2,
+                            rowD, ib.l2g, ib.dg, -INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dkdv_blk", st);
       k_bwd_dkdv_blk<D><<<P.Nb * nkt, kThreads, kv_smem<D>(), st>>>(
-          tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
+          tk, tv, tqh, toh, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
           static_cast<__nv_bfloat16*>(dv), make_watch(status));
     }
   }

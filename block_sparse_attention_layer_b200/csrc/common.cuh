@@ -9,7 +9,6 @@
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
-#include <functional>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -171,25 +170,12 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
                                 float scale, uint32_t* sel, vmoba_head_stats* stats, void* ws,
                                 const WsLayout& L, int num_sms, cudaStream_t st,
                                 int by_count = 0, double kcount = 0.0, bool rownorm = false);
-// What the tensor-core score passes (score_tc.cu) need from the selection
-// around them: the search state and histograms, the outputs, and the
-// one-warp digit walks to run after each histogram pass.
-struct SelPassOps {
-  SelState* st;
-  uint32_t* hc;
-  double* hm;
-  uint32_t* sel;
-  float* pool;
-  void* bsplit;
-  int* status;
-  int num_sms;
-  bool pool_only;       // one pass writing S to `pool`, nothing else
-  std::function<cudaError_t(int, cudaStream_t)> scan, tie_scan;
-};
-// bf16 Q: the score passes of a selection (max, three histogram passes with
-// their scans, the tie passes, the bitmap) or, with pool_only, the pool.
-cudaError_t launch_score_passes_tc(const Prob& P, const void* q, const float* blocks,
-                                   float scale, const SelPassOps& ops, cudaStream_t stream);
+// bf16 Q: the score pool S = scale q b^T of every head on the tensor cores
+// (score_tc.cu), written to `pool` with each head's max in st[h].max_key;
+// bsplit receives the bf16 hi / lo split of the block means.
+cudaError_t launch_score_pool_tc(const Prob& P, const void* q, const float* blocks, float scale,
+                                 void* bsplit, float* pool, SelState* st, int* status,
+                                 int num_sms, cudaStream_t stream);
 // The score pool S = scale q b^T of every head into the workspace.
 cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks, float scale,
                               void* ws, const WsLayout& L, int num_sms, cudaStream_t st);

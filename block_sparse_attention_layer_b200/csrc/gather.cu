@@ -4,7 +4,9 @@
 // [128 n, 128 n + 128) of the copy: row r holds the r-th query of the tile,
 // rows past the list end are zero.  The backward kernels (dQ pass, dK/dV
 // pass) then fetch query tiles with plain 2-D TMA instead of scattered
-// loads; the forward gathers its own query rows from Q.  With no row source
+// loads; the forward gathers its own query rows from Q.  Q and dO are
+// written twice: bf16 for the dQ pass and fp16 (exact within fp16's range)
+// for the dK/dV pass, whose MMAs take fp16 operands.  With no row source
 // (a == nullptr) only the per-row values are rewritten.  One warp per item; D / 8
 // lanes x 16 bytes move a row of head_dim D, 8 instructions in flight.
 #include "tc_prims.cuh"
@@ -19,7 +21,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
                const __nv_bfloat16* __restrict__ b, __nv_bfloat16* __restrict__ ag,
-               __nv_bfloat16* __restrict__ bg, const float* __restrict__ fa,
+               __nv_bfloat16* __restrict__ bg, __half* __restrict__ ah, __half* __restrict__ bh,
+               const float* __restrict__ fa,
                const float* __restrict__ fb, float* __restrict__ fag, float* __restrict__ fbg,
                float fa_pad) {
   const uint32_t* col_rows = pv.col_rows + (size_t)h * P.cap;
@@ -51,7 +54,11 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
       for (int u = 0; u < kInFlight; ++u) {
         const size_t dst = (base + r0 + kRpi * u + half) * D;
         reinterpret_cast<uint4*>(ag + dst)[c] = va[u];
-        if (b) reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
+        reinterpret_cast<uint4*>(ah + dst)[c] = tc::bf16x8_to_f16x8(va[u]);
+        if (b) {
+          reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
+          reinterpret_cast<uint4*>(bh + dst)[c] = tc::bf16x8_to_f16x8(vb[u]);
+        }
       }
     }
     if (fa) {
@@ -78,17 +85,18 @@ size_t item_rows_capacity(const Prob& P) {
 
 cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 const __nv_bfloat16* a, const __nv_bfloat16* b,
-                                __nv_bfloat16* ag, __nv_bfloat16* bg, const float* fa,
+                                __nv_bfloat16* ag, __nv_bfloat16* bg, __half* ah, __half* bh,
+                                const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st) {
   {
     VMOBA_TRACE("k_gather_items", st);
     if (P.d == 128)
-      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg,
-                                                       fa_pad);
+      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, ah, bh, fa, fb,
+                                                       fag, fbg, fa_pad);
     else
-      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, fa, fb, fag, fbg,
-                                                      fa_pad);
+      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, ah, bh, fa, fb,
+                                                      fag, fbg, fa_pad);
   }
   count_launches(1);
   return cudaGetLastError();
@@ -101,6 +109,7 @@ namespace vmoba {
 size_t item_bufs_bytes(const Prob& P) {
   const size_t rows = item_rows_capacity(P);
   return 2 * align_up(rows * P.d * sizeof(__nv_bfloat16), 256) +
+         2 * align_up(rows * P.d * sizeof(__half), 256) +
          2 * align_up(rows * sizeof(float), 256);
 }
 

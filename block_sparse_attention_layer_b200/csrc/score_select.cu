@@ -14,13 +14,11 @@
 // Exact ties at the cut are ranked by flat index i*N_b + j (ascending) with
 // three more count-only radix passes that return at once unless needed.
 //
-// bf16 inputs (every workload of the method) run the passes on the tensor
-// cores over a pool recomputed tile by tile (score_tc.cu): init -> split of
-// B -> max -> {hist, scan} x 3 -> {tie, tie_scan} x 3 -> emit -> stats, with
-// no pool in memory.  fp32 inputs (whose 1e-4 output bar the bf16 split of
-// Q could not meet) compute the pool once with fp32 FMAs on the CUDA cores
-// and read it in each pass: init -> score -> {hist, scan} x 3 ->
-// {tie_hist, tie_scan} x 3 -> emit -> stats.
+// The pool is written once -- by the tensor cores for bf16 inputs
+// (score_tc.cu; every workload of the method), with fp32 FMAs on the CUDA
+// cores for fp32 inputs, whose 1e-4 output bar the bf16 split of Q could not
+// meet -- and read by each pass: init -> pool (and max) -> {hist, scan} x 3
+// -> {tie_hist, tie_scan} x 3 -> emit -> stats.
 //
 // The ablation's "topk + global" variant (VMoBA notes, ablation table) runs
 // the same passes with the digit walk counting pairs instead of mass: the
@@ -495,16 +493,9 @@ cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   float* S = ws_ptr<float>(ws, L.scores);
-  if (P.dtype == VMOBA_BF16) {
-    SelPassOps ops{};
-    ops.st = st;
-    ops.pool = S;
-    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
-    ops.status = ws_ptr<int>(ws, L.status);
-    ops.num_sms = num_sms;
-    ops.pool_only = true;
-    return launch_score_passes_tc(P, q, blocks, scale, ops, stream);
-  }
+  if (P.dtype == VMOBA_BF16)
+    return launch_score_pool_tc(P, q, blocks, scale, ws_ptr<void>(ws, L.bsplit), S, st,
+                                ws_ptr<int>(ws, L.status), num_sms, stream);
   e = (P.d == 128) ? launch_score<float, 128>(P, q, blocks, scale, S, st, stream)
                    : launch_score<float, 64>(P, q, blocks, scale, S, st, stream);
   count_launches(1);
@@ -547,14 +538,9 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
     // the tensor cores write the pool (and each head's max) once; the radix
     // passes below read it with many CTAs per SM, whose shared-memory
     // histogram atomics hide each other's latency
-    SelPassOps ops{};
-    ops.st = st;
-    ops.pool = ws_ptr<float>(ws, L.scores);
-    ops.bsplit = ws_ptr<void>(ws, L.bsplit);
-    ops.status = ws_ptr<int>(ws, L.status);
-    ops.num_sms = num_sms;
-    ops.pool_only = true;
-    e = launch_score_passes_tc(P, q, blocks, scale, ops, stream);
+    e = launch_score_pool_tc(P, q, blocks, scale, ws_ptr<void>(ws, L.bsplit),
+                             ws_ptr<float>(ws, L.scores), st, ws_ptr<int>(ws, L.status), num_sms,
+                             stream);
     if (e != cudaSuccess) return e;
   }
   {
