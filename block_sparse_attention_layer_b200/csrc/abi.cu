@@ -94,10 +94,6 @@ ItemBufs item_bufs(const Prob& P, void* ws, const WsLayout& L) {
   ItemBufs b{};
   b.rows = item_rows_capacity(P);
   char* p = ws_ptr<char>(ws, L.items);
-  b.qg = reinterpret_cast<__nv_bfloat16*>(p);
-  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
-  b.dog = reinterpret_cast<__nv_bfloat16*>(p);
-  p += align_up(b.rows * P.d * sizeof(__nv_bfloat16), 256);
   b.qh = reinterpret_cast<__half*>(p);
   p += align_up(b.rows * P.d * sizeof(__half), 256);
   b.doh = reinterpret_cast<__half*>(p);

@@ -15,14 +15,14 @@
 //    all query tiles of block j's list: S^T = K Q^T, dP^T = V dO^T,
 //    P^T and dS^T in TMEM, dV += P^T dO, dK += dS^T Q; dK, dV of the tile's
 //    keys are complete at the end and are written in original key order.
-//    Its MMAs take fp16 operands: dK and dV sum over every query of a
-//    block's list (tens of thousands in the large layers), and with P and
-//    dS rounded to bf16 (8 significant bits) the rounding alone moves
-//    them by more than 2e-2; fp16 (11 bits) keeps it near 1/8 of that.
-//    The K / V tile is converted in shared memory once per CTA and the
-//    query tiles come from fp16 item-ordered copies (exact conversions of
-//    the bf16 inputs within fp16's range, |x| <= 65504; P is in [0, 1] and
-//    dS = P (dP - D) must stay below 65504 too).  Its D_i is the sum of P dP over the row's
+// Both passes take fp16 operands: dK and dV sum over every query of a
+// block's list (tens of thousands in the large layers), and with P and dS
+// rounded to bf16 (8 significant bits) the rounding alone moves them by more
+// than 2e-2; fp16 (11 bits) keeps it near 1/8 of that.  K' and V' are
+// copied to fp16 once per call and the query tiles come from fp16
+// item-ordered copies (exact conversions of the bf16 inputs within fp16's
+// range, |x| <= 65504; P is in [0, 1] and dS = P (dP - D) must stay below
+// 65504 too).  Its D_i is the sum of P dP over the row's
 //    selected keys, accumulated by the dQ pass, not dO_i . O_i from the
 //    forward's output copy: dK sums D's error times P q over every query of
 //    the list, and the output copy carries the forward's bf16 P.
@@ -197,9 +197,9 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idSS = idesc_bf16(128, 128, false, false);
-      const uint32_t idSS_last = idesc_bf16(128, (kc_last + 15) & ~15, false, false);
-      const uint32_t idDQ = idesc_bf16(128, D, false, true);
+      const uint32_t idSS = idesc_f16(128, 128, false, false);
+      const uint32_t idSS_last = idesc_f16(128, (kc_last + 15) & ~15, false, false);
+      const uint32_t idDQ = idesc_f16(128, D, false, true);
       const int ks_last = (kc_last + 15) / 16;
       const uint32_t qb = smem_u32(sQ), ob = smem_u32(sO);
       const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / G + 1 : 0;
@@ -346,8 +346,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                                        Dx2);
             const uint64_t p2 = f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1]));
             const float2 ds = f32x2_split(mul_x2(p2, dd));
-            pk[e >> 1] = pack_bf16x2((full || x < lim) ? ds.x : 0.f,
-                                     (full || x + 1 < lim) ? ds.y : 0.f);
+            pk[e >> 1] = pack_f16x2((full || x < lim) ? ds.x : 0.f,
+                                    (full || x + 1 < lim) ? ds.y : 0.f);
             dacc = fma_x2(p2,
                           f32x2((full || x < lim) ? __uint_as_float(dp[e]) : 0.f,
                                 (full || x + 1 < lim) ? __uint_as_float(dp[e + 1]) : 0.f),
@@ -469,7 +469,7 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq,
 // 64-127 (one key row per thread) and the epilogue (dV / dK).
 // =====================================================================
 struct KvBars {
-  uint64_t kv_full, kv_conv;           // K / V tile landed (bf16) / converted to fp16
+  uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
   uint64_t st_full, dpt_full, p_full, ds_full;
   uint64_t acc_final;
@@ -518,7 +518,6 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    mbar_init(&bars->kv_conv, 64);
     for (int i = 0; i < 2; ++i) { mbar_init(&bars->qd_full[i], 1); mbar_init(&bars->qd_empty[i], 1); }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
@@ -582,7 +581,7 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           mma_ts(tD, tA + packed_col(kk), desc_sw128(bb + kk * 2048, kHalf, 1024), idAcc,
                  (g > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(&bars->kv_conv, 0, wt, abort) &&
+      bool ok = mbar_wait(&bars->kv_full, 0, wt, abort) &&
                 mbar_wait(&bars->qd_full[0], 0, wt, abort);
       if (ok) {
         tc_fence_after();
@@ -617,19 +616,6 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
       }
       if (ok) mma_commit(&bars->acc_final);
-    }
-  } else if (warp == 2 || warp == 3) {
-    // the K / V tile to fp16 in place once it lands (the swizzled layout is a
-    // permutation of 16-byte granules, so converting granule by granule
-    // keeps it), made visible to the tensor core's proxy before its barrier;
-    // the query tiles arrive in fp16 from the item-ordered copies
-    const int x0 = threadIdx.x - 64;
-    bool ok = ng > 0 && __all_sync(0xffffffffu, mbar_wait(&bars->kv_full, 0, wt, abort));
-    if (ok) {
-      uint4* gkv = reinterpret_cast<uint4*>(sK);             // K then V: 2 * kTileB bytes
-      for (int x = x0; x < (int)(2 * kTileB / 16); x += 64) gkv[x] = bf16x8_to_f16x8(gkv[x]);
-      fence_proxy_async();
-      mbar_arrive(&bars->kv_conv);
     }
   } else if (warp >= 4) {
     const int wq = warp & 3, wg = (warp - 4) >> 2;   // lane quarter, query-column group
@@ -770,9 +756,21 @@ k_bwd_dkdv_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
 }  // namespace
 
+namespace {
+// bf16 -> fp16 of a contiguous array, 16 bytes per step (n a multiple of 8)
+__global__ void k_to_f16(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = tc::bf16x8_to_f16x8(__ldg(src + i));
+}
+}  // namespace
+
 size_t bwd_blk_ws_bytes(const Prob& P) {
-  // rowD + lse2 ([n_h][s] fp32 each)
-  return 2 * align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
+  // rowD + lse2 ([n_h][s] fp32 each); for the tensor-core path also fp16
+  // copies of K' and V' ([n_h][s][d] each)
+  size_t b = 2 * align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
+  if (uses_blk_path(P)) b += 2 * align_up(sizeof(__half) * (size_t)P.n_h * P.s * P.d, 256);
+  return b;
 }
 
 namespace {
@@ -782,24 +780,37 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
                     const PairsView& pv, void* part, const ItemBufs& ib, const float* o32,
                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
                     void* ws_bwd, float scale, int* status, int num_sms, cudaStream_t st) {
-  CUtensorMap tk, tv, tq, to, tqh, toh, tpd;
+  CUtensorMap tk, tv, tq, to, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
   float* part_dq = static_cast<float*>(part);
+  // fp16 copies of K' and V' (the backward's MMAs take fp16 operands)
+  const size_t f32_bytes = align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
+  __half* kh = reinterpret_cast<__half*>(static_cast<char*>(ws_bwd) + 2 * f32_bytes);
+  __half* vh = reinterpret_cast<__half*>(
+      reinterpret_cast<char*>(kh) + align_up(sizeof(__half) * (size_t)P.n_h * P.s * D, 256));
   // the dQ pass's per-pair shares of D (two per item row), where the
   // forward kept its (m, l)
   float* part_d = reinterpret_cast<float*>(
       static_cast<char*>(part) + align_up(item_rows_capacity(P) * D * sizeof(float), 256));
-  if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
-      !make_tmap_bf16_2d(&tq, ib.qg, ib.rows, D, 128) ||
-      !make_tmap_bf16_2d(&to, ib.dog, ib.rows, D, 128) ||
-      !make_tmap_2d(&tqh, ib.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
-      !make_tmap_2d(&toh, ib.doh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ib.rows, D, 64, 128) ||
+  const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!make_tmap_2d(&tk, kh, f16, 2, rows, D, 64, 128) ||
+      !make_tmap_2d(&tv, vh, f16, 2, rows, D, 64, 128) ||
+      !make_tmap_2d(&tq, ib.qh, f16, 2, ib.rows, D, 64, 128) ||
+      !make_tmap_2d(&to, ib.doh, f16, 2, ib.rows, D, 64, 128) ||
       !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), D,
                     32, 32))
     return cudaErrorInvalidValue;
   float* rowD = static_cast<float*>(ws_bwd);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws_bwd) +
                                          align_up(sizeof(float) * (size_t)P.n_h * P.s, 256));
+  {
+    VMOBA_TRACE("k_to_f16", st);
+    const size_t n16 = (size_t)P.n_h * P.s * D / 8;
+    k_to_f16<<<num_sms * 8, 256, 0, st>>>(static_cast<const uint4*>(kp),
+                                          reinterpret_cast<uint4*>(kh), n16);
+    k_to_f16<<<num_sms * 8, 256, 0, st>>>(static_cast<const uint4*>(vp),
+                                          reinterpret_cast<uint4*>(vh), n16);
+  }
   const int warps = P.s * P.n_h;
   {
     VMOBA_TRACE("k_bwd_rows", st);
@@ -818,8 +829,8 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   for (int h = 0; h < P.n_h; ++h) {
     // padding rows get -LSE log2(e) = -inf, so their P is exactly 0
     e = launch_gather_items(P, h, pv, static_cast<const __nv_bfloat16*>(q),
-                            static_cast<const __nv_bfloat16*>(dout), ib.qg, ib.dog, ib.qh, ib.doh,
-                            lse2, rowD, ib.l2g, ib.dg, -INFINITY, num_sms, st);
+                            static_cast<const __nv_bfloat16*>(dout), ib.qh, ib.doh, lse2, rowD,
+                            ib.l2g, ib.dg, -INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
@@ -833,17 +844,17 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
           static_cast<__nv_bfloat16*>(dq), rowD);
     }
     // the exact D of this head into item order for the dK/dV pass
-    e = launch_gather_items(P, h, pv, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, lse2,
-                            rowD, ib.l2g, ib.dg, -INFINITY, num_sms, st);
+    e = launch_gather_items(P, h, pv, nullptr, nullptr, nullptr, nullptr, lse2, rowD, ib.l2g,
+                            ib.dg, -INFINITY, num_sms, st);
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dkdv_blk", st);
       k_bwd_dkdv_blk<D><<<P.Nb * nkt, kThreads, kv_smem<D>(), st>>>(
-          tk, tv, tqh, toh, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
+          tk, tv, tq, to, P, h, pv, ib.dg, ib.l2g, sl2, scale, static_cast<__nv_bfloat16*>(dk),
           static_cast<__nv_bfloat16*>(dv), make_watch(status));
     }
   }
-  count_launches(1 + 4 * P.n_h);
+  count_launches(3 + 4 * P.n_h);
   return cudaGetLastError();
 }
 

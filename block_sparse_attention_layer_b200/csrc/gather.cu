@@ -5,8 +5,8 @@
 // rows past the list end are zero.  The backward kernels (dQ pass, dK/dV
 // pass) then fetch query tiles with plain 2-D TMA instead of scattered
 // loads; the forward gathers its own query rows from Q.  Q and dO are
-// written twice: bf16 for the dQ pass and fp16 (exact within fp16's range)
-// for the dK/dV pass, whose MMAs take fp16 operands.  With no row source
+// stored in fp16 (exact within fp16's range), the operand type of the
+// backward's MMAs.  With no row source
 // (a == nullptr) only the per-row values are rewritten.  One warp per item; D / 8
 // lanes x 16 bytes move a row of head_dim D, 8 instructions in flight.
 #include "tc_prims.cuh"
@@ -20,9 +20,8 @@ constexpr int kInFlight = 8;             // warp instructions in flight per batc
 template <int D>
 __global__ void __launch_bounds__(256)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
-               const __nv_bfloat16* __restrict__ b, __nv_bfloat16* __restrict__ ag,
-               __nv_bfloat16* __restrict__ bg, __half* __restrict__ ah, __half* __restrict__ bh,
-               const float* __restrict__ fa,
+               const __nv_bfloat16* __restrict__ b, __half* __restrict__ ah,
+               __half* __restrict__ bh, const float* __restrict__ fa,
                const float* __restrict__ fb, float* __restrict__ fag, float* __restrict__ fbg,
                float fa_pad) {
   const uint32_t* col_rows = pv.col_rows + (size_t)h * P.cap;
@@ -53,12 +52,8 @@ k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
 #pragma unroll
       for (int u = 0; u < kInFlight; ++u) {
         const size_t dst = (base + r0 + kRpi * u + half) * D;
-        reinterpret_cast<uint4*>(ag + dst)[c] = va[u];
         reinterpret_cast<uint4*>(ah + dst)[c] = tc::bf16x8_to_f16x8(va[u]);
-        if (b) {
-          reinterpret_cast<uint4*>(bg + dst)[c] = vb[u];
-          reinterpret_cast<uint4*>(bh + dst)[c] = tc::bf16x8_to_f16x8(vb[u]);
-        }
+        if (b) reinterpret_cast<uint4*>(bh + dst)[c] = tc::bf16x8_to_f16x8(vb[u]);
       }
     }
     if (fa) {
@@ -85,18 +80,17 @@ size_t item_rows_capacity(const Prob& P) {
 
 cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 const __nv_bfloat16* a, const __nv_bfloat16* b,
-                                __nv_bfloat16* ag, __nv_bfloat16* bg, __half* ah, __half* bh,
-                                const float* fa,
+                                __half* ah, __half* bh, const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st) {
   {
     VMOBA_TRACE("k_gather_items", st);
     if (P.d == 128)
-      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, ah, bh, fa, fb,
-                                                       fag, fbg, fa_pad);
+      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
+                                                       fa_pad);
     else
-      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ag, bg, ah, bh, fa, fb,
-                                                      fag, fbg, fa_pad);
+      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
+                                                      fa_pad);
   }
   count_launches(1);
   return cudaGetLastError();
@@ -108,8 +102,7 @@ namespace vmoba {
 
 size_t item_bufs_bytes(const Prob& P) {
   const size_t rows = item_rows_capacity(P);
-  return 2 * align_up(rows * P.d * sizeof(__nv_bfloat16), 256) +
-         2 * align_up(rows * P.d * sizeof(__half), 256) +
+  return 2 * align_up(rows * P.d * sizeof(__half), 256) +
          2 * align_up(rows * sizeof(float), 256);
 }
 

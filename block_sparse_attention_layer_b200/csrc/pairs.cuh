@@ -96,11 +96,9 @@ __device__ __forceinline__ WorkItem decode_item_pair(const PairsView& pv, const 
   return a;
 }
 
-// Item-ordered copies (gather.cu): bf16 rows of Q and dO (dQ pass), the same
-// rows in fp16 (dK/dV pass, whose MMAs take fp16), fp32 -LSE*log2e and D.
+// Item-ordered copies (gather.cu) for the backward passes: fp16 rows of Q and
+// dO (the bf16 inputs converted; their MMAs take fp16), fp32 -LSE*log2e and D.
 struct ItemBufs {
-  __nv_bfloat16* qg;
-  __nv_bfloat16* dog;
   __half* qh;
   __half* doh;
   float* l2g;
@@ -123,8 +121,7 @@ cudaError_t launch_attn_fwd_blk(const Prob& P, const void* q, const void* kp, co
 size_t item_rows_capacity(const Prob& P);
 cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
                                 const __nv_bfloat16* a, const __nv_bfloat16* b,
-                                __nv_bfloat16* ag, __nv_bfloat16* bg, __half* ah, __half* bh,
-                                const float* fa,
+                                __half* ah, __half* bh, const float* fa,
                                 const float* fb, float* fag, float* fbg, float fa_pad,
                                 int num_sms, cudaStream_t st);
 

@@ -120,7 +120,9 @@ size_t vmoba_workspace_size(const vmoba_shape* shape);
  * word (vmoba_get_status); nothing is read or written past the buffers. */
 size_t vmoba_workspace_size_bounded(const vmoba_shape* shape, double max_pair_fraction);
 
-/* Bytes of the extra backward workspace (row terms D = rowsum(dO*O)), or 0. */
+/* Bytes of the extra backward workspace, or 0: the row terms D and -LSE
+ * log2(e) ([n_heads][s] fp32 each) and, for bf16 layers, fp16 copies of K'
+ * and V' (the backward's tensor-core MMAs take fp16 operands). */
 size_t vmoba_bwd_workspace_size(const vmoba_shape* shape);
 
 /* Step 1 (notes, key design 1: "rearrange K in (T H W), B = mean(K')").
