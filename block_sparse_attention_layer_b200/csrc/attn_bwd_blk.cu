@@ -318,13 +318,23 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         tmem_ld32(tmem + b * 128 + lane_off + cb, pr);
         tmem_ld32(tmem + b * 128 + lane_off + cb + 32, pr + 32);
         tmem_ld_wait();
+        if (full) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float2 t = f32x2_split(
-              fma_x2(f32x2(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1])), sl2x2, nl2x2));
-          // columns past the chunk's keys: S is not written there, P = 0
-          pr[e] = __float_as_uint((full || e < lim) ? fast_exp2(t.x) : 0.f);
-          pr[e + 1] = __float_as_uint((full || e + 1 < lim) ? fast_exp2(t.y) : 0.f);
+          for (int e = 0; e < 64; e += 2) {
+            const float2 t = f32x2_split(
+                fma_x2(f32x2(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1])), sl2x2, nl2x2));
+            pr[e] = __float_as_uint(fast_exp2(t.x));
+            pr[e + 1] = __float_as_uint(fast_exp2(t.y));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float2 t = f32x2_split(
+                fma_x2(f32x2(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1])), sl2x2, nl2x2));
+            // columns past the chunk's keys: S is not written there, P = 0
+            pr[e] = __float_as_uint(e < lim ? fast_exp2(t.x) : 0.f);
+            pr[e + 1] = __float_as_uint(e + 1 < lim ? fast_exp2(t.y) : 0.f);
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -338,20 +348,28 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           tmem_ld32(tdP + lane_off + cb + hh * 32, dp);
           tmem_ld_wait();
           uint32_t pk[16];
+          if (full) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int x = hh * 32 + e;
-            // dP past the chunk's keys is stale; P = 0 there must not meet it
-            const uint64_t dd = sub_x2(f32x2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
-                                       Dx2);
-            const uint64_t p2 = f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1]));
-            const float2 ds = f32x2_split(mul_x2(p2, dd));
-            pk[e >> 1] = pack_f16x2((full || x < lim) ? ds.x : 0.f,
-                                    (full || x + 1 < lim) ? ds.y : 0.f);
-            dacc = fma_x2(p2,
-                          f32x2((full || x < lim) ? __uint_as_float(dp[e]) : 0.f,
-                                (full || x + 1 < lim) ? __uint_as_float(dp[e + 1]) : 0.f),
-                          dacc);
+            for (int e = 0; e < 32; e += 2) {
+              const int x = hh * 32 + e;
+              const uint64_t dp2 = f32x2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1]));
+              const uint64_t p2 = f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1]));
+              const float2 ds = f32x2_split(mul_x2(p2, sub_x2(dp2, Dx2)));
+              pk[e >> 1] = pack_f16x2(ds.x, ds.y);
+              dacc = fma_x2(p2, dp2, dacc);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int x = hh * 32 + e;
+              // dP past the chunk's keys is stale; P = 0 there must not meet it
+              const uint64_t dp2 = f32x2(x < lim ? __uint_as_float(dp[e]) : 0.f,
+                                         x + 1 < lim ? __uint_as_float(dp[e + 1]) : 0.f);
+              const uint64_t p2 = f32x2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1]));
+              const float2 ds = f32x2_split(mul_x2(p2, sub_x2(dp2, Dx2)));
+              pk[e >> 1] = pack_f16x2(ds.x, ds.y);
+              dacc = fma_x2(p2, dp2, dacc);
+            }
           }
           // dS into the group's columns [cb + 16 hh, +16): dP columns already read
           tmem_st16(tdP + lane_off + cb + hh * 16, pk);

@@ -437,8 +437,9 @@ k_fwd_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUte
 // Combine the partial (m, l, O / l) of every query's selected blocks:
 // O_i = sum_j 2^(m_j - M) l_j (O / l)_j / sum_j 2^(m_j - M) l_j,
 // LSE_i = (M + log2 sum_j 2^(m_j - M) l_j) ln 2.
-// One warp per query row, D / 32 dims per lane, blocks in ascending order;
-// the partials sit at the pairs' item rows (slot_row).
+// One warp per query row: the two half-warps take alternate blocks (in
+// ascending order, D / 16 dims per lane) and add their sums at the end; the
+// partials sit at the pairs' item rows (slot_row).
 template <int D>
 __global__ void __launch_bounds__(256)
 k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
@@ -461,7 +462,10 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
   for (uint32_t b = 32 + lane; b < cnt; b += 32) M = fmaxf(M, part_ml[__ldg(srow + b)].x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int V = D / 32;                  // dims per lane: V / 2 fp16 pairs
+  // each half-warp reads one pair's row (V fp16 values per lane, one vector
+  // load), so a warp instruction covers two pairs; the halves meet at the end
+  constexpr int V = D / 16;
+  const int hw = lane >> 4, hl = lane & 15;
   float acc[V];
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
@@ -480,37 +484,53 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
     const float my_w = b + lane < cnt ? exp2f(ml.x - M) * ml.y : 0.f;
     const int kn = (int)min(32u, cnt - b);
 #pragma unroll 4
-    for (int k = 0; k < kn; ++k) {
-      const uint32_t row = __shfl_sync(0xffffffffu, my_row, k);
-      const float wl = __shfl_sync(0xffffffffu, my_w, k);
-      Lsum += wl;
-      uint32_t u[V / 2];                     // this lane's V fp16 values, one vector load
-      if constexpr (V == 4) {
-        const uint2 x = reinterpret_cast<const uint2*>(part_o + (size_t)row * D)[lane];
-        u[0] = x.x;
-        u[1] = x.y;
-      } else {
-        u[0] = reinterpret_cast<const uint32_t*>(part_o + (size_t)row * D)[lane];
-      }
+    for (int k = 0; k < kn; k += 2) {
+      const int kk = k + hw;                 // <= kn <= 32
+      const uint32_t row = __shfl_sync(0xffffffffu, my_row, kk & 31);
+      const float w = __shfl_sync(0xffffffffu, my_w, kk & 31);
+      if (kk < kn) {
+        Lsum += w;
+        uint32_t u[V / 2];
+        if constexpr (V == 8) {
+          const uint4 x = reinterpret_cast<const uint4*>(part_o + (size_t)row * D)[hl];
+          u[0] = x.x;
+          u[1] = x.y;
+          u[2] = x.z;
+          u[3] = x.w;
+        } else {
+          const uint2 x = reinterpret_cast<const uint2*>(part_o + (size_t)row * D)[hl];
+          u[0] = x.x;
+          u[1] = x.y;
+        }
 #pragma unroll
-      for (int e = 0; e < V / 2; ++e) {
-        const float2 a = unpack_f16x2(u[e]);
-        acc[2 * e] = fmaf(wl, a.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(wl, a.y, acc[2 * e + 1]);
+        for (int e = 0; e < V / 2; ++e) {
+          const float2 a = unpack_f16x2(u[e]);
+          acc[2 * e] = fmaf(w, a.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(w, a.y, acc[2 * e + 1]);
+        }
       }
     }
   }
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  Lsum += __shfl_xor_sync(0xffffffffu, Lsum, 16);
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   const size_t row = ((size_t)i * P.n_h + h) * D;
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] *= inv;
-  if constexpr (V == 4) {
-    reinterpret_cast<float4*>(o32 + row)[lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    reinterpret_cast<uint2*>(out + row)[lane] =
-        make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-  } else {
-    reinterpret_cast<float2*>(o32 + row)[lane] = make_float2(acc[0], acc[1]);
-    reinterpret_cast<uint32_t*>(out + row)[lane] = pack_bf16x2(acc[0], acc[1]);
+  if (hw == 0) {
+    if constexpr (V == 8) {
+      reinterpret_cast<float4*>(o32 + row)[2 * hl] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      reinterpret_cast<float4*>(o32 + row)[2 * hl + 1] =
+          make_float4(acc[4], acc[5], acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out + row)[hl] =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    } else {
+      reinterpret_cast<float4*>(o32 + row)[hl] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      reinterpret_cast<uint2*>(out + row)[hl] =
+          make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    }
   }
   if (lane == 0)
     lse[(size_t)h * P.s + i] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.6931471805599453f : -INFINITY;

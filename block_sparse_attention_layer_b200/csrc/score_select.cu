@@ -181,13 +181,26 @@ k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t*
   const float* base = S + (size_t)h * pool;
   const size_t beg = (size_t)blockIdx.x * kHistChunk;
   const size_t end = min(beg + (size_t)kHistChunk, pool);
-  for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) {
-    float x = __ldg(base + f);
+  auto add = [&](float x) {
     uint32_t dig;
     if (digit_of<PASS>(f2key(x), prefix, dig)) {
       atomicAdd(&cnt[dig], 1u);
       atomicAdd(&mass[dig], expf(x - m));
     }
+  };
+  if ((pool & 3) == 0) {
+    // 16-byte loads: the head's pool starts 16-byte aligned and beg, end
+    // are multiples of 4
+    const float4* b4 = reinterpret_cast<const float4*>(base);
+    for (size_t f = beg / 4 + threadIdx.x; f < end / 4; f += kHistThreads) {
+      const float4 v = __ldg(b4 + f);
+      add(v.x);
+      add(v.y);
+      add(v.z);
+      add(v.w);
+    }
+  } else {
+    for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) add(__ldg(base + f));
   }
   __syncthreads();
   for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
@@ -396,6 +409,40 @@ k_emit(Prob P, const float* __restrict__ S, const SelState* __restrict__ st,
   const int state = st[h].state;
   const uint32_t cut = st[h].cut_key, idx_cut = st[h].idx_cut;
   const int rows_per_cta = 8 * 4;
+  if ((P.Nb & 3) == 0) {
+    // 16-byte loads (rows start 16-byte aligned): lane l holds blocks
+    // 4l .. 4l+3 of each 128-block span; 8 lanes' nibbles make one word
+    for (int rr = warp; rr < rows_per_cta; rr += 8) {
+      const int i = blockIdx.x * rows_per_cta + rr;
+      if (i >= P.s) break;
+      const float* row = S + ((size_t)h * P.s + i) * P.Nb;
+      for (int j0 = 0; j0 < P.Nb; j0 += 128) {
+        const int j = j0 + 4 * lane;
+        uint32_t nib = 0u;
+        if (j < P.Nb) {
+          if (state == kSel_All) {
+            nib = 0xFu;
+          } else {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
+            const float xs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t key = f2key(xs[e]);
+              const uint32_t idx = (uint32_t)((size_t)i * P.Nb + j + e);
+              if (key > cut || (key == cut && idx <= idx_cut)) nib |= 1u << e;
+            }
+          }
+        }
+        uint32_t word = nib << (4 * (lane & 7));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        const int w = (j0 >> 5) + (lane >> 3);
+        if ((lane & 7) == 0 && w < P.Wb) sel[((size_t)h * P.s + i) * P.Wb + w] = word;
+      }
+    }
+    return;
+  }
   for (int rr = warp; rr < rows_per_cta; rr += 8) {
     const int i = blockIdx.x * rows_per_cta + rr;
     if (i >= P.s) break;
