@@ -81,18 +81,24 @@ __global__ void k_bwd_rows(Prob P, const float* __restrict__ o32,
 }
 
 // =====================================================================
-// dQ pass.  TMEM: S0 [0,128), S1 [128,256), dP [256,384) (then dS), dQ
-// [384,384+D).  Roles: warp 0 TMA (the item's Q and dO tiles from the
+// dQ pass.  Roles: warp 0 TMA (the item's Q and dO tiles from the
 // item-ordered copies, then the block's K, V chunks), warp 1 MMA, warps
 // 4-7 / 8-11 softmax of key columns 0-63 / 64-127 + epilogue (warps 2-3
-// idle).  Per chunk J the softmax forms P(J) from S(J) and frees S, then
-// dS(J) = P (dP - D) once dP(J) is there; the MMA issue order S(J+1),
-// dQ(J) += dS(J) K, dP(J+1) lets S(J+1) run while dS(J) is formed and
-// dP(J+1) while P(J+1) is.
+// idle).  Per chunk J the softmax reads S(J) and frees it, forms P(J), then
+// dS(J) = P (dP - D) once dP(J) is there.  Two TMEM schedules, dQ at
+// [384,384+D) in both:
+//  - long blocks (more than two key chunks): S double-buffered at [0,128),
+//    [128,256), dP (then dS) at [256,384); issue order S(J+1), dQ(J),
+//    dP(J+1): S(J+1) runs while dS(J) is formed, dP(J+1) while P(J+1) is;
+//  - short blocks (DB): S at [0,128), dP double-buffered at [128,256),
+//    [256,384); issue order S(J+1), dP(J+1), dQ(J): chunk J+1's MMAs need
+//    not wait for dQ(J) to take dS(J) out of a shared dP buffer.  With long
+//    blocks this order asks for K(J+2) right after dQ(J) is issued, before
+//    the two-stage K ring can refill, which costs more than it gains.
 // =====================================================================
 struct DqBars {
   uint64_t full_k[2], empty_k[2], full_v[2], empty_v[2];
-  uint64_t s_full[2], s_free[2], dp_full, ds_full;
+  uint64_t s_full[2], s_free[2], dp_full[2], ds_full[2];
   uint64_t qd_full, qd_empty, dq_final, dq_free;
   uint32_t tmem_base;
   int abort;
@@ -105,7 +111,7 @@ constexpr size_t dq_smem() {
 }
 static_assert(dq_smem<128>() <= 232448, "shared memory per CTA");
 
-template <int D>
+template <int D, bool DB>
 __global__ void __launch_bounds__(kThreads, 1)
 k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
@@ -135,9 +141,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       mbar_init(&bars->full_k[i], 1); mbar_init(&bars->empty_k[i], 1);
       mbar_init(&bars->full_v[i], 1); mbar_init(&bars->empty_v[i], 1);
       mbar_init(&bars->s_full[i], 1); mbar_init(&bars->s_free[i], kSoftmaxWarps);
+      mbar_init(&bars->dp_full[i], 1); mbar_init(&bars->ds_full[i], kSoftmaxWarps);
     }
-    mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->ds_full, kSoftmaxWarps);
     mbar_init(&bars->qd_full, 1);
     mbar_init(&bars->qd_empty, 1);
     mbar_init(&bars->dq_final, 1);
@@ -153,7 +158,17 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tdP = tmem + 256, tDQ = tmem + 384;
+  const uint32_t tDQ = tmem + 384;
+  // TMEM column of S(J) and of dP(J), and the barrier slot / phase parity of
+  // chunk J's S and dP barriers, for the two schedules above
+  auto tS = [&](int J) -> uint32_t { return DB ? tmem : tmem + 128 * (uint32_t)(J & 1); };
+  auto tdP = [&](int J) -> uint32_t {
+    return DB ? tmem + 128 + 128 * (uint32_t)(J & 1) : tmem + 256;
+  };
+  auto s_slot = [](int J) { return DB ? 0 : (J & 1); };
+  auto s_par = [](int J) -> uint32_t { return DB ? (J & 1) : ((J >> 1) & 1); };
+  auto d_slot = [](int J) { return DB ? (J & 1) : 0; };
+  auto d_par = [](int J) -> uint32_t { return DB ? ((J >> 1) & 1) : (J & 1); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -205,11 +220,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / G + 1 : 0;
       const int total = my_items * nch;                 // chunks of this CTA
       bool ok = true;
-      // S(J) = Q K^T into S[J & 1]; the chunk's first S of an item waits for its Q / dO
+      // S(J) = Q K^T; the chunk's first S of an item waits for its Q / dO,
+      // every S for the softmax to have read the S it overwrites
       auto issue_s = [&](int J) -> bool {
         const int st = J & 1, c = J % nch, itl = J / nch;
         if (c == 0 && !mbar_wait(&bars->qd_full, itl & 1, wt, abort)) return false;
-        if (J >= 2 && !mbar_wait(&bars->s_free[st], ((J >> 1) - 1) & 1, wt, abort))
+        const int prev = DB ? J - 1 : J - 2;
+        if (prev >= 0 && !mbar_wait(&bars->s_free[s_slot(prev)], s_par(prev), wt, abort))
           return false;
         if (!mbar_wait(&bars->full_k[st], (J >> 1) & 1, wt, abort)) return false;
         tc_fence_after();
@@ -218,13 +235,14 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tmem + st * 128, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
-                 idc, kk > 0 ? 1u : 0u);
+          mma_ss(tS(J), desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idc,
+                 kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->s_full[st]);
+        mma_commit(&bars->s_full[s_slot(J)]);
         return true;
       };
-      // dP(J) = dO V^T; overwrites dS(J-1), whose dQ MMA was issued before
+      // dP(J) = dO V^T; overwrites dS(J-1) (DB: dS(J-2)), whose dQ MMA was
+      // issued before
       auto issue_dp = [&](int J) -> bool {
         const int st = J & 1, c = J % nch;
         if (!mbar_wait(&bars->full_v[st], (J >> 1) & 1, wt, abort)) return false;
@@ -234,25 +252,25 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tdP, desc_sw128(ob + off, 16, 1024), desc_sw128(vb + off, 16, 1024), idc,
+          mma_ss(tdP(J), desc_sw128(ob + off, 16, 1024), desc_sw128(vb + off, 16, 1024), idc,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->empty_v[st]);
-        mma_commit(&bars->dp_full);
+        mma_commit(&bars->dp_full[d_slot(J)]);
         if (c == nch - 1) mma_commit(&bars->qd_empty);  // item's last reader of Q / dO
         return true;
       };
       // dQ += dS(J) K(J); dS packed over the dP columns
       auto issue_dq = [&](int J) -> bool {
         const int st = J & 1, c = J % nch, itl = J / nch;
-        if (!mbar_wait(&bars->ds_full, J & 1, wt, abort)) return false;
+        if (!mbar_wait(&bars->ds_full[d_slot(J)], d_par(J), wt, abort)) return false;
         if (c == 0 && itl > 0 && !mbar_wait(&bars->dq_free, (itl - 1) & 1, wt, abort))
           return false;
         tc_fence_after();
         const uint32_t kb = smem_u32(sK + st * kTileB);
         const int ks = c == nch - 1 ? ks_last : 8;
         for (int kk = 0; kk < ks; ++kk)
-          mma_ts(tDQ, tdP + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
+          mma_ts(tDQ, tdP(J) + packed_col(kk), desc_sw128(kb + kk * 2048, kHalf, 1024), idDQ,
                  (c > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty_k[st]);
         if (c == nch - 1) mma_commit(&bars->dq_final);
@@ -265,7 +283,8 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           // next item: its Q / dO arrive after this item's last dP, so issue dQ first
           ok = issue_dq(J) && issue_s(J + 1) && issue_dp(J + 1);
         } else if (more) {
-          ok = issue_s(J + 1) && issue_dq(J) && issue_dp(J + 1);
+          ok = DB ? (issue_s(J + 1) && issue_dp(J + 1) && issue_dq(J))
+                  : (issue_s(J + 1) && issue_dq(J) && issue_dp(J + 1));
         } else {
           ok = issue_dq(J);
         }
@@ -297,27 +316,30 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       // up and the dK/dV pass uses that sum
       uint64_t dacc = f32x2(0.f, 0.f);
       for (int c = 0; c < nch; ++c, ++J) {
-        const int b = J & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (J >> 1) & 1, wt, abort));
+        const int sb = s_slot(J), db = d_slot(J);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], s_par(J), wt, abort));
         if (!ok) break;
         tc_fence_after();
         const int lim = (c == nch - 1 ? kc_last : kTile) - cb;   // valid columns of this group
         if (lim <= 0) {
           // no key of this chunk in the group's columns: the dQ MMA reads none of them
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->s_free[b]);
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, wt, abort));
+          if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full[db], d_par(J), wt, abort));
           if (!ok) break;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->ds_full);
+          if (lane == 0) mbar_arrive(&bars->ds_full[db]);
           continue;
         }
         const bool full = lim >= 64;
         // P for the group's 64 key columns; rows past the tile's end give P = 0
         uint32_t pr[64];
-        tmem_ld32(tmem + b * 128 + lane_off + cb, pr);
-        tmem_ld32(tmem + b * 128 + lane_off + cb + 32, pr + 32);
+        tmem_ld32(tS(J) + lane_off + cb, pr);
+        tmem_ld32(tS(J) + lane_off + cb + 32, pr + 32);
         tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[sb]);   // S may be overwritten now
         if (full) {
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
@@ -336,16 +358,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             pr[e + 1] = __float_as_uint(e + 1 < lim ? fast_exp2(t.y) : 0.f);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[b]);    // S[b] may be overwritten now
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, J & 1, wt, abort));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full[db], d_par(J), wt, abort));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {                  // 32 dP columns per wait
           uint32_t dp[32];
-          tmem_ld32(tdP + lane_off + cb + hh * 32, dp);
+          tmem_ld32(tdP(J) + lane_off + cb + hh * 32, dp);
           tmem_ld_wait();
           uint32_t pk[16];
           if (full) {
@@ -372,12 +391,12 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
           }
           // dS into the group's columns [cb + 16 hh, +16): dP columns already read
-          tmem_st16(tdP + lane_off + cb + hh * 16, pk);
+          tmem_st16(tdP(J) + lane_off + cb + hh * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->ds_full);
+        if (lane == 0) mbar_arrive(&bars->ds_full[db]);
       }
       if (!ok) break;
       if (n + G < n_items) fetch(n + G, nx_l2, nx_d);
@@ -835,10 +854,15 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
     k_bwd_rows<D><<<(warps + 7) / 8, 256, 0, st>>>(
         P, o32, static_cast<const __nv_bfloat16*>(dout), lse, rowD, lse2);
   }
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_dq_blk<D>,
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_dq_blk<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)dq_smem<D>());
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_bwd_dq_blk<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dq_smem<D>());
+  if (e != cudaSuccess) return e;
+  // blocks of at most two key chunks take the double-buffered dP schedule
+  const bool dq_db = (P.L + kTile - 1) / kTile <= 2;
   e = cudaFuncSetAttribute(k_bwd_dkdv_blk<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kv_smem<D>());
   if (e != cudaSuccess) return e;
@@ -852,8 +876,12 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
     if (e != cudaSuccess) return e;
     {
       VMOBA_TRACE("k_bwd_dq_blk", st);
-      k_bwd_dq_blk<D><<<num_sms, kThreads, dq_smem<D>(), st>>>(
-          tk, tv, tq, to, tpd, P, h, pv, ib.dg, ib.l2g, sl2, part_d, make_watch(status));
+      if (dq_db)
+        k_bwd_dq_blk<D, true><<<num_sms, kThreads, dq_smem<D>(), st>>>(
+            tk, tv, tq, to, tpd, P, h, pv, ib.dg, ib.l2g, sl2, part_d, make_watch(status));
+      else
+        k_bwd_dq_blk<D, false><<<num_sms, kThreads, dq_smem<D>(), st>>>(
+            tk, tv, tq, to, tpd, P, h, pv, ib.dg, ib.l2g, sl2, part_d, make_watch(status));
     }
     {
       VMOBA_TRACE("k_bwd_dq_merge", st);
