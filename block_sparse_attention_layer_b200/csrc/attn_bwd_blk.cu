@@ -407,27 +407,35 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_final, it_local & 1, wt, abort));
       if (!ok) break;
       tc_fence_after();
-      constexpr int kQc = D / 2;                      // dQ columns of each group
-#pragma unroll 1
-      for (int cc = 0; cc < kQc / 32; ++cc) {          // this group's D / 2 dQ columns
-        uint32_t xr[32];
-        tmem_ld32(tDQ + lane_off + kQc * wg + cc * 32, xr);
+      // the partial leaves rounded to fp16 (the merge adds the partials in
+      // fp32): a thread's 64 columns of its row are one 128-byte staging
+      // row, and each warp's 32 rows one asynchronous store; the groups take
+      // columns 0-63 / 64-127 (head_dim 64: group 0 takes all of them)
+      if (D == 128 || wg == 0) {
+        const int c0 = D == 128 ? 64 * wg : 0;
+        uint32_t xr[64];
+        tmem_ld32(tDQ + lane_off + c0, xr);
+        tmem_ld32(tDQ + lane_off + c0 + 32, xr + 32);
         tmem_ld_wait();
         // the staging tile is free once the previous store has read it
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
         // row `lane` into the staging tile in the 128-byte swizzle of the
         // store's tensor map: 16-byte granule g at g ^ (row & 7)
+        uint32_t* stw = reinterpret_cast<uint32_t*>(stg);
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          *reinterpret_cast<float4*>(stg + lane * 32 + ((g ^ (lane & 7)) << 2)) =
-              make_float4(__uint_as_float(xr[4 * g]), __uint_as_float(xr[4 * g + 1]),
-                          __uint_as_float(xr[4 * g + 2]), __uint_as_float(xr[4 * g + 3]));
+        for (int g = 0; g < 8; ++g) {
+          uint4 u;
+          u.x = pack_f16x2(__uint_as_float(xr[8 * g]), __uint_as_float(xr[8 * g + 1]));
+          u.y = pack_f16x2(__uint_as_float(xr[8 * g + 2]), __uint_as_float(xr[8 * g + 3]));
+          u.z = pack_f16x2(__uint_as_float(xr[8 * g + 4]), __uint_as_float(xr[8 * g + 5]));
+          u.w = pack_f16x2(__uint_as_float(xr[8 * g + 6]), __uint_as_float(xr[8 * g + 7]));
+          *reinterpret_cast<uint4*>(stw + lane * 32 + ((g ^ (lane & 7)) << 2)) = u;
+        }
         fence_proxy_async();
         __syncwarp();
-        // the warp's 32 item rows, 32 columns, in one asynchronous store
         if (lane == 0) {
-          tma_store_2d(&tm_pd, stg, kQc * wg + cc * 32, n * kTile + wq * 32);
+          tma_store_2d(&tm_pd, stw, c0, n * kTile + wq * 32);
           bulk_commit();
         }
       }
@@ -445,11 +453,13 @@ k_bwd_dq_blk(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   }
 }
 
-// dQ_i = scale * sum_j partial_ij, blocks in ascending order; one warp per row
-// (D / 32 dims per lane).  The partials sit at the pairs' item rows (slot_row).
+// dQ_i = scale * sum_j partial_ij; one warp per row, the two half-warps take
+// alternate blocks (in ascending order, D / 16 fp16 dims per lane) and add
+// their sums at the end.  The partials sit at the pairs' item rows
+// (slot_row).
 template <int D>
 __global__ void __launch_bounds__(256)
-k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq,
+k_bwd_dq_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_dq,
                const float2* __restrict__ part_d, float scale, __nv_bfloat16* __restrict__ dq,
                float* __restrict__ rowD) {
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -467,26 +477,47 @@ k_bwd_dq_merge(Prob P, int h, PairsView pv, const float* __restrict__ part_dq,
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
   if (lane == 0 && cnt > 0) rowD[(size_t)h * P.s + i] = dsum;
-  __nv_bfloat16* dst = dq + ((size_t)i * P.n_h + h) * D;
-  if constexpr (D == 128) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int V = D / 16;
+  const int hw = lane >> 4, hl = lane & 15;
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
 #pragma unroll 4
-    for (uint32_t k = 0; k < cnt; ++k) {
-      const uint32_t row = __ldg(srow + k);
-      const float4 o = reinterpret_cast<const float4*>(part_dq + (size_t)row * D)[lane];
-      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+  for (uint32_t k = hw; k < cnt; k += 2) {
+    const uint32_t row = __ldg(srow + k);
+    uint32_t u[V / 2];
+    if constexpr (V == 8) {
+      const uint4 x = reinterpret_cast<const uint4*>(part_dq + (size_t)row * D)[hl];
+      u[0] = x.x;
+      u[1] = x.y;
+      u[2] = x.z;
+      u[3] = x.w;
+    } else {
+      const uint2 x = reinterpret_cast<const uint2*>(part_dq + (size_t)row * D)[hl];
+      u[0] = x.x;
+      u[1] = x.y;
     }
-    reinterpret_cast<uint2*>(dst)[lane] = make_uint2(pack_bf16x2(acc.x * scale, acc.y * scale),
-                                                     pack_bf16x2(acc.z * scale, acc.w * scale));
-  } else {
-    float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 4
-    for (uint32_t k = 0; k < cnt; ++k) {
-      const uint32_t row = __ldg(srow + k);
-      const float2 o = reinterpret_cast<const float2*>(part_dq + (size_t)row * D)[lane];
-      acc.x += o.x; acc.y += o.y;
+#pragma unroll
+    for (int e = 0; e < V / 2; ++e) {
+      const float2 a = unpack_f16x2(u[e]);
+      acc[2 * e] += a.x;
+      acc[2 * e + 1] += a.y;
     }
-    reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(acc.x * scale, acc.y * scale);
+  }
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  if (hw == 0) {
+    __nv_bfloat16* dst = dq + ((size_t)i * P.n_h + h) * D;
+    if constexpr (V == 8) {
+      reinterpret_cast<uint4*>(dst)[hl] =
+          make_uint4(pack_bf16x2(acc[0] * scale, acc[1] * scale),
+                     pack_bf16x2(acc[2] * scale, acc[3] * scale),
+                     pack_bf16x2(acc[4] * scale, acc[5] * scale),
+                     pack_bf16x2(acc[6] * scale, acc[7] * scale));
+    } else {
+      reinterpret_cast<uint2*>(dst)[hl] = make_uint2(pack_bf16x2(acc[0] * scale, acc[1] * scale),
+                                                     pack_bf16x2(acc[2] * scale, acc[3] * scale));
+    }
   }
 }
 
@@ -819,7 +850,7 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
                     void* ws_bwd, float scale, int* status, int num_sms, cudaStream_t st) {
   CUtensorMap tk, tv, tq, to, tpd;
   const uint64_t rows = (uint64_t)P.n_h * P.s;
-  float* part_dq = static_cast<float*>(part);
+  __half* part_dq = static_cast<__half*>(part);
   // fp16 copies of K' and V' (the backward's MMAs take fp16 operands)
   const size_t f32_bytes = align_up(sizeof(float) * (size_t)P.n_h * P.s, 256);
   __half* kh = reinterpret_cast<__half*>(static_cast<char*>(ws_bwd) + 2 * f32_bytes);
@@ -828,14 +859,13 @@ cudaError_t bwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   // the dQ pass's per-pair shares of D (two per item row), where the
   // forward kept its (m, l)
   float* part_d = reinterpret_cast<float*>(
-      static_cast<char*>(part) + align_up(item_rows_capacity(P) * D * sizeof(float), 256));
+      static_cast<char*>(part) + align_up(item_rows_capacity(P) * D * sizeof(__half), 256));
   const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (!make_tmap_2d(&tk, kh, f16, 2, rows, D, 64, 128) ||
       !make_tmap_2d(&tv, vh, f16, 2, rows, D, 64, 128) ||
       !make_tmap_2d(&tq, ib.qh, f16, 2, ib.rows, D, 64, 128) ||
       !make_tmap_2d(&to, ib.doh, f16, 2, ib.rows, D, 64, 128) ||
-      !make_tmap_2d(&tpd, part_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, item_rows_capacity(P), D,
-                    32, 32))
+      !make_tmap_2d(&tpd, part_dq, f16, 2, item_rows_capacity(P), D, 64, 32))
     return cudaErrorInvalidValue;
   float* rowD = static_cast<float*>(ws_bwd);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws_bwd) +

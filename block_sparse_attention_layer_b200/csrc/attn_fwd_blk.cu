@@ -540,9 +540,10 @@ k_fwd_merge(Prob P, int h, PairsView pv, const __half* __restrict__ part_o,
 
 size_t blk_partial_bytes(const Prob& P) {
   // one head's partials, one row per work-item row (item_rows_capacity rows):
-  // d fp32 (dQ pass) or d fp16 (forward O / l), then the forward's (m, l)
+  // d fp16 (forward O / l, dQ pass), then the forward's (m, l) or the dQ
+  // pass's two shares of D
   const size_t rows = item_rows_capacity(P);
-  return align_up(rows * P.d * sizeof(float), 256) + align_up(rows * sizeof(float2), 256);
+  return align_up(rows * P.d * sizeof(__half), 256) + align_up(rows * sizeof(float2), 256);
 }
 
 namespace {
@@ -556,7 +557,7 @@ cudaError_t fwd_blk(const Prob& P, const void* q, const void* kp, const void* vp
   const size_t prows = item_rows_capacity(P);
   __half* part_o = static_cast<__half*>(part);    // fp16 O / l, then (m, l) at a fixed offset
   float2* part_ml = reinterpret_cast<float2*>(
-      static_cast<char*>(part) + align_up(prows * D * sizeof(float), 256));
+      static_cast<char*>(part) + align_up(prows * D * sizeof(__half), 256));
   if (!make_tmap_bf16_2d(&tk, kp, rows, D, 128) || !make_tmap_bf16_2d(&tv, vp, rows, D, 128) ||
       !make_tmap_2d(&tpo, part_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, prows, D, 64, 32))
     return cudaErrorInvalidValue;

@@ -223,7 +223,11 @@ int vmoba_attn_fwd(const vmoba_shape* shape, const void* q, const void* k_perm,
  * required), so the bf16 rounding of the stored output does not enter the
  * gradients.  lse from vmoba_attn_fwd; dout [s][n_heads][d].  Writes dq, dk,
  * dv [s][n_heads][d] (dtype, original token order; a key no selected query
- * attends gets zeros).  ws_bwd: vmoba_bwd_workspace_size bytes. */
+ * attends gets zeros).  ws_bwd: vmoba_bwd_workspace_size bytes.
+ * Range: the bf16 / tensor-core path computes on fp16 copies of Q, dO, K'
+ * and V' with fp16 P and dS, and keeps each (query, block) share of dQ (the
+ * block's sum of dS k_n, before the scale) in fp16; values above 65504 in
+ * magnitude are outside its contract.  The fp32 path has no such limit. */
 int vmoba_attn_bwd(const vmoba_shape* shape, const void* q, const void* k_perm,
                    const void* v_perm, const uint32_t* sel_bits, void* ws,
                    size_t ws_bytes, float scale, const float* lse, const void* dout,
