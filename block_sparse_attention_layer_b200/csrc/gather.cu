@@ -6,19 +6,21 @@
 // pass) then fetch query tiles with plain 2-D TMA instead of scattered
 // loads; the forward gathers its own query rows from Q.  Q and dO are
 // stored in fp16 (exact within fp16's range), the operand type of the
-// backward's MMAs.  With no row source
-// (a == nullptr) only the per-row values are rewritten.  One warp per item; D / 8
-// lanes x 16 bytes move a row of head_dim D, 8 instructions in flight.
+// backward's MMAs.  With no row source (a == nullptr) only the per-row
+// values are rewritten.  One warp per item; D / 8 lanes x 16 bytes move a row
+// of head_dim D, 4 instructions in flight per source, at most 64 registers a
+// thread so that four 256-thread CTAs share an SM (8 in flight at 88
+// registers, two CTAs per SM, were 8 % slower on the 3D layers).
 #include "tc_prims.cuh"
 #include "pairs.cuh"
 
 namespace vmoba {
 namespace {
 
-constexpr int kInFlight = 8;             // warp instructions in flight per batch
+constexpr int kInFlight = 4;             // warp instructions in flight per batch
 
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_gather_items(Prob P, int h, PairsView pv, const __nv_bfloat16* __restrict__ a,
                const __nv_bfloat16* __restrict__ b, __half* __restrict__ ah,
                __half* __restrict__ bh, const float* __restrict__ fa,
@@ -86,10 +88,10 @@ cudaError_t launch_gather_items(const Prob& P, int h, const PairsView& pv,
   {
     VMOBA_TRACE("k_gather_items", st);
     if (P.d == 128)
-      k_gather_items<128><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
+      k_gather_items<128><<<num_sms * 8, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
                                                        fa_pad);
     else
-      k_gather_items<64><<<num_sms * 4, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
+      k_gather_items<64><<<num_sms * 8, 256, 0, st>>>(P, h, pv, a, b, ah, bh, fa, fb, fag, fbg,
                                                       fa_pad);
   }
   count_launches(1);
