@@ -25,6 +25,9 @@
 // cut is then the k-th pair of the same ranking; the masses still ride
 // along for the stats (a last-pass bucket holds one score value, so its
 // share of the mass is exact).
+#include <algorithm>
+#include <cmath>
+
 #include "common.cuh"
 #include "tc_prims.cuh"
 
@@ -41,11 +44,11 @@ __device__ __forceinline__ float word_elem<float>(const uint32_t* w, int k) {
   return __uint_as_float(w[k]);
 }
 
-__global__ void k_init(SelState* st, uint32_t* hc, double* hm, int n_h) {
+__global__ void k_init(SelState* st, uint32_t* hc, unsigned long long* hm, int n_h) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_h * kHistBins;
        i += gridDim.x * blockDim.x) {
     hc[i] = 0u;
-    hm[i] = 0.0;
+    hm[i] = 0ull;
   }
   if (blockIdx.x == 0 && threadIdx.x < n_h) {
     SelState s{};
@@ -156,6 +159,17 @@ k_score(Prob P, const E* __restrict__ q, const float* __restrict__ B, float scal
 // ------------------------------------------------------------- histograms
 constexpr int kHistThreads = 256;
 constexpr int kHistChunk = 64 * 1024;   // pool elements per CTA
+// Bucket masses are summed in fixed point, so that their values do not depend
+// on the order in which the atomics land: a CTA adds each element's mass
+// exp(x - max) <= 1 as an integer multiple of 2^-kMassBitsCta (2^16 elements
+// of at most 2^47 each stay below 2^63), in three 16-bit parts with 32-bit
+// shared atomics (faster than fp32 shared atomics, and than 64-bit ones),
+// then adds its bucket totals, rounded to 2^-F (F = 63 - ceil(log2 pool), at
+// most kMassBitsCta), into the head's 64-bit global buckets, which therefore
+// cannot overflow either.  An element's mass is off by at most 2^-48 (about
+// 4e-15 of the head's largest), far below the fp32 rounding of the scores.
+constexpr int kMassBitsCta = 47;
+static_assert(kHistChunk == 1 << (63 - kMassBitsCta), "per-CTA fixed-point range");
 
 template <int PASS>
 __device__ __forceinline__ bool digit_of(uint32_t key, uint32_t prefix, uint32_t& dig) {
@@ -168,12 +182,18 @@ __device__ __forceinline__ bool digit_of(uint32_t key, uint32_t prefix, uint32_t
 template <int PASS>
 __global__ void __launch_bounds__(kHistThreads)
 k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t* __restrict__ hc,
-       double* __restrict__ hm) {
-  __shared__ uint32_t cnt[kHistBins];
-  __shared__ float mass[kHistBins];
+       unsigned long long* __restrict__ hm, int shift) {
+  // the mass in three 16-bit parts, each summed by 32-bit shared atomics
+  // (at most 2^16 elements of at most 2^16 each: no part overflows)
+  __shared__ uint32_t cnt[kHistBins], m0[kHistBins], m1[kHistBins], m2[kHistBins];
   const int h = blockIdx.y;
   if (st[h].state != kSel_Search) return;
-  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) { cnt[b] = 0u; mass[b] = 0.f; }
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
+    cnt[b] = 0u;
+    m0[b] = 0u;
+    m1[b] = 0u;
+    m2[b] = 0u;
+  }
   __syncthreads();
   const float m = key2f(st[h].max_key);
   const uint32_t prefix = st[h].prefix;
@@ -185,7 +205,10 @@ k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t*
     uint32_t dig;
     if (digit_of<PASS>(f2key(x), prefix, dig)) {
       atomicAdd(&cnt[dig], 1u);
-      atomicAdd(&mass[dig], expf(x - m));
+      const unsigned long long v = __float2ull_rn(expf(x - m) * 140737488355328.f);   // 2^47
+      atomicAdd(&m0[dig], (uint32_t)(v & 0xFFFFu));
+      atomicAdd(&m1[dig], (uint32_t)((v >> 16) & 0xFFFFu));
+      atomicAdd(&m2[dig], (uint32_t)(v >> 32));
     }
   };
   if ((pool & 3) == 0) {
@@ -206,7 +229,9 @@ k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t*
   for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
     if (cnt[b]) {
       atomicAdd(&hc[h * kHistBins + b], cnt[b]);
-      atomicAdd(&hm[h * kHistBins + b], (double)mass[b]);
+      const unsigned long long v = (unsigned long long)m0[b] + ((unsigned long long)m1[b] << 16) +
+                                   ((unsigned long long)m2[b] << 32);
+      atomicAdd(&hm[h * kHistBins + b], shift == 0 ? v : (v + (1ull << (shift - 1))) >> shift);
     }
   }
 }
@@ -215,23 +240,26 @@ k_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint32_t*
 // reaches the target, record the bucket and the mass/count strictly above.
 template <int PASS>
 __global__ void __launch_bounds__(32)
-k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __restrict__ hm,
-       float tau, int by_count, double kcount) {
+k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc,
+       unsigned long long* __restrict__ hm, double qinv, float tau, int by_count, double kcount) {
   const int h = blockIdx.x, lane = threadIdx.x;
   SelState& S = st[h];
   if (S.state != kSel_Search) return;
   uint32_t* c = hc + h * kHistBins;
-  double* mm = hm + h * kHistBins;
+  unsigned long long* mi = hm + h * kHistBins;
+  // bucket mass as a double (fixed point, quantum qinv)
+  auto mm = [&](int d) { return (double)mi[d] * qinv; };
   const int nb = (PASS == 2) ? 1024 : 2048;
   const int per = nb / 32;
   // lane l owns digits nb-1-l*per ... nb-per-l*per (descending)
-  double lm = 0.0;
+  unsigned long long li = 0;
   unsigned long long lc = 0;
   for (int k = 0; k < per; ++k) {
     int d = nb - 1 - lane * per - k;
-    lm += mm[d];
+    li += mi[d];
     lc += c[d];
   }
+  const double lm = (double)li * qinv;
   double above = S.mass_above, target = S.target;
   unsigned long long cabove = S.count_above;
   if (PASS == 0) {
@@ -284,12 +312,12 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     for (int k = 0; k < per; ++k) {
       int d = nb - 1 - lane * per - k;
       if (c[d]) {
-        if (reach(acc + mm[d], cacc + c[d])) { chosen = d; break; }
+        if (reach(acc + mm(d), cacc + c[d])) { chosen = d; break; }
         last = d;
         acc_last = acc;
         cacc_last = cacc;
       }
-      acc += mm[d];
+      acc += mm(d);
       cacc += c[d];
     }
     if (chosen < 0) { chosen = last; acc = acc_last; cacc = cacc_last; }
@@ -305,7 +333,7 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     S.count_above = cacc;
     if (PASS == 2) {
       const uint32_t nt = c[chosen];
-      const double e = mm[chosen] / (double)nt;   // one score value: equal shares
+      const double e = mm(chosen) / (double)nt;   // one score value: equal shares
       const double need = by_count ? target - (double)cacc : target - acc;
       const double rr = by_count ? need : ((need > 0.0 && e > 0.0) ? ceil(need / e) : 1.0);
       const uint32_t r = (rr < 1.0) ? 1u : (rr >= (double)nt ? nt : (uint32_t)rr);
@@ -324,7 +352,7 @@ k_scan(Prob P, SelState* __restrict__ st, uint32_t* __restrict__ hc, double* __r
     }
   }
   __syncwarp();
-  for (int d = lane; d < kHistBins; d += 32) { c[d] = 0u; mm[d] = 0.0; }
+  for (int d = lane; d < kHistBins; d += 32) { c[d] = 0u; mi[d] = 0ull; }
 }
 
 // ---- ties at the cut: rank by flat index (count-only radix select) ----
@@ -534,7 +562,7 @@ cudaError_t launch_score_pool(const Prob& P, const void* q, const float* blocks,
   {
     VMOBA_TRACE("k_init", stream);
     k_init<<<64, 256, 0, stream>>>(st, ws_ptr<uint32_t>(ws, L.hist_count),
-                                   ws_ptr<double>(ws, L.hist_mass), P.n_h);
+                                   ws_ptr<unsigned long long>(ws, L.hist_mass), P.n_h);
   }
   count_launches(1);
   cudaError_t e = cudaGetLastError();
@@ -555,7 +583,13 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
                                 int by_count, double kcount, bool rownorm) {
   SelState* st = ws_ptr<SelState>(ws, L.sel_state);
   uint32_t* hc = ws_ptr<uint32_t>(ws, L.hist_count);
-  double* hm = ws_ptr<double>(ws, L.hist_mass);
+  unsigned long long* hm = ws_ptr<unsigned long long>(ws, L.hist_mass);
+  // global fixed-point scale of the bucket masses (see kMassBitsCta)
+  const size_t pool_elems = (size_t)P.s * P.Nb;
+  const int lg = pool_elems <= 1 ? 0 : 64 - __builtin_clzll((unsigned long long)(pool_elems - 1));
+  const int fbits = std::min(kMassBitsCta, 63 - lg);
+  const int shift = kMassBitsCta - fbits;
+  const double qinv = std::ldexp(1.0, -fbits);
 
   {
     VMOBA_TRACE("k_init", stream);
@@ -566,9 +600,9 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
   int launches = 1;
   auto scan = [&](int pass, cudaStream_t s) -> cudaError_t {
     VMOBA_TRACE("k_scan", s);
-    if (pass == 0) k_scan<0><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
-    if (pass == 1) k_scan<1><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
-    if (pass == 2) k_scan<2><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, tau, by_count, kcount);
+    if (pass == 0) k_scan<0><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, qinv, tau, by_count, kcount);
+    if (pass == 1) k_scan<1><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, qinv, tau, by_count, kcount);
+    if (pass == 2) k_scan<2><<<P.n_h, 32, 0, s>>>(P, st, hc, hm, qinv, tau, by_count, kcount);
     ++launches;
     return cudaGetLastError();
   };
@@ -616,9 +650,9 @@ cudaError_t launch_score_select(const Prob& P, const void* q, const float* block
     for (int pass = 0; pass < 3; ++pass) {
       {
         VMOBA_TRACE("k_hist", stream);
-        if (pass == 0) k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-        if (pass == 1) k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
-        if (pass == 2) k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm);
+        if (pass == 0) k_hist<0><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm, shift);
+        if (pass == 1) k_hist<1><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm, shift);
+        if (pass == 2) k_hist<2><<<hgrid, kHistThreads, 0, stream>>>(P, S, st, hc, hm, shift);
       }
       ++launches;
       if ((e = scan(pass, stream)) != cudaSuccess) return e;
