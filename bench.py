@@ -363,6 +363,15 @@ def run_ours(args, rank, world, local):
         if name in flops_per_pair and ms > 0:
             kern[name]["tflops"] = round(flops_per_pair[name] * tot_pairs * K / (ms * 1e-3) / 1e12, 2)
     dom = max(trace, key=lambda n: trace[n][1]) if trace else None
+    # the score pool's GEMM: algorithmic 2 s N_b d FLOPs per head (one product;
+    # the bf16 hi + lo split of B runs it twice) and the fp32 pool it writes
+    if trace.get("k_score_tc", (0, 0.0))[1] > 0:
+        ms = trace["k_score_tc"][1] / K
+        nbs = [V.num_blocks(sh) for sh in shapes]
+        kern["k_score_tc"]["tflops"] = round(
+            sum(2 * s * nb * d * nh for nb in nbs) / (ms * 1e-3) / 1e12, 2)
+        kern["k_score_tc"]["pool_write_GBps"] = round(
+            sum(4 * s * nb * nh for nb in nbs) / (ms * 1e-3) / 1e9, 1)
     part_bytes = sum(metrics.partition_bytes(s, nh, d, 2, V.num_blocks(sh)) for sh in shapes)
     sel_bytes = sum(metrics.select_bytes(s, nh, V.num_blocks(sh)) for sh in shapes)
     achieved = {
