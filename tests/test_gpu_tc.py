@@ -307,3 +307,26 @@ def test_paper_10_48_60_setting(name, mode):
                                                               blk, scale, dout[:, h], j)
             assert out_err(gk[keys, h], dk_ref, "bf16") <= TOL["bf16"]
             assert out_err(gv[keys, h], dv_ref, "bf16") <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_selection_repeatable_on_large_pool(mode):
+    """The selection's bucket masses are integer (fixed-point) sums, so two
+    selections of the same 55296-token layer agree bit for bit on every head
+    (the 3D pool holds 15.9 M pairs per head, where an order-dependent float
+    sum moves the cut by pairs whose mass is at its rounding)."""
+    from synth import torch_latents as TL
+    w = synth.WORKLOADS[4]
+    q, k, v = TL.make_qkv(w.wid, mode, w.T, w.H, w.W, w.n_heads, w.head_dim)
+    sh = LayerShape(w.T, w.H, w.W, w.n_heads, w.head_dim, mode, *w.boxes[mode], "bf16")
+    L = VMoBALayer(sh, max_pair_fraction=0.25)
+    runs = []
+    for _ in range(3):
+        L.select(q, k, v, 0.25)
+        torch.cuda.synchronize()
+        st = L.head_stats()
+        runs.append((L.sel.cpu().numpy().copy(), st["n_selected"].copy(), st["mass"].copy()))
+    for bits, n, m in runs[1:]:
+        assert np.array_equal(bits, runs[0][0])
+        assert np.array_equal(n, runs[0][1])
+        assert np.array_equal(m, runs[0][2])
