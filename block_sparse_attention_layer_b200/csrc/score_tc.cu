@@ -40,7 +40,8 @@ struct Geo {
   static constexpr int kHalves = D / 64;
   static constexpr uint32_t kQ = kHalves * kHalf;           // one 128-query tile
   static constexpr uint32_t kB = 2 * kHalves * kHalf;       // one 128-block chunk, hi + lo
-  static constexpr size_t kSmem = 1024 + 2 * kQ + 2 * kB + 256;
+  static constexpr uint32_t kStage = 8 * 32 * 32 * 4;      // epilogue: 32 x 32 fp32 per warp
+  static constexpr size_t kSmem = 1024 + 2 * kQ + 2 * kB + kStage + 256;
 };
 static_assert(Geo<128>::kSmem <= 232448, "shared memory per CTA");
 
@@ -66,7 +67,8 @@ k_score_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                                       // 2 tiles
   uint8_t* sB = sQ + 2 * G::kQ;                             // 2 chunks
-  PoolBars* bars = reinterpret_cast<PoolBars*>(sB + 2 * G::kB);
+  float* sStage = reinterpret_cast<float*>(sB + 2 * G::kB);  // 8 x 32 x 32 floats
+  PoolBars* bars = reinterpret_cast<PoolBars*>(sB + 2 * G::kB + G::kStage);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,17 +178,19 @@ k_score_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // ------------------------------------------------------------ epilogue
     const int wq = warp & 3, g = (warp - 4) >> 2;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    // N_b a multiple of 4: every row of the pool starts 16-byte aligned and
-    // the valid columns of a 32-column group come in whole fours
-    const bool vec = (P.Nb & 3) == 0;
+    // the warp's 32 rows x 32 columns pass through a staging tile (column e
+    // of row r at r * 32 + (e ^ r): conflict-free by row and by column) and
+    // leave one row per store instruction, 128 contiguous bytes, whatever
+    // N_b's alignment
+    float* stg = sStage + (warp - 4) * 1024;
     float vmax = -INFINITY;
     bool ok = true;
     int A = 0;
     for (int it = 0; it < my_tiles && ok; ++it) {
       const int t = k0 + it * cph;
-      const int i = t * 128 + wq * 32 + lane;                 // this thread's query row
-      const bool row_ok = i < P.s;
-      float* prow = pool + ((size_t)h * P.s + (row_ok ? i : 0)) * P.Nb;
+      const int i0 = t * 128 + wq * 32;                       // the warp's first query row
+      const bool row_ok = i0 + lane < P.s;                     // this thread's row
+      const int nrows = min(32, P.s - i0);
       for (int c = 0; c < nch; ++c, ++A) {
         const int as = A & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_full[as], (A >> 1) & 1, wt, abort));
@@ -199,35 +203,22 @@ k_score_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           tmem_ld32(tmem + as * 128 + lane_off + g * 64, xr);
           if (vc > 32) tmem_ld32(tmem + as * 128 + lane_off + g * 64 + 32, xr + 32);
           tmem_ld_wait();
-          if (row_ok) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              if (32 * u >= vc) break;
-              const int ve = min(32, vc - 32 * u);
-              if (vec) {
-                // the row's (up to) 32 scores in 16-byte stores
-                float4* dst = reinterpret_cast<float4*>(prow + j0 + 32 * u);
+          for (int u = 0; u < 2; ++u) {
+            if (32 * u >= vc) break;
+            const int ve = min(32, vc - 32 * u);
+            __syncwarp();                                     // the last half's reads are done
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                  if (e < ve) {
-                    const float4 v4 = make_float4(__uint_as_float(xr[32 * u + e]) * scale,
-                                                  __uint_as_float(xr[32 * u + e + 1]) * scale,
-                                                  __uint_as_float(xr[32 * u + e + 2]) * scale,
-                                                  __uint_as_float(xr[32 * u + e + 3]) * scale);
-                    dst[e >> 2] = v4;
-                    vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
-                  }
-                }
-              } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  if (e < ve) {
-                    const float x = __uint_as_float(xr[32 * u + e]) * scale;
-                    prow[j0 + 32 * u + e] = x;
-                    vmax = fmaxf(vmax, x);
-                  }
-                }
-              }
+            for (int e = 0; e < 32; ++e) {
+              const float x = __uint_as_float(xr[32 * u + e]) * scale;
+              stg[lane * 32 + (e ^ lane)] = x;
+              if (row_ok && e < ve) vmax = fmaxf(vmax, x);
+            }
+            __syncwarp();
+            float* dst = pool + ((size_t)h * P.s + i0) * P.Nb + j0 + 32 * u + lane;
+            if (lane < ve) {
+#pragma unroll 4
+              for (int r = 0; r < nrows; ++r) dst[(size_t)r * P.Nb] = stg[r * 32 + (lane ^ r)];
             }
           }
         }
