@@ -429,6 +429,55 @@ k_tie_scan(SelState* __restrict__ st, uint32_t* __restrict__ hc) {
 
 // ------------------------------------------------------------------ emit
 // One warp per (row, 32-block word): bit j set iff pair (i, j) is selected.
+// Vector form of the bitmap pass for N_b a multiple of V (every row starts
+// 4 V-byte aligned): lane l holds blocks V l .. V l + V - 1 of each 32 V-block
+// span, and 32 / V lanes' V-bit groups make one 32-bit word.
+template <int V>
+__device__ __forceinline__ void emit_rows_vec(const Prob& P, const float* __restrict__ S,
+                                              uint32_t* __restrict__ sel, int h, int warp,
+                                              int lane, int state, uint32_t cut, uint32_t idx_cut,
+                                              int rows_per_cta) {
+  constexpr int kLpw = 32 / V;                        // lanes per bitmap word
+  for (int rr = warp; rr < rows_per_cta; rr += 8) {
+    const int i = blockIdx.x * rows_per_cta + rr;
+    if (i >= P.s) break;
+    const float* row = S + ((size_t)h * P.s + i) * P.Nb;
+    for (int j0 = 0; j0 < P.Nb; j0 += 32 * V) {
+      const int j = j0 + V * lane;
+      uint32_t bits = 0u;
+      if (j < P.Nb) {
+        if (state == kSel_All) {
+          bits = (1u << V) - 1u;
+        } else {
+          float xs[V];
+          if constexpr (V == 4) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
+            xs[0] = v.x;
+            xs[1] = v.y;
+            xs[2] = v.z;
+            xs[3] = v.w;
+          } else {
+            const float2 v = __ldg(reinterpret_cast<const float2*>(row + j));
+            xs[0] = v.x;
+            xs[1] = v.y;
+          }
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            const uint32_t key = f2key(xs[e]);
+            const uint32_t idx = (uint32_t)((size_t)i * P.Nb + j + e);
+            if (key > cut || (key == cut && idx <= idx_cut)) bits |= 1u << e;
+          }
+        }
+      }
+      uint32_t word = bits << (V * (lane & (kLpw - 1)));
+#pragma unroll
+      for (int o = 1; o < kLpw; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+      const int w = (j0 >> 5) + lane / kLpw;
+      if ((lane & (kLpw - 1)) == 0 && w < P.Wb) sel[((size_t)h * P.s + i) * P.Wb + w] = word;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256)
 k_emit(Prob P, const float* __restrict__ S, const SelState* __restrict__ st,
        uint32_t* __restrict__ sel) {
@@ -437,38 +486,11 @@ k_emit(Prob P, const float* __restrict__ S, const SelState* __restrict__ st,
   const int state = st[h].state;
   const uint32_t cut = st[h].cut_key, idx_cut = st[h].idx_cut;
   const int rows_per_cta = 8 * 4;
-  if ((P.Nb & 3) == 0) {
-    // 16-byte loads (rows start 16-byte aligned): lane l holds blocks
-    // 4l .. 4l+3 of each 128-block span; 8 lanes' nibbles make one word
-    for (int rr = warp; rr < rows_per_cta; rr += 8) {
-      const int i = blockIdx.x * rows_per_cta + rr;
-      if (i >= P.s) break;
-      const float* row = S + ((size_t)h * P.s + i) * P.Nb;
-      for (int j0 = 0; j0 < P.Nb; j0 += 128) {
-        const int j = j0 + 4 * lane;
-        uint32_t nib = 0u;
-        if (j < P.Nb) {
-          if (state == kSel_All) {
-            nib = 0xFu;
-          } else {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
-            const float xs[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t key = f2key(xs[e]);
-              const uint32_t idx = (uint32_t)((size_t)i * P.Nb + j + e);
-              if (key > cut || (key == cut && idx <= idx_cut)) nib |= 1u << e;
-            }
-          }
-        }
-        uint32_t word = nib << (4 * (lane & 7));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        const int w = (j0 >> 5) + (lane >> 3);
-        if ((lane & 7) == 0 && w < P.Wb) sel[((size_t)h * P.s + i) * P.Wb + w] = word;
-      }
-    }
+  if ((P.Nb & 1) == 0) {
+    if ((P.Nb & 3) == 0)
+      emit_rows_vec<4>(P, S, sel, h, warp, lane, state, cut, idx_cut, rows_per_cta);
+    else
+      emit_rows_vec<2>(P, S, sel, h, warp, lane, state, cut, idx_cut, rows_per_cta);
     return;
   }
   for (int rr = warp; rr < rows_per_cta; rr += 8) {
