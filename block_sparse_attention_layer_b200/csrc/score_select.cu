@@ -369,10 +369,23 @@ k_tie_hist(Prob P, const float* __restrict__ S, SelState* __restrict__ st, uint3
   const float* base = S + (size_t)h * pool;
   const size_t beg = (size_t)blockIdx.x * kHistChunk;
   const size_t end = min(beg + (size_t)kHistChunk, pool);
-  for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) {
-    if (f2key(__ldg(base + f)) != cut) continue;
-    uint32_t idx = (uint32_t)f, dig;
-    if (digit_of<TP>(idx, prefix, dig)) atomicAdd(&cnt[dig], 1u);
+  auto add = [&](float x, size_t f) {
+    if (f2key(x) != cut) return;
+    uint32_t dig;
+    if (digit_of<TP>((uint32_t)f, prefix, dig)) atomicAdd(&cnt[dig], 1u);
+  };
+  if ((pool & 3) == 0) {
+    // 16-byte loads, as in the mass histogram
+    const float4* b4 = reinterpret_cast<const float4*>(base);
+    for (size_t f = beg / 4 + threadIdx.x; f < end / 4; f += kHistThreads) {
+      const float4 v = __ldg(b4 + f);
+      add(v.x, 4 * f);
+      add(v.y, 4 * f + 1);
+      add(v.z, 4 * f + 2);
+      add(v.w, 4 * f + 3);
+    }
+  } else {
+    for (size_t f = beg + threadIdx.x; f < end; f += kHistThreads) add(__ldg(base + f), f);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < kHistBins; b += kHistThreads)
