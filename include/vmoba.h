@@ -205,7 +205,7 @@ int vmoba_build_plan(const vmoba_shape* shape, const uint32_t* sel_bits,
  * vmoba_partition; sel_bits the bitmap the plan was built from.  Writes
  * out [s][n_heads][d] (dtype) and lse [n_heads][s] fp32 (natural log), and
  * keeps an fp32 copy of O in the workspace for vmoba_attn_bwd.
- * Range: the bf16 / head_dim 128 path keeps each (query, block) partial
+ * Range: the bf16 (tensor-core) path keeps each (query, block) partial
  * result as O/l in fp16 (a convex combination of V rows, so |O/l| <= max|V|);
  * inputs with |V| above 65504, the largest finite fp16, are outside its
  * contract (their partials overflow to inf).  The fp32 path has no such
